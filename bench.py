@@ -1,0 +1,375 @@
+#!/usr/bin/env python
+"""Store-h decode attention throughput on B200: cached positions per second.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one full decode step of the workload: for every loop iteration,
+append the new token's h row (quantised) and run store-h attention with the
+per-iteration safety check, for every lane.  Inputs are synthetic and seeded.
+Timing: CUDA events on the launching stream, W untimed warm-up steps, K timed
+steps bracketed by a barrier and a device synchronize, max over ranks.
+Each rank (N > 1) runs its own independent batch (weak scaling, no collective
+on the data path).  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "store-h decode attention cached positions/s on 1 B200; % of roofline"
+UNIT = "cached positions/s"
+DEFAULT_WORKLOAD = "int4_2b"
+DTYPE_OF_FMT = {0: "fp16", 1: "int8", 2: "int4"}
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the CPU-baseline sample")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+# ----------------------------------------------------------------------------- shared helpers
+def workload_for_rank(name, rank):
+    from synth.workloads import get_workload
+    import dataclasses
+    w = get_workload(name)
+    if rank:
+        w = dataclasses.replace(w, seed=w.seed + 1000 * rank)   # an independent batch per rank
+    return w
+
+
+def row_bytes(w):
+    return {0: 2 * w.d, 1: w.d + 4, 2: w.d // 2 + 2 * (w.d // 64)}[w.fmt]
+
+
+def workload_config(w, n_gpus, extra=None):
+    cfg = {"workload": w.name, "d_model": w.d, "n_heads": w.H, "head_dim": w.hd, "n_pre": w.n_pre,
+           "L_max": w.L_max, "h_format": DTYPE_OF_FMT[w.fmt], "batch_per_gpu": w.B,
+           "ctx_per_lane": (w.ctx[0] if len(set(w.ctx)) == 1 else "U[1024,8192] seeded"),
+           "loops_per_lane": (w.loops[0] if len(set(w.loops)) == 1 else "16x4,16x16,16x32"),
+           "global_batch": w.B * n_gpus, "parallelism": f"lanes x{n_gpus} (independent batches)",
+           "cache_inputs_vs_l2": "cache read per step > 126 MB L2 (no flush needed)"}
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+class OracleSample:
+    """A bounded sample of the workload for the CPU oracle: whole (lane, iteration)
+    decodes, each with its lane's resident cache prepared once (not timed)."""
+
+    def __init__(self, w):
+        self.w = w
+        self.pairs = [(it, b) for it in range(w.L_max) for b in range(w.B) if it < w.loops[b]]
+        self.prepared = []
+        self.W = [w.weight(k) for k in "qkv"]
+
+    def _prepare(self, i):
+        import oracle
+        w = self.w
+        it, b = self.pairs[i % len(self.pairs)]
+        layer = w.n_pre + it
+        cache = oracle.OracleCache(w.fmt, w.d, w.n_pre, w.L_max)
+        cache.append(layer, 0, 0, w.h_rows(layer, b, 0, w.ctx[b]))
+        return it, b, cache, w.h_new(it)[b:b + 1], w.residual(it)[b:b + 1]
+
+    def decode(self, i):
+        """Time the oracle as it stands on pair i: append, explicit K/V rebuild, softmax, norm check."""
+        import numpy as np
+        import oracle
+        while len(self.prepared) <= i:
+            self.prepared.append(self._prepare(len(self.prepared)))
+        it, b, cache, hn, res = self.prepared[i]
+        w = self.w
+        t0 = time.perf_counter()
+        oracle.decode_iteration(cache, it, [w.loops[b]], [w.ctx[b]], hn, *self.W, w.H, w.hd, res, w.threshold,
+                                np.zeros(1, np.uint8), np.full(1, -1, np.int32))
+        return w.ctx[b], time.perf_counter() - t0
+
+    def run(self, budget_s, max_pairs=None):
+        """Decode pairs 0, 1, ... until the budget is spent; returns (positions/s, s, description)."""
+        pos, spent, n = 0, 0.0, 0
+        while n == 0 or (spent < budget_s and (max_pairs is None or n < max_pairs)):
+            p, t = self.decode(n)
+            pos, spent, n = pos + p, spent + t, n + 1
+        desc = (f"{n} (lane, iteration) decodes of {self.w.name} by the FP64 oracle (append + explicit K/V "
+                f"rebuild + softmax + norm check), {pos} cached positions, {spent:.2f} s")
+        return pos / spent, spent, desc
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    src = os.path.join(ROOT, "store_kv_attention_b200", "csrc")
+    for fn in sorted(os.listdir(src)):
+        if fn.endswith((".cu", ".cuh")):
+            with open(os.path.join(src, fn), "rb") as f:
+                h.update(fn.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload):
+    """DRAM bytes per launch of the streaming kernel from a committed ncu summary, if it
+    was taken on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "stream_kernel_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    e = rec.get(workload)
+    if not e or e.get("source_sha") != kernel_source_sha():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    QUERY = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        import torch
+        ident = None
+        try:
+            ident = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+        except Exception:
+            pass
+        self.cmd = ["nvidia-smi", "--query-gpu=" + self.QUERY, "--format=csv,noheader,nounits", "-lms", "100"]
+        if ident:
+            self.cmd += ["-i", ident]
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in getattr(self, "lines", []):
+            f = [x.strip() for x in line.split(",")]
+            try:
+                sm.append(float(f[0]))
+                mx = float(f[1])
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, f[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    w = workload_for_rank(args.workload, 0)
+    sample = OracleSample(w)
+    # a step = the same bounded sample of the workload (2 lane-iteration decodes)
+    for _ in range(args.warmup):
+        sample.run(0.0, max_pairs=2)
+    t, pos = 0.0, 0.0
+    desc = ""
+    for _ in range(args.steps):
+        v, s, desc = sample.run(float("inf"), max_pairs=2)
+        t += s
+        pos += v * s
+    value = pos / t
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * t / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded)", "config": workload_config(w, args.gpus),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                             "sample": "per step: " + desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import store_kv_attention_b200 as tl
+    from synth.device import DeviceWorkload
+
+    torch.cuda.set_device(local_rank)
+    w = workload_for_rank(args.workload, rank)
+    dw = DeviceWorkload(w, device=f"cuda:{local_rank}")
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        dw.step()
+    torch.cuda.synchronize()
+    if tl.poll_status(dw.cache) != tl.TL_OK:
+        raise RuntimeError("device status after warm-up: " + tl.lib.tl_last_error_message().decode())
+
+    K = args.steps
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clocks:
+        with tl.ProfileHook(K * w.L_max) as prof:
+            barrier()
+            torch.cuda.synchronize()
+            start.record(stream)
+            for _ in range(K):
+                dw.step()
+            end.record(stream)
+            torch.cuda.synchronize()
+            barrier()
+    ms = start.elapsed_time(end)
+    t = torch.tensor([ms], dtype=torch.float64, device=f"cuda:{local_rank}")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    pos_step = w.cached_positions_per_step()
+    value = world * K * pos_step / (ms_max / 1000.0)
+
+    # dominant kernel (context streaming): algorithmic bytes per launch / CUDA-event duration
+    kms = prof.stream_kernel_ms()
+    rb = row_bytes(w)
+    bytes_per_launch = [sum((w.ctx[b] + 1) * rb for b in range(w.B) if it < w.loops[b]) for it in range(w.L_max)]
+    total_bytes = sum(bytes_per_launch[i % w.L_max] for i in range(len(kms)))
+    achieved_gbs = total_bytes / (sum(kms) / 1000.0) / 1e9
+    peak, peak_kind = load_peaks()
+    traffic = recorded_traffic(w.name)
+    roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": peak, "unit": "GB/s",
+                "frac": achieved_gbs / peak, "traffic": traffic, "peak_source": peak_kind,
+                "kernel": "stream (context streaming: dequant, scores, softmax, p.h)",
+                "algorithmic_bytes_per_launch": statistics.mean(bytes_per_launch),
+                "avg_launch_ms": statistics.mean(kms)}
+    step_bytes = sum(bytes_per_launch) + 3 * 2 * w.d * w.d
+    step_roofline_ms = step_bytes / (peak * 1e9) * 1e3
+
+    # end to end through the public API: pinned host inputs in, results out, every step
+    h_new_host = dw.h_new.cpu().pin_memory()
+    res_host = dw.residual.cpu().pin_memory()
+    out_host = torch.empty(dw.out.shape, dtype=torch.float32).pin_memory()
+    flags_host = torch.empty(w.B, dtype=torch.uint8).pin_memory()
+    first_host = torch.empty(w.B, dtype=torch.int32).pin_memory()
+    h2d = h_new_host.numel() * 2 + res_host.numel() * 4
+    d2h = out_host.numel() * 4 + w.B + w.B * 4
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        dw.h_new.copy_(h_new_host, non_blocking=True)
+        dw.residual.copy_(res_host, non_blocking=True)
+        dw.reset_flags()
+        dw.step()
+        out_host.copy_(dw.out, non_blocking=True)
+        flags_host.copy_(dw.flags, non_blocking=True)
+        first_host.copy_(dw.first, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    t2 = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=f"cuda:{local_rank}")
+    if world > 1:
+        dist.all_reduce(t2, op=dist.ReduceOp.MAX)
+    e2e_value = world * K * pos_step / (float(t2.item()) / 1000.0)
+
+    if rank != 0:
+        return
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        v, s, desc = OracleSample(w).run(args.cpu_seconds)
+        cpu = {"value": v, "unit": UNIT, "cores": blas_threads(), "kind": "oracle", "sample": desc}
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": DTYPE_OF_FMT[w.fmt] + "-h codes, fp16 tensor operands, fp32 accumulate",
+            "data": "synthetic (seeded generator: SplitMix64 + Box-Muller)",
+            "config": workload_config(w, world, {"cached_positions_per_step_per_gpu": pos_step,
+                                                 "step_roofline_ms_hbm": step_roofline_ms,
+                                                 "step_frac_of_hbm_roofline": step_roofline_ms / (ms_max / K)}),
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": prof.launches,
+            "clocks": clocks.summary()}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        if args.impl == "ours":
+            torch.cuda.set_device(local_rank)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        else:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=300))
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,235 @@
+/*
+ * tl_storeh.h — C ABI of the store-h decode-attention library (libtlstoreh.so).
+ *
+ * The method (TinyLoop documentation pages):
+ *   - Store-h KV cache: the cache keeps the pre-QKV LayerNorm output h of every
+ *     (layer, token) instead of K and V; attention rebuilds K = W_k h and
+ *     V = W_v h with the loop block's shared weights.
+ *     [Novel Contributions, "Novel Mechanism: Store-h KV Cache";
+ *      Architecture-Exclusive Features, "Store-h KV cache"]
+ *   - Storage modes FP16-h, INT8-h, INT4-h [same section, mode table].
+ *   - Variable-L cache of n_pre + L_max layers; loop iteration i uses layer
+ *     n_pre + i; a call with loop count L reads only the first n_pre + L layers.
+ *     [Architecture-Exclusive Features, "Variable-L KV cache"]
+ *   - L-aware batching: every lane of one batch runs its own loop count.
+ *     [Architecture-Exclusive Features, "L-aware batching"]
+ *   - Per-iteration safety check on the L2 norm of the FP32 residual.
+ *     [Novel Contributions, "Novel: Per-Iteration Safety Check"]
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers to memory the caller allocated
+ *     and owns; the library never allocates, frees or retains them, and keeps
+ *     no state between calls.
+ *   - Work is enqueued asynchronously on `stream` (NULL = legacy default stream);
+ *     a return of TL_OK means "validated and launched", not "finished".
+ *   - Arguments are validated on the host before anything is launched; a
+ *     non-TL_OK return means nothing was enqueued, except TL_ERR_CUDA, which
+ *     reports a failed launch.  tl_last_error_message() gives details.
+ *   - fp16 data are IEEE binary16 passed as `const void*`; weights are fp16
+ *     row-major [out = d_model][in = d_model] (K = W_k h means
+ *     K[r] = sum_c W_k[r][c] h[c]); head j owns rows j*head_dim .. (j+1)*head_dim-1.
+ *   - Per-lane values read from device arrays (loops, ctx_len, start_pos) are
+ *     range-checked on the device: an out-of-range lane is skipped (no output
+ *     written, flags untouched) and TL_ERR_DEVICE_RANGE is recorded in the
+ *     workspace status word (see tl_storeh_poll_status).  Device kernels never
+ *     trap; every wait inside a kernel is bounded and records
+ *     TL_ERR_DEVICE_TIMEOUT instead of hanging.
+ */
+#ifndef TL_STOREH_H
+#define TL_STOREH_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define TL_STOREH_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define TL_API __attribute__((visibility("default")))
+#else
+#define TL_API
+#endif
+
+/* Same type as cudaStream_t (CUDA runtime) and CUstream (driver API). */
+typedef struct CUstream_st* tl_stream_t;
+
+typedef enum {
+  TL_OK = 0,
+  TL_ERR_INVALID_ARG = 1,    /* NULL pointer, negative count, bad enum value */
+  TL_ERR_SHAPE = 2,          /* d_model != n_heads * head_dim, or a size that breaks a layout rule */
+  TL_ERR_CAPACITY = 3,       /* n_lanes > max_lanes, layer/iter outside the cache, workspace too small */
+  TL_ERR_UNSUPPORTED = 4,    /* a shape the kernels are not built for (see tl_storeh_desc) */
+  TL_ERR_CUDA = 5,           /* a CUDA runtime call or launch failed */
+  TL_ERR_DEVICE_TIMEOUT = 6, /* a bounded wait inside a kernel gave up (recorded on the device) */
+  TL_ERR_DEVICE_RANGE = 7    /* a per-lane device value was out of range; that lane was skipped */
+} tl_status;
+
+/* How a cached h row is stored. */
+typedef enum {
+  TL_H_FP16 = 0,       /* d fp16 values: 2*d bytes, no scale */
+  TL_H_INT8_TOKEN = 1, /* d int8 codes + one fp32 scale per row:
+                          scale = amax/127 (fp32 IEEE division),
+                          code = clamp(rne(x / scale), -127, 127) */
+  TL_H_INT4_G64 = 2    /* d/2 bytes of int4 codes + one fp16 scale per group of 64 along d:
+                          scale = fp16_rne(amax_g / 7.0f),
+                          code = clamp(rne(x / (float)scale), -7, 7);
+                          byte j of a group = (code[2j] & 0xF) | (code[2j+1] & 0xF) << 4 */
+} tl_h_format;
+
+/*
+ * Shape of one store-h cache.  Supported: head_dim in {64, 128};
+ * d_model = n_heads * head_dim with d_model a multiple of 256 and at most 4096;
+ * n_heads <= 16; 1 <= max_ctx <= 65536 counts every position including the newest token.
+ */
+typedef struct {
+  int32_t d_model;
+  int32_t n_heads;
+  int32_t head_dim;
+  int32_t n_pre;     /* unique layers before the loop block */
+  int32_t L_max;     /* loop iterations the cache is sized for */
+  int32_t max_lanes; /* batch lanes the cache is sized for */
+  int32_t max_ctx;   /* positions per (layer, lane) */
+  int32_t fmt;       /* tl_h_format */
+} tl_storeh_desc;
+
+/*
+ * Device memory of one cache, allocated by the caller with the sizes from
+ * tl_storeh_cache_bytes.  Layout, row-major:
+ *   codes [n_pre + L_max][max_lanes][max_ctx][row_code_bytes]
+ *   scales[n_pre + L_max][max_lanes][max_ctx][row_scales]   (NULL for TL_H_FP16)
+ * row_code_bytes = 2d (FP16), d (INT8), d/2 (INT4);
+ * row_scales = 0 (FP16), 1 fp32 (INT8), d/64 fp16 (INT4).
+ * Both base addresses must be 256-byte aligned.
+ */
+typedef struct {
+  void* codes;
+  void* scales;
+} tl_storeh_cache;
+
+/* Bytes the caller must allocate for the cache described by `desc`.
+ * Errors: TL_ERR_INVALID_ARG (NULL), TL_ERR_SHAPE / TL_ERR_UNSUPPORTED (desc). */
+TL_API tl_status tl_storeh_cache_bytes(const tl_storeh_desc* desc, size_t* codes_bytes, size_t* scales_bytes);
+
+/* Bytes of device workspace tl_storeh_attn_decode needs for up to `n_lanes`
+ * lanes (256-byte aligned, contents need no initialisation, must not be shared
+ * by two calls in flight at once). */
+TL_API tl_status tl_storeh_workspace_bytes(const tl_storeh_desc* desc, int32_t n_lanes, size_t* bytes);
+
+/*
+ * Quantise fp16 h rows and write them into cache layer `layer`
+ * [Architecture-Exclusive Features, "Store-h KV cache" — the write side;
+ *  "Variable-L KV cache" — layer n_pre+i is filled by loop iteration i].
+ *
+ *   h_rows     device fp16 [n_lanes][n_rows][d_model]
+ *   start_pos  device int32 [n_lanes]: row r of lane b goes to position start_pos[b] + r
+ *   row_count  device int32 [n_lanes] or NULL: lane b writes rows r < row_count[b]
+ *              (NULL: all n_rows)
+ *   loops      device int32 [n_lanes] or NULL: lane b is skipped when
+ *              layer >= n_pre + loops[b] (NULL: no lane is skipped)
+ * Cache lane index = b.  Rows whose position falls outside [0, max_ctx) are not
+ * written.  Codes and scales are bit-exact with the definitions in tl_h_format.
+ * Errors: TL_ERR_INVALID_ARG, TL_ERR_CAPACITY (n_lanes > max_lanes, layer outside
+ * [0, n_pre + L_max)), TL_ERR_SHAPE, TL_ERR_UNSUPPORTED, TL_ERR_CUDA.
+ */
+TL_API tl_status tl_storeh_append(const tl_storeh_desc* desc, tl_storeh_cache cache, int32_t layer,
+                           const void* h_rows, int32_t n_lanes, int32_t n_rows,
+                           const int32_t* start_pos, const int32_t* row_count,
+                           const int32_t* loops, tl_stream_t stream);
+
+/*
+ * One loop iteration `iter` of store-h decode attention for a batch of lanes
+ * [Novel Contributions, "Novel Mechanism: Store-h KV Cache"; Architecture-
+ * Exclusive Features, "Store-h KV cache", "Variable-L KV cache", "L-aware
+ * batching"].  For every lane b with iter < loops[b]:
+ *   rows c = 0 .. ctx_len[b] of cache layer n_pre + iter are dequantised
+ *   (row ctx_len[b] is the new token, already appended by tl_storeh_append);
+ *   q = W_q h_new[b]; K_c = W_k h_c; V_c = W_v h_c; per head j:
+ *   s_c = q_j . K_cj / sqrt(head_dim), p = softmax(s), out[b][j] = sum_c p_c V_cj.
+ * The kernels use the algebraically equal absorbed form (q_j^T W_k[j] applied
+ * to h, then W_v[j] applied to sum_c p_c h_c).  Lanes with iter >= loops[b]
+ * are left untouched (their out rows are not written).
+ *
+ *   loops, ctx_len  device int32 [n_lanes]; 0 <= ctx_len[b] < max_ctx, loops[b] <= L_max
+ *   h_new           device fp16 [n_lanes][d_model]: the new token's h (unquantised), for q
+ *   W_q, W_k, W_v   device fp16 [d_model][d_model] (may be rows of one stacked [3d][d] buffer)
+ *   out             device fp32 [n_lanes][n_heads][head_dim]
+ *   residual        device fp32 [n_lanes][d_model] or NULL.  When given, the
+ *                   per-iteration safety check of tl_residual_norm_check runs
+ *                   in the same enqueue, with `threshold`, `abort_flags`,
+ *                   `first_abort_iter` and `norms_out` as described there.
+ *   workspace       device scratch of at least tl_storeh_workspace_bytes(desc, n_lanes)
+ * Errors: TL_ERR_INVALID_ARG, TL_ERR_CAPACITY, TL_ERR_SHAPE, TL_ERR_UNSUPPORTED,
+ * TL_ERR_CUDA; device-side conditions via tl_storeh_poll_status.
+ */
+TL_API tl_status tl_storeh_attn_decode(const tl_storeh_desc* desc, tl_storeh_cache cache, int32_t iter,
+                                const int32_t* loops, const int32_t* ctx_len, const void* h_new,
+                                const void* W_q, const void* W_k, const void* W_v, float* out,
+                                const float* residual, float threshold, uint8_t* abort_flags,
+                                int32_t* first_abort_iter, float* norms_out, void* workspace,
+                                size_t workspace_bytes, int32_t n_lanes, tl_stream_t stream);
+
+/*
+ * Per-iteration safety check [Novel Contributions, "Novel: Per-Iteration
+ * Safety Check"; Architecture-Exclusive Features, "Per-iteration safety check"].
+ * For every lane b with iter < loops[b] (all lanes when loops is NULL):
+ *   n2 = sum_k residual[b][k]^2 accumulated in FP64 (each term exact);
+ *   if n2 > threshold^2 (strict): abort_flags[b] = 1 and, if the flag was 0,
+ *   first_abort_iter[b] = iter.  Flags are sticky (never cleared here).
+ *   norms_out[b] = sqrt(n2) as fp32 when norms_out is not NULL.
+ * Lanes with iter >= loops[b] are left untouched.
+ *   residual          device fp32 [n_lanes][d]
+ *   abort_flags       device uint8 [n_lanes], caller-initialised (0 = running)
+ *   first_abort_iter  device int32 [n_lanes], caller-initialised (e.g. -1)
+ * Errors: TL_ERR_INVALID_ARG, TL_ERR_CUDA.
+ */
+TL_API tl_status tl_residual_norm_check(const float* residual, int32_t n_lanes, int32_t d, float threshold,
+                                 int32_t iter, const int32_t* loops, uint8_t* abort_flags,
+                                 int32_t* first_abort_iter, float* norms_out, tl_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the status word that kernels
+ * of tl_storeh_attn_decode record in `workspace`.  Returns TL_OK,
+ * TL_ERR_DEVICE_TIMEOUT (a bounded device wait gave up), TL_ERR_DEVICE_RANGE
+ * (a lane's loops/ctx_len was out of range and the lane was skipped) or
+ * TL_ERR_CUDA.  The status word starts at the beginning of the workspace;
+ * a freshly allocated workspace must be cleared once with this call (or
+ * zero-filled) before its first use.
+ */
+TL_API tl_status tl_storeh_poll_status(void* workspace, size_t workspace_bytes, tl_stream_t stream);
+
+/*
+ * Measurement hook (optional).  While a tl_profile is installed on the calling
+ * thread, every tl_storeh_* call made from that thread counts the kernels it
+ * launches in `launches`, and records begin_events[k] / end_events[k]
+ * (cudaEvent_t handles created by the caller) on the call's stream right before
+ * and right after each launch of the context-streaming kernel of
+ * tl_storeh_attn_decode, for k = recorded++ while recorded < capacity.
+ * Pass NULL to uninstall.  The struct must outlive its installation.
+ */
+typedef struct {
+  void** begin_events;
+  void** end_events;
+  int32_t capacity;
+  int32_t recorded;
+  int64_t launches;
+} tl_profile;
+
+TL_API tl_status tl_set_profile(tl_profile* profile);
+
+/* Static description of a status code. */
+TL_API const char* tl_status_string(tl_status status);
+
+/* Details of the most recent non-TL_OK return on the calling thread. */
+TL_API const char* tl_last_error_message(void);
+
+/* TL_STOREH_ABI_VERSION of the loaded library. */
+TL_API int32_t tl_storeh_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TL_STOREH_H */

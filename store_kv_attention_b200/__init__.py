@@ -1,0 +1,229 @@
+"""Python binding of libtlstoreh.so, the store-h decode-attention library (sm_100a).
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels.  PyTorch supplies device memory and streams.  There is no CPU
+fallback: the first call fails loudly when the library is missing.
+
+The same names as the C ABI in ``include/tl_storeh.h``:
+``cache_bytes``, ``workspace_bytes``, ``append``, ``attn_decode``,
+``residual_norm_check``, ``poll_status``.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+from typing import Optional
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtlstoreh.so")
+
+TL_OK = 0
+TL_ERR_INVALID_ARG = 1
+TL_ERR_SHAPE = 2
+TL_ERR_CAPACITY = 3
+TL_ERR_UNSUPPORTED = 4
+TL_ERR_CUDA = 5
+TL_ERR_DEVICE_TIMEOUT = 6
+TL_ERR_DEVICE_RANGE = 7
+
+TL_H_FP16 = 0
+TL_H_INT8_TOKEN = 1
+TL_H_INT4_G64 = 2
+
+# every symbol include/tl_storeh.h declares
+EXPORTS = ["tl_storeh_cache_bytes", "tl_storeh_workspace_bytes", "tl_storeh_append", "tl_storeh_attn_decode",
+           "tl_residual_norm_check", "tl_storeh_poll_status", "tl_status_string", "tl_last_error_message",
+           "tl_storeh_abi_version", "tl_set_profile"]
+
+
+class TLError(RuntimeError):
+    def __init__(self, status: int, fn: str, msg: str):
+        super().__init__(f"{fn} -> {status}: {msg}")
+        self.status = status
+
+
+class Desc(ctypes.Structure):
+    _fields_ = [("d_model", ctypes.c_int32), ("n_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("n_pre", ctypes.c_int32), ("L_max", ctypes.c_int32), ("max_lanes", ctypes.c_int32),
+                ("max_ctx", ctypes.c_int32), ("fmt", ctypes.c_int32)]
+
+
+class Profile(ctypes.Structure):
+    _fields_ = [("begin_events", ctypes.POINTER(ctypes.c_void_p)), ("end_events", ctypes.POINTER(ctypes.c_void_p)),
+                ("capacity", ctypes.c_int32), ("recorded", ctypes.c_int32), ("launches", ctypes.c_int64)]
+
+
+class Cache(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
+
+
+_lib_handle = None
+
+
+def _load():
+    """Load libtlstoreh.so once (raises when it is missing: there is no fallback)."""
+    global _lib_handle
+    if _lib_handle is not None:
+        return _lib_handle
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m store_kv_attention_b200.build_lib` "
+                          "(there is no CPU fallback)")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, f32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+    P = ctypes.POINTER
+    L.tl_storeh_cache_bytes.argtypes = [P(Desc), P(sz), P(sz)]
+    L.tl_storeh_workspace_bytes.argtypes = [P(Desc), i32, P(sz)]
+    L.tl_storeh_append.argtypes = [P(Desc), Cache, i32, vp, i32, i32, vp, vp, vp, vp]
+    L.tl_storeh_attn_decode.argtypes = [P(Desc), Cache, i32, vp, vp, vp, vp, vp, vp, vp, vp, f32, vp, vp, vp, vp,
+                                        sz, i32, vp]
+    L.tl_residual_norm_check.argtypes = [vp, i32, i32, f32, i32, vp, vp, vp, vp, vp]
+    L.tl_storeh_poll_status.argtypes = [vp, sz, vp]
+    for f in ("tl_storeh_cache_bytes", "tl_storeh_workspace_bytes", "tl_storeh_append", "tl_storeh_attn_decode",
+              "tl_residual_norm_check", "tl_storeh_poll_status"):
+        getattr(L, f).restype = ctypes.c_int
+    L.tl_status_string.argtypes = [ctypes.c_int]
+    L.tl_status_string.restype = ctypes.c_char_p
+    L.tl_last_error_message.argtypes = []
+    L.tl_last_error_message.restype = ctypes.c_char_p
+    L.tl_storeh_abi_version.restype = ctypes.c_int32
+    L.tl_set_profile.argtypes = [P(Profile)]
+    L.tl_set_profile.restype = ctypes.c_int
+    _lib_handle = L
+    return L
+
+
+def __getattr__(name):
+    if name == "lib":
+        return _load()
+    raise AttributeError(name)
+
+
+def _check(st: int, fn: str) -> None:
+    if st != TL_OK:
+        raise TLError(st, fn, _load().tl_last_error_message().decode())
+
+
+def _ptr(t) -> Optional[int]:
+    """Device pointer of a tensor (None -> NULL)."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+@dataclasses.dataclass
+class StoreHDesc:
+    d_model: int
+    n_heads: int
+    head_dim: int
+    n_pre: int
+    L_max: int
+    max_lanes: int
+    max_ctx: int
+    fmt: int
+
+    def c(self) -> Desc:
+        return Desc(self.d_model, self.n_heads, self.head_dim, self.n_pre, self.L_max, self.max_lanes,
+                    self.max_ctx, self.fmt)
+
+
+def cache_bytes(desc: StoreHDesc):
+    cb, sb = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(_load().tl_storeh_cache_bytes(ctypes.byref(desc.c()), ctypes.byref(cb), ctypes.byref(sb)),
+           "tl_storeh_cache_bytes")
+    return cb.value, sb.value
+
+
+def workspace_bytes(desc: StoreHDesc, n_lanes: int) -> int:
+    b = ctypes.c_size_t()
+    _check(_load().tl_storeh_workspace_bytes(ctypes.byref(desc.c()), n_lanes, ctypes.byref(b)),
+           "tl_storeh_workspace_bytes")
+    return b.value
+
+
+class StoreHCache:
+    """Device buffers of one cache (torch uint8 tensors) plus a decode workspace."""
+
+    def __init__(self, desc: StoreHDesc, device="cuda", n_lanes: Optional[int] = None):
+        import torch
+        self.desc = desc
+        cb, sb = cache_bytes(desc)
+        self.codes = torch.empty(cb, dtype=torch.uint8, device=device)
+        self.scales = torch.empty(max(sb, 256), dtype=torch.uint8, device=device) if sb else None
+        n = n_lanes or desc.max_lanes
+        self.ws_bytes = workspace_bytes(desc, n)
+        self.workspace = torch.zeros(self.ws_bytes, dtype=torch.uint8, device=device)
+
+    def c(self) -> Cache:
+        return Cache(self.codes.data_ptr(), self.scales.data_ptr() if self.scales is not None else None)
+
+
+def append(cache: StoreHCache, layer: int, h_rows, start_pos, row_count=None, loops=None, stream=None) -> None:
+    """h_rows: fp16 [n_lanes, n_rows, d] (device); start_pos/row_count/loops int32 [n_lanes] (device)."""
+    n_lanes, n_rows = int(h_rows.shape[0]), int(h_rows.shape[1])
+    _check(_load().tl_storeh_append(ctypes.byref(cache.desc.c()), cache.c(), layer, _ptr(h_rows), n_lanes, n_rows,
+                                _ptr(start_pos), _ptr(row_count), _ptr(loops), _stream(stream)), "tl_storeh_append")
+
+
+def attn_decode(cache: StoreHCache, it: int, loops, ctx_len, h_new, W_q, W_k, W_v, out,
+                residual=None, threshold: float = 0.0, abort_flags=None, first_abort_iter=None,
+                norms_out=None, stream=None) -> None:
+    n_lanes = int(h_new.shape[0])
+    _check(_load().tl_storeh_attn_decode(ctypes.byref(cache.desc.c()), cache.c(), it, _ptr(loops), _ptr(ctx_len),
+                                     _ptr(h_new), _ptr(W_q), _ptr(W_k), _ptr(W_v), _ptr(out), _ptr(residual),
+                                     float(threshold), _ptr(abort_flags), _ptr(first_abort_iter), _ptr(norms_out),
+                                     cache.workspace.data_ptr(), cache.ws_bytes, n_lanes, _stream(stream)),
+           "tl_storeh_attn_decode")
+
+
+def residual_norm_check(residual, threshold: float, it: int, loops, abort_flags, first_abort_iter,
+                        norms_out=None, stream=None) -> None:
+    n_lanes, d = int(residual.shape[0]), int(residual.shape[1])
+    _check(_load().tl_residual_norm_check(_ptr(residual), n_lanes, d, float(threshold), it, _ptr(loops),
+                                      _ptr(abort_flags), _ptr(first_abort_iter), _ptr(norms_out), _stream(stream)),
+           "tl_residual_norm_check")
+
+
+def poll_status(cache: StoreHCache, stream=None) -> int:
+    """Synchronise and return (and clear) the device status of the cache's workspace."""
+    return _load().tl_storeh_poll_status(cache.workspace.data_ptr(), cache.ws_bytes, _stream(stream))
+
+
+class ProfileHook:
+    """Context manager: counts the library's kernel launches on this thread and
+    brackets every context-streaming kernel launch with CUDA events."""
+
+    def __init__(self, capacity: int):
+        import torch
+        self.events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                       for _ in range(capacity)]
+        self._b = (ctypes.c_void_p * capacity)(*[e[0].cuda_event for e in self.events])
+        self._e = (ctypes.c_void_p * capacity)(*[e[1].cuda_event for e in self.events])
+        self.p = Profile(self._b, self._e, capacity, 0, 0)
+
+    def __enter__(self):
+        _check(_load().tl_set_profile(ctypes.byref(self.p)), "tl_set_profile")
+        return self
+
+    def __exit__(self, *exc):
+        _load().tl_set_profile(None)
+        return False
+
+    @property
+    def launches(self) -> int:
+        return int(self.p.launches)
+
+    def stream_kernel_ms(self):
+        """Durations (ms) of the bracketed streaming-kernel launches (call after a synchronize)."""
+        return [b.elapsed_time(e) for b, e in self.events[: self.p.recorded]]

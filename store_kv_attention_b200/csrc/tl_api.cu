@@ -1,0 +1,219 @@
+// C ABI of libtlstoreh.so: host-side validation and kernel launches.
+// The operations are defined in include/tl_storeh.h.
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "tl_internal.cuh"
+
+namespace {
+
+thread_local char g_msg[512] = "";
+
+tl_status fail(tl_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof g_msg, fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+tl_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(TL_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+// Validates a cache descriptor and converts it to the internal shape.
+tl_status check_desc(const tl_storeh_desc* d, tl::Shape* s) {
+  if (!d) return fail(TL_ERR_INVALID_ARG, "desc is NULL");
+  if (d->fmt < TL_H_FP16 || d->fmt > TL_H_INT4_G64) return fail(TL_ERR_INVALID_ARG, "fmt %d is not a tl_h_format", d->fmt);
+  if (d->d_model <= 0 || d->n_heads <= 0 || d->head_dim <= 0 || d->n_pre < 0 || d->L_max <= 0 ||
+      d->max_lanes <= 0 || d->max_ctx <= 0)
+    return fail(TL_ERR_INVALID_ARG, "desc has a non-positive size");
+  if ((int64_t)d->n_heads * d->head_dim != d->d_model)
+    return fail(TL_ERR_SHAPE, "d_model %d != n_heads %d * head_dim %d", d->d_model, d->n_heads, d->head_dim);
+  if (d->head_dim != 64 && d->head_dim != 128) return fail(TL_ERR_UNSUPPORTED, "head_dim %d not in {64, 128}", d->head_dim);
+  if (d->d_model % 256 != 0 || d->d_model > 4096)
+    return fail(TL_ERR_UNSUPPORTED, "d_model %d must be a multiple of 256 and at most 4096", d->d_model);
+  if (d->n_heads > tl::kMaxHeads) return fail(TL_ERR_UNSUPPORTED, "n_heads %d > %d", d->n_heads, tl::kMaxHeads);
+  if (d->max_ctx > tl::kMaxCtx) return fail(TL_ERR_UNSUPPORTED, "max_ctx %d > %d", d->max_ctx, tl::kMaxCtx);
+  if ((int64_t)(d->n_pre + d->L_max) * d->max_lanes * d->max_ctx > ((int64_t)1 << 40))
+    return fail(TL_ERR_CAPACITY, "cache has too many rows");
+  *s = tl::Shape{d->d_model, d->n_heads, d->head_dim, d->n_pre, d->L_max, d->max_lanes, d->max_ctx, d->fmt};
+  return TL_OK;
+}
+
+tl_status check_cache(const tl::Shape& s, const tl_storeh_cache& c) {
+  if (!c.codes) return fail(TL_ERR_INVALID_ARG, "cache.codes is NULL");
+  if (s.fmt != TL_H_FP16 && !c.scales) return fail(TL_ERR_INVALID_ARG, "cache.scales is NULL");
+  if (!aligned(c.codes, 256) || (c.scales && !aligned(c.scales, 256)))
+    return fail(TL_ERR_INVALID_ARG, "cache buffers must be 256-byte aligned");
+  return TL_OK;
+}
+
+}  // namespace
+
+namespace tl {
+
+tl_profile*& current_profile() {
+  thread_local tl_profile* p = nullptr;
+  return p;
+}
+
+void profile_stream_begin(cudaStream_t st) {
+  tl_profile* p = current_profile();
+  if (p && p->recorded < p->capacity) cudaEventRecord((cudaEvent_t)p->begin_events[p->recorded], st);
+}
+
+void profile_stream_end(cudaStream_t st) {
+  tl_profile* p = current_profile();
+  if (p && p->recorded < p->capacity) cudaEventRecord((cudaEvent_t)p->end_events[p->recorded++], st);
+}
+
+}  // namespace tl
+
+extern "C" {
+
+tl_status tl_set_profile(tl_profile* profile) {
+  if (profile && profile->capacity > 0 && (!profile->begin_events || !profile->end_events))
+    return fail(TL_ERR_INVALID_ARG, "profile events are NULL");
+  tl::current_profile() = profile;
+  return TL_OK;
+}
+
+int32_t tl_storeh_abi_version(void) { return TL_STOREH_ABI_VERSION; }
+
+const char* tl_last_error_message(void) { return g_msg; }
+
+const char* tl_status_string(tl_status st) {
+  switch (st) {
+    case TL_OK: return "TL_OK";
+    case TL_ERR_INVALID_ARG: return "TL_ERR_INVALID_ARG: a NULL pointer, negative count or bad enum value";
+    case TL_ERR_SHAPE: return "TL_ERR_SHAPE: inconsistent sizes";
+    case TL_ERR_CAPACITY: return "TL_ERR_CAPACITY: request exceeds the cache or workspace";
+    case TL_ERR_UNSUPPORTED: return "TL_ERR_UNSUPPORTED: shape not supported by the kernels";
+    case TL_ERR_CUDA: return "TL_ERR_CUDA: a CUDA call failed";
+    case TL_ERR_DEVICE_TIMEOUT: return "TL_ERR_DEVICE_TIMEOUT: a bounded device wait gave up";
+    case TL_ERR_DEVICE_RANGE: return "TL_ERR_DEVICE_RANGE: a per-lane device value was out of range";
+  }
+  return "unknown tl_status";
+}
+
+tl_status tl_storeh_cache_bytes(const tl_storeh_desc* desc, size_t* codes_bytes, size_t* scales_bytes) {
+  tl::Shape s;
+  tl_status st = check_desc(desc, &s);
+  if (st != TL_OK) return st;
+  if (!codes_bytes || !scales_bytes) return fail(TL_ERR_INVALID_ARG, "output pointer is NULL");
+  *codes_bytes = s.rows_total() * s.row_code_bytes();
+  *scales_bytes = s.rows_total() * s.row_scales() * s.scale_bytes();
+  return TL_OK;
+}
+
+tl_status tl_storeh_workspace_bytes(const tl_storeh_desc* desc, int32_t n_lanes, size_t* bytes) {
+  tl::Shape s;
+  tl_status st = check_desc(desc, &s);
+  if (st != TL_OK) return st;
+  if (!bytes) return fail(TL_ERR_INVALID_ARG, "bytes is NULL");
+  if (n_lanes <= 0) return fail(TL_ERR_INVALID_ARG, "n_lanes %d <= 0", n_lanes);
+  if (n_lanes > s.max_lanes) return fail(TL_ERR_CAPACITY, "n_lanes %d > max_lanes %d", n_lanes, s.max_lanes);
+  *bytes = tl::workspace_layout(s, n_lanes).total;
+  return TL_OK;
+}
+
+tl_status tl_storeh_append(const tl_storeh_desc* desc, tl_storeh_cache cache, int32_t layer,
+                           const void* h_rows, int32_t n_lanes, int32_t n_rows,
+                           const int32_t* start_pos, const int32_t* row_count,
+                           const int32_t* loops, tl_stream_t stream) {
+  tl::Shape s;
+  tl_status st = check_desc(desc, &s);
+  if (st != TL_OK) return st;
+  if ((st = check_cache(s, cache)) != TL_OK) return st;
+  if (!h_rows || !start_pos) return fail(TL_ERR_INVALID_ARG, "h_rows / start_pos is NULL");
+  if (!aligned(h_rows, 16)) return fail(TL_ERR_INVALID_ARG, "h_rows must be 16-byte aligned");
+  if (n_lanes <= 0 || n_rows < 0) return fail(TL_ERR_INVALID_ARG, "n_lanes %d / n_rows %d", n_lanes, n_rows);
+  if (n_lanes > s.max_lanes) return fail(TL_ERR_CAPACITY, "n_lanes %d > max_lanes %d", n_lanes, s.max_lanes);
+  if (layer < 0 || layer >= s.layers()) return fail(TL_ERR_CAPACITY, "layer %d outside [0, %d)", layer, s.layers());
+  if (n_rows == 0) return TL_OK;
+  cudaError_t e = tl::launch_append(s, cache.codes, cache.scales, layer, (const __half*)h_rows, n_lanes, n_rows,
+                                    start_pos, row_count, loops, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "tl_storeh_append launch");
+  return TL_OK;
+}
+
+tl_status tl_residual_norm_check(const float* residual, int32_t n_lanes, int32_t d, float threshold,
+                                 int32_t iter, const int32_t* loops, uint8_t* abort_flags,
+                                 int32_t* first_abort_iter, float* norms_out, tl_stream_t stream) {
+  if (!residual || !abort_flags || !first_abort_iter)
+    return fail(TL_ERR_INVALID_ARG, "residual / abort_flags / first_abort_iter is NULL");
+  if (n_lanes <= 0 || d <= 0 || iter < 0) return fail(TL_ERR_INVALID_ARG, "n_lanes %d, d %d, iter %d", n_lanes, d, iter);
+  if (!(threshold >= 0.0f)) return fail(TL_ERR_INVALID_ARG, "threshold must be a non-negative number");
+  cudaError_t e = tl::launch_norm_check(residual, n_lanes, d, threshold, iter, loops, nullptr, 0, 0, abort_flags,
+                                        first_abort_iter, norms_out, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "tl_residual_norm_check launch");
+  return TL_OK;
+}
+
+tl_status tl_storeh_attn_decode(const tl_storeh_desc* desc, tl_storeh_cache cache, int32_t iter,
+                                const int32_t* loops, const int32_t* ctx_len, const void* h_new,
+                                const void* W_q, const void* W_k, const void* W_v, float* out,
+                                const float* residual, float threshold, uint8_t* abort_flags,
+                                int32_t* first_abort_iter, float* norms_out, void* workspace,
+                                size_t workspace_bytes, int32_t n_lanes, tl_stream_t stream) {
+  tl::Shape s;
+  tl_status st = check_desc(desc, &s);
+  if (st != TL_OK) return st;
+  if ((st = check_cache(s, cache)) != TL_OK) return st;
+  if (!loops || !ctx_len || !h_new || !W_q || !W_k || !W_v || !out || !workspace)
+    return fail(TL_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (!aligned(h_new, 16) || !aligned(W_q, 16) || !aligned(W_k, 16) || !aligned(W_v, 16) || !aligned(out, 16))
+    return fail(TL_ERR_INVALID_ARG, "h_new, W_q, W_k, W_v and out must be 16-byte aligned");
+  if (!aligned(workspace, 256)) return fail(TL_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (n_lanes <= 0) return fail(TL_ERR_INVALID_ARG, "n_lanes %d <= 0", n_lanes);
+  if (n_lanes > s.max_lanes) return fail(TL_ERR_CAPACITY, "n_lanes %d > max_lanes %d", n_lanes, s.max_lanes);
+  if (iter < 0 || iter >= s.L_max) return fail(TL_ERR_CAPACITY, "iter %d outside [0, L_max=%d)", iter, s.L_max);
+  if (residual && (!abort_flags || !first_abort_iter))
+    return fail(TL_ERR_INVALID_ARG, "residual given without abort_flags / first_abort_iter");
+  if (residual && !(threshold >= 0.0f)) return fail(TL_ERR_INVALID_ARG, "threshold must be a non-negative number");
+  tl::Workspace wl = tl::workspace_layout(s, n_lanes);
+  if (workspace_bytes < wl.total)
+    return fail(TL_ERR_CAPACITY, "workspace %zu bytes < %zu needed", workspace_bytes, wl.total);
+
+  tl::DecodeArgs a{s, cache.codes, cache.scales, iter, loops, ctx_len, (const __half*)h_new,
+                   (const __half*)W_q, (const __half*)W_k, (const __half*)W_v, out, n_lanes,
+                   (uint8_t*)workspace, wl};
+  cudaStream_t cs = (cudaStream_t)stream;
+  cudaError_t e = tl::launch_prologue(a, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "decode prologue launch");
+  tl::profile_stream_begin(cs);
+  e = tl::launch_stream(a, cs);
+  tl::profile_stream_end(cs);
+  if (e != cudaSuccess) return cuda_fail(e, "decode stream launch");
+  e = tl::launch_epilogue(a, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "decode epilogue launch");
+  if (residual) {
+    e = tl::launch_norm_check(residual, n_lanes, s.d, threshold, iter, loops, ctx_len, s.max_ctx, s.L_max,
+                              abort_flags, first_abort_iter, norms_out, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "decode norm check launch");
+  }
+  return TL_OK;
+}
+
+tl_status tl_storeh_poll_status(void* workspace, size_t workspace_bytes, tl_stream_t stream) {
+  if (!workspace || workspace_bytes < 256) return fail(TL_ERR_INVALID_ARG, "workspace is NULL or too small");
+  cudaStream_t cs = (cudaStream_t)stream;
+  uint32_t word = 0;
+  cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof word, cudaMemcpyDeviceToHost, cs);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the status word");
+  if (word != 0) {
+    e = cudaMemsetAsync(workspace, 0, sizeof word, cs);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the status word");
+  }
+  if (word & tl::kStatusTimeout) return fail(TL_ERR_DEVICE_TIMEOUT, "device status word 0x%x", word);
+  if (word & tl::kStatusRange) return fail(TL_ERR_DEVICE_RANGE, "device status word 0x%x", word);
+  return TL_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,111 @@
+// Internal declarations shared by the host API and the kernels of libtlstoreh.so.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "tl_storeh.h"
+
+namespace tl {
+
+// ---------------------------------------------------------------- status word bits
+// The first 256 bytes of the decode workspace hold the device status word.
+enum : uint32_t {
+  kStatusRange = 1u << 0,    // a lane's loops / ctx_len was out of range; the lane was skipped
+  kStatusTimeout = 1u << 1,  // a bounded wait gave up
+};
+
+constexpr int kInt4Group = 64;
+constexpr int kMaxHeads = 16;        // heads are padded to 16 in the kernels
+constexpr int kSplitRows = 1024;     // context rows per split (a function of the lane's own ctx only)
+constexpr int kMaxCtx = 65536;       // positions per (layer, lane) the kernels support
+constexpr int kMaxSplits = kMaxCtx / kSplitRows;
+
+// ---------------------------------------------------------------- shapes
+struct Shape {
+  int d, H, hd, n_pre, L_max, max_lanes, max_ctx, fmt;
+  __host__ __device__ int layers() const { return n_pre + L_max; }
+  __host__ __device__ size_t row_code_bytes() const {
+    return fmt == TL_H_FP16 ? 2 * (size_t)d : fmt == TL_H_INT8_TOKEN ? (size_t)d : (size_t)d / 2;
+  }
+  __host__ __device__ int row_scales() const { return fmt == TL_H_FP16 ? 0 : fmt == TL_H_INT8_TOKEN ? 1 : d / kInt4Group; }
+  __host__ __device__ size_t scale_bytes() const { return fmt == TL_H_INT8_TOKEN ? 4 : 2; }
+  __host__ __device__ size_t rows_total() const { return (size_t)layers() * max_lanes * max_ctx; }
+};
+
+__host__ __device__ inline int splits_for_rows(int n_rows) { return (n_rows + kSplitRows - 1) / kSplitRows; }
+
+// ---------------------------------------------------------------- workspace layout
+// All offsets are 256-byte aligned.
+struct Workspace {
+  size_t status_off;   // uint32 status word (+ padding)
+  size_t q_off;        // fp32 [n_lanes][d]       q = W_q h_new
+  size_t qt_off;       // fp16 [n_lanes][16][d]   absorbed query, scaled by log2(e)/sqrt(hd)
+  size_t ml_off;       // fp32 [n_lanes][S_max][16][2]   per-split running max and sum
+  size_t u_off;        // fp32 [n_lanes][S_max][16][d]   per-split unnormalised sum_c p_c h_c
+  size_t total;
+  int s_max;
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+inline Workspace workspace_layout(const Shape& s, int n_lanes) {
+  Workspace w;
+  w.s_max = splits_for_rows(s.max_ctx);
+  size_t off = 0;
+  w.status_off = off;
+  off += 256;
+  w.q_off = off;
+  off = align256(off + (size_t)n_lanes * s.d * 4);
+  w.qt_off = off;
+  off = align256(off + (size_t)n_lanes * kMaxHeads * s.d * 2);
+  w.ml_off = off;
+  off = align256(off + (size_t)n_lanes * w.s_max * kMaxHeads * 2 * 4);
+  w.u_off = off;
+  off = align256(off + (size_t)n_lanes * w.s_max * kMaxHeads * (size_t)s.d * 4);
+  w.total = off;
+  return w;
+}
+
+// ---------------------------------------------------------------- measurement hook
+tl_profile*& current_profile();                  // thread-local; NULL when not installed
+inline void count_launch(int n = 1) {
+  if (tl_profile* p = current_profile()) p->launches += n;
+}
+void profile_stream_begin(cudaStream_t st);      // records begin_events[recorded] if installed
+void profile_stream_end(cudaStream_t st);        // records end_events[recorded++] if installed
+
+// ---------------------------------------------------------------- launchers (return cudaError_t)
+cudaError_t launch_append(const Shape& s, void* codes, void* scales, int layer, const __half* h_rows,
+                          int n_lanes, int n_rows, const int32_t* start_pos, const int32_t* row_count,
+                          const int32_t* loops, cudaStream_t st);
+
+// ctx_len == NULL: standalone check; otherwise lanes with out-of-range loops/ctx_len are skipped.
+cudaError_t launch_norm_check(const float* residual, int n_lanes, int d, float threshold, int iter,
+                              const int32_t* loops, const int32_t* ctx_len, int max_ctx, int L_max, uint8_t* flags,
+                              int32_t* first, float* norms, cudaStream_t st);
+
+struct DecodeArgs {
+  Shape s;
+  const void* codes;
+  const void* scales;
+  int iter;
+  const int32_t* loops;
+  const int32_t* ctx_len;
+  const __half* h_new;
+  const __half* Wq;
+  const __half* Wk;
+  const __half* Wv;
+  float* out;
+  int n_lanes;
+  uint8_t* ws;
+  Workspace wl;
+};
+
+cudaError_t launch_prologue(const DecodeArgs& a, cudaStream_t st);
+cudaError_t launch_stream(const DecodeArgs& a, cudaStream_t st);
+cudaError_t launch_epilogue(const DecodeArgs& a, cudaStream_t st);
+
+}  // namespace tl

@@ -42,6 +42,10 @@ class Workload:
     outlier_p: float = 0.0
     outlier_mul: float = 1.0
     forced_lanes: int = 0       # lanes forced above the threshold in the flag-mix variant
+    lane_ids: Optional[List[int]] = None  # generator lane of each batch position (default: itself)
+
+    def lane_id(self, b: int) -> int:
+        return b if self.lane_ids is None else self.lane_ids[b]
 
     @property
     def B(self) -> int:
@@ -66,21 +70,21 @@ class Workload:
         return normal_f16(self.seed, tid, 0, self.d * self.d, 1.0 / math.sqrt(self.d)).reshape(self.d, self.d)
 
     # ------------------------------------------------------------ h rows
-    def h_rows(self, layer: int, lane: int, pos0: int, n: int) -> np.ndarray:
-        """h rows (fp16 [n, d]) at cache coordinate (layer, lane, pos0 .. pos0+n-1)."""
-        return h_rows_f16(self.seed, row_id(layer, lane, np.arange(pos0, pos0 + n)), self.d,
+    def h_rows(self, layer: int, b: int, pos0: int, n: int) -> np.ndarray:
+        """h rows (fp16 [n, d]) of batch lane b at cache coordinate (layer, pos0 .. pos0+n-1)."""
+        return h_rows_f16(self.seed, row_id(layer, self.lane_id(b), np.arange(pos0, pos0 + n)), self.d,
                           self.outlier_p, self.outlier_mul)
 
-    def h_rows_into(self, out: np.ndarray, layer: int, lane: int, pos0: int) -> None:
+    def h_rows_into(self, out: np.ndarray, layer: int, b: int, pos0: int) -> None:
         n = out.shape[0]
-        h_rows_f16_into(out, self.seed, row_id(layer, lane, np.arange(pos0, pos0 + n)), self.d,
+        h_rows_f16_into(out, self.seed, row_id(layer, self.lane_id(b), np.arange(pos0, pos0 + n)), self.d,
                         self.outlier_p, self.outlier_mul)
 
     def h_new(self, it: int) -> np.ndarray:
         """New-token h for loop iteration ``it`` (fp16 [B, d]): the row at position ctx[b]
         of cache layer n_pre+it, so context rows and new rows share one stream."""
         layer = self.n_pre + it
-        ids = np.array([row_id(layer, b, self.ctx[b]) for b in range(self.B)], dtype=np.uint64)
+        ids = np.array([row_id(layer, self.lane_id(b), self.ctx[b]) for b in range(self.B)], dtype=np.uint64)
         return h_rows_f16(self.seed, ids, self.d, self.outlier_p, self.outlier_mul)
 
     # ------------------------------------------------------------ residual
@@ -93,11 +97,12 @@ class Workload:
         near the threshold."""
         out = np.empty((self.B, self.d), dtype=np.float32)
         for b in range(self.B):
-            z = normal_f64(self.seed, TID_RESIDUAL, (it * 256 + b) * self.d, self.d)
+            lid = self.lane_id(b)
+            z = normal_f64(self.seed, TID_RESIDUAL, (it * 256 + lid) * self.d, self.d)
             if not flag_mix:
                 out[b] = (z * self.residual_scale).astype(np.float32)
             else:
-                target = 2.0 * self.threshold if b < max(1, self.forced_lanes) else 0.5 * self.threshold
+                target = 2.0 * self.threshold if lid < max(1, self.forced_lanes) else 0.5 * self.threshold
                 out[b] = (z * (target / np.sqrt(np.sum(z * z)))).astype(np.float32)
         return out
 
@@ -136,6 +141,15 @@ def get_workload(name: str) -> Workload:
 
 
 WORKLOADS = ["tiny_fp16", "fp16_407m", "int8_b16", "int4_2b", "int4_mixed"]
+
+
+def select_lanes(w: Workload, lanes: List[int]) -> Workload:
+    """The same workload restricted to some of its lanes (each keeps its own rows and counts)."""
+    w2 = dataclasses.replace(w)
+    w2.ctx = [w.ctx[b] for b in lanes]
+    w2.loops = [w.loops[b] for b in lanes]
+    w2.lane_ids = [w.lane_id(b) for b in lanes]
+    return w2
 
 
 def small_variant(w: Workload, ctx: Optional[List[int]] = None, loops: Optional[List[int]] = None,

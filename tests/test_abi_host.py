@@ -1,0 +1,108 @@
+"""The C-ABI library on the host (no GPU): it loads, exports every symbol the
+header declares, sizes caches and workspaces, and rejects bad arguments
+before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _header_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"^\s*(?:TL_API\s+)?(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(tl_[a-z0-9_]+)\s*\(",
+                                text, re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def tl():
+    from store_kv_attention_b200 import build_lib
+    build_lib.build()
+    import store_kv_attention_b200 as m
+    return m
+
+
+def test_exports_every_declared_symbol(tl):
+    declared = _header_functions()
+    assert len(declared) >= 9
+    assert sorted(tl.EXPORTS) == declared
+    raw = ctypes.CDLL(tl.LIB_PATH)
+    for name in declared:
+        assert hasattr(raw, name), name
+    assert tl.lib.tl_storeh_abi_version() == 1
+
+
+def _desc(tl, **kw):
+    base = dict(d_model=2048, n_heads=16, head_dim=128, n_pre=2, L_max=8, max_lanes=32, max_ctx=4097,
+                fmt=tl.TL_H_INT4_G64)
+    base.update(kw)
+    return tl.StoreHDesc(**base)
+
+
+def test_cache_bytes_match_layout(tl):
+    cb, sb = tl.cache_bytes(_desc(tl))
+    rows = 10 * 32 * 4097
+    assert cb == rows * 1024 and sb == rows * 32 * 2
+    cb, sb = tl.cache_bytes(_desc(tl, fmt=tl.TL_H_INT8_TOKEN, d_model=1024, n_heads=16, head_dim=64))
+    assert cb == rows * 1024 and sb == rows * 4
+    cb, sb = tl.cache_bytes(_desc(tl, fmt=tl.TL_H_FP16, d_model=1024, n_heads=16, head_dim=64))
+    assert cb == rows * 2048 and sb == 0
+
+
+def test_workspace_bytes(tl):
+    b = tl.workspace_bytes(_desc(tl), 32)
+    assert b % 256 == 0 and b > 32 * 16 * 2048 * 4
+    with pytest.raises(tl.TLError) as e:
+        tl.workspace_bytes(_desc(tl), 33)
+    assert e.value.status == tl.TL_ERR_CAPACITY
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(d_model=2048, n_heads=15), 2),          # d != H * hd -> TL_ERR_SHAPE
+    (dict(head_dim=96, n_heads=16, d_model=1536), 4),
+    (dict(d_model=4352, n_heads=34, head_dim=128), 4),
+    (dict(n_heads=32, head_dim=64, d_model=2048), 4),
+    (dict(fmt=7), 1),
+    (dict(max_ctx=0), 1),
+    (dict(max_ctx=70000), 4),
+    (dict(L_max=0), 1),
+])
+def test_desc_validation(tl, kw, status):
+    with pytest.raises(tl.TLError) as e:
+        tl.cache_bytes(_desc(tl, **kw))
+    assert e.value.status == status
+
+
+def test_calls_rejected_before_launch(tl):
+    L = tl.lib
+    d = _desc(tl).c()
+    fake = ctypes.c_void_p(1 << 20)          # 256-aligned stand-in, never dereferenced
+    cache = tl.Cache(1 << 20, 1 << 21)
+    # NULL descriptor
+    assert L.tl_storeh_append(None, cache, 0, fake, 1, 1, fake, None, None, None) == tl.TL_ERR_INVALID_ARG
+    # lanes beyond capacity, layer outside the cache
+    assert L.tl_storeh_append(ctypes.byref(d), cache, 0, fake, 33, 1, fake, None, None, None) == tl.TL_ERR_CAPACITY
+    assert L.tl_storeh_append(ctypes.byref(d), cache, 10, fake, 1, 1, fake, None, None, None) == tl.TL_ERR_CAPACITY
+    # misaligned cache
+    bad = tl.Cache((1 << 20) + 16, 1 << 21)
+    assert L.tl_storeh_append(ctypes.byref(d), bad, 0, fake, 1, 1, fake, None, None, None) == tl.TL_ERR_INVALID_ARG
+    # zero rows is a no-op
+    assert L.tl_storeh_append(ctypes.byref(d), cache, 0, fake, 1, 0, fake, None, None, None) == tl.TL_OK
+    ws = tl.workspace_bytes(_desc(tl), 4)
+    args = lambda it, n, wsb, res=None, flags=None: (ctypes.byref(d), cache, it, fake, fake, fake, fake, fake, fake,
+                                                     fake, res, 50.0, flags, flags, None, fake, wsb, n, None)
+    assert L.tl_storeh_attn_decode(*args(8, 4, ws)) == tl.TL_ERR_CAPACITY        # iter >= L_max
+    assert L.tl_storeh_attn_decode(*args(0, 4, ws - 256)) == tl.TL_ERR_CAPACITY  # workspace too small
+    assert L.tl_storeh_attn_decode(*args(0, 0, ws)) == tl.TL_ERR_INVALID_ARG
+    assert L.tl_storeh_attn_decode(*args(0, 4, ws, res=fake)) == tl.TL_ERR_INVALID_ARG  # residual w/o flags
+    assert L.tl_residual_norm_check(None, 1, 8, 1.0, 0, None, fake, fake, None, None) == tl.TL_ERR_INVALID_ARG
+    assert L.tl_residual_norm_check(fake, 1, 8, float("nan"), 0, None, fake, fake, None, None) == tl.TL_ERR_INVALID_ARG
+    assert b"threshold" in L.tl_last_error_message()
+    assert L.tl_status_string(tl.TL_ERR_DEVICE_TIMEOUT).startswith(b"TL_ERR_DEVICE_TIMEOUT")

@@ -1,0 +1,255 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Bars: codes and scales bit-exact; abort flags and first-abort iterations
+identical; attention outputs within max-abs 2e-3 and relative L2 1e-3 of the
+oracle per (lane, iteration); a mixed-batch lane bitwise equal to its solo
+run; nothing outside a lane's layers and positions is read.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from synth.workloads import get_workload, select_lanes, small_variant
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS = 2e-3
+REL_L2 = 1e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from store_kv_attention_b200 import build_lib
+    build_lib.build()
+
+
+def _dw(w, **kw):
+    from synth.device import DeviceWorkload
+    return DeviceWorkload(w, **kw)
+
+
+def _oracle_lane(w, it, b, form="explicit"):
+    layer = w.n_pre + it
+    rows = np.concatenate([w.h_rows(layer, b, 0, w.ctx[b]), w.h_new(it)[b:b + 1]])
+    codes, scales = oracle.quantize_rows(rows, w.fmt)
+    hh = oracle.dequantize_rows(codes, scales, w.fmt, w.d)
+    W = [w.weight(k) for k in "qkv"]
+    f = oracle.attend_explicit if form == "explicit" else oracle.attend_absorbed
+    return f(hh, w.h_new(it)[b], *W, w.H, w.hd)
+
+
+def _assert_close(got, want, tag):
+    got = np.asarray(got, dtype=np.float64)
+    assert np.all(np.isfinite(got)), tag
+    err = np.abs(got - want)
+    rel = np.linalg.norm(got - want) / np.linalg.norm(want)
+    assert err.max() <= MAX_ABS and rel <= REL_L2, f"{tag}: max-abs {err.max():.3g} rel-L2 {rel:.3g}"
+    return err.max(), rel
+
+
+# --------------------------------------------------------------------------- append: codes
+@pytest.mark.parametrize("fmt", [0, 1, 2])
+def test_append_codes_bit_exact(fmt):
+    import store_kv_attention_b200 as tl
+    d = 2048 if fmt == 2 else 1024
+    H, hd = (16, 128) if fmt == 2 else (16, 64)
+    rng = np.random.default_rng(11 + fmt)
+    n = 300
+    h = (rng.standard_normal((n, d)) * np.exp(rng.uniform(-4, 4, (n, 1)))).astype(np.float16)
+    h[0] = 0                                                 # zero row -> scale 0, codes 0
+    h[1, :64] = np.array([7, 0.5, 1.5, 2.5, 3.5, -3.5, 6.5, -7] * 8, np.float16)  # ties
+    h[2] = np.float16(1e-7)                                  # fp16 subnormals
+    h[3, ::2] *= np.float16(100)                            # wide range inside a row
+    desc = tl.StoreHDesc(d, H, hd, n_pre=1, L_max=2, max_lanes=2, max_ctx=n + 5, fmt=fmt)
+    cache = tl.StoreHCache(desc)
+    cache.codes.fill_(0xAB)
+    if cache.scales is not None:
+        cache.scales.fill_(0xCD)
+    hd_t = torch.from_numpy(h.view(np.int16)).view(torch.float16).cuda()
+    rows = torch.stack([hd_t, hd_t.flip(0)])                 # lane 1 gets the rows reversed
+    start = torch.tensor([3, 0], dtype=torch.int32, device="cuda")
+    tl.append(cache, 2, rows, start)
+    torch.cuda.synchronize()
+    cb = oracle.row_code_bytes(fmt, d)
+    codes = cache.codes.view(3, 2, n + 5, cb).cpu().numpy()
+    for lane, src, p0 in ((0, h, 3), (1, h[::-1].copy(), 0)):
+        want_c, want_s = oracle.quantize_rows(src, fmt)
+        assert np.array_equal(codes[2, lane, p0:p0 + n], want_c), f"codes lane {lane}"
+        if fmt != 0:
+            ns = oracle.row_scale_count(fmt, d)
+            sdt = np.float32 if fmt == 1 else np.float16
+            sc = cache.scales.view(-1)[:3 * 2 * (n + 5) * ns * np.dtype(sdt).itemsize].cpu().numpy()
+            sc = sc.view(sdt).reshape(3, 2, n + 5, ns)
+            assert np.array_equal(sc[2, lane, p0:p0 + n].view(np.uint8), want_s.astype(sdt).view(np.uint8))
+    # untouched positions stay untouched
+    assert np.all(codes[2, 0, :3] == 0xAB) and np.all(codes[2, 1, n:] == 0xAB) and np.all(codes[:2] == 0xAB)
+
+
+def test_append_skips_lanes_past_their_loops_and_out_of_range_rows():
+    import store_kv_attention_b200 as tl
+    d, H, hd = 256, 4, 64
+    desc = tl.StoreHDesc(d, H, hd, n_pre=1, L_max=3, max_lanes=3, max_ctx=8, fmt=0)
+    cache = tl.StoreHCache(desc)
+    cache.codes.fill_(0)
+    rows = torch.ones((3, 4, d), dtype=torch.float16, device="cuda")
+    loops = torch.tensor([1, 2, 3], dtype=torch.int32, device="cuda")
+    start = torch.tensor([0, 6, 0], dtype=torch.int32, device="cuda")     # lane 1 runs past max_ctx
+    count = torch.tensor([4, 4, 2], dtype=torch.int32, device="cuda")
+    tl.append(cache, 2, rows, start, row_count=count, loops=loops)         # layer 2 = iteration 1
+    torch.cuda.synchronize()
+    c = cache.codes.view(4, 3, 8, 2 * d).cpu().numpy()
+    assert np.all(c[2, 0] == 0)                        # loops=1: layer 2 is beyond the lane's depth
+    assert np.all(c[2, 1, 6:8] != 0) and np.all(c[2, 1, :6] == 0)
+    assert np.all(c[2, 2, :2] != 0) and np.all(c[2, 2, 2:] == 0)
+
+
+# --------------------------------------------------------------------------- safety check
+@pytest.mark.parametrize("flag_mix", [False, True])
+def test_norm_flags_identical(flag_mix):
+    import store_kv_attention_b200 as tl
+    w = get_workload("int4_mixed")
+    res = [w.residual(it, flag_mix) for it in range(6)]
+    loops = np.array(w.loops, np.int32)
+    loops[5] = 0
+    f = np.zeros(w.B, np.uint8)
+    fi = np.full(w.B, -1, np.int32)
+    df = torch.zeros(w.B, dtype=torch.uint8, device="cuda")
+    dfi = torch.full((w.B,), -1, dtype=torch.int32, device="cuda")
+    dl = torch.from_numpy(loops).cuda()
+    for it in range(6):
+        r = res[it].copy()
+        if it == 2:
+            r *= 0.01          # a quiet iteration: flags stay sticky
+        f, fi, nrm = oracle.residual_norm_check(r, w.threshold, it, loops, f, fi)
+        dn = torch.full((w.B,), float("nan"), device="cuda")
+        tl.residual_norm_check(torch.from_numpy(r).cuda(), w.threshold, it, dl, df, dfi, norms_out=dn)
+        torch.cuda.synchronize()
+        assert np.array_equal(df.cpu().numpy(), f) and np.array_equal(dfi.cpu().numpy(), fi)
+        act = ~np.isnan(nrm)
+        assert np.allclose(dn.cpu().numpy()[act], nrm[act], rtol=1e-6)
+    if flag_mix:
+        assert 0 < f.sum() < w.B
+
+
+# --------------------------------------------------------------------------- decode: small sizes
+SMALL = [
+    ("tiny_fp16", None, None),
+    ("fp16_407m", [0, 1, 127, 128, 129, 1030, 2200], [8, 3, 8, 1, 5, 8, 2]),
+    ("int8_b16", [0, 5, 255, 1023, 1024, 2047, 2049], [8, 8, 2, 7, 8, 4, 8]),
+    ("int4_2b", [0, 3, 130, 1000, 1025, 2048, 3000], [8, 1, 8, 6, 8, 8, 3]),
+    ("int4_mixed", [1, 129, 700, 1024, 2500, 64], [4, 16, 32, 4, 16, 32]),
+]
+
+
+def _small(name, ctx, loops):
+    w = get_workload(name)
+    if ctx is None:
+        return w
+    return small_variant(w, ctx=ctx, loops=loops, name=name + "_small")
+
+
+@pytest.mark.parametrize("name,ctx,loops", SMALL, ids=[s[0] for s in SMALL])
+def test_decode_matches_oracle_small(name, ctx, loops):
+    w = _small(name, ctx, loops)
+    dw = _dw(w, flag_mix=True)
+    dw.step()
+    torch.cuda.synchronize()
+    out = dw.out.cpu().numpy()
+    f = np.zeros(w.B, np.uint8)
+    fi = np.full(w.B, -1, np.int32)
+    its = range(w.L_max) if w.L_max <= 8 else [0, 3, 4, 15, 16, 31]
+    for it in range(w.L_max):
+        for b in range(w.B):
+            active = it < w.loops[b]
+            if not active:
+                assert np.all(np.isnan(out[it, b])), f"inactive lane {b} iteration {it} was written"
+            elif it in its:
+                _assert_close(out[it, b], _oracle_lane(w, it, b), f"{name} lane {b} it {it}")
+        f, fi, _ = oracle.residual_norm_check(w.residual(it, True), w.threshold, it, np.array(w.loops), f, fi)
+    assert np.array_equal(dw.flags.cpu().numpy(), f) and np.array_equal(dw.first.cpu().numpy(), fi)
+    import store_kv_attention_b200 as tl
+    assert tl.poll_status(dw.cache) == tl.TL_OK
+
+
+def test_mixed_batch_lane_bitwise_equals_solo():
+    """Architecture-Exclusive Features, "L-aware batching": a lane of a mixed batch
+    gives bit-for-bit the result of the same lane run alone."""
+    w = _small("int4_mixed", [1, 129, 700, 1024, 2500, 64], [4, 16, 32, 4, 16, 32])
+    mixed = _dw(w)
+    mixed.step()
+    torch.cuda.synchronize()
+    a_all = mixed.out.cpu().numpy()
+    for b in (1, 4, 5):
+        solo = _dw(select_lanes(w, [b]))
+        solo.step()
+        torch.cuda.synchronize()
+        s = solo.out[:, 0].cpu().numpy()
+        assert np.array_equal(a_all[:, b].view(np.uint32), s.view(np.uint32)), f"lane {b}"
+        assert solo.flags.item() == mixed.flags[b].item() and solo.first.item() == mixed.first[b].item()
+
+
+def test_poisoned_layers_and_positions_are_not_read():
+    import store_kv_attention_b200 as tl
+    w = _small("int8_b16", [3, 300, 1100], [2, 8, 5])
+    clean = _dw(w)
+    clean.step()
+    dirty = _dw(w, fill=False)
+    # poison everything first (0x7f / 0x80 int8 codes and NaN scales), then write the real rows
+    dirty.cache.codes.fill_(0x7F)
+    dirty.cache.scales.view(torch.float32)[:].fill_(float("nan"))
+    dirty.fill_context()
+    dirty.step()
+    torch.cuda.synchronize()
+    a, b = clean.out.cpu().numpy(), dirty.out.cpu().numpy()
+    assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+    assert tl.poll_status(dirty.cache) == tl.TL_OK
+
+
+def test_out_of_range_lane_is_skipped_and_reported():
+    import store_kv_attention_b200 as tl
+    w = _small("tiny_fp16", [5, 9], [2, 2])
+    w.L_max = 2
+    dw = _dw(w)
+    dw.ctx[1] = w.max_ctx + 7           # beyond the cache
+    dw.decode(0)
+    torch.cuda.synchronize()
+    out = dw.out[0].cpu().numpy()
+    assert np.all(np.isfinite(out[0])) and np.all(np.isnan(out[1]))
+    assert tl.poll_status(dw.cache) == tl.TL_ERR_DEVICE_RANGE
+    assert tl.poll_status(dw.cache) == tl.TL_OK        # cleared by the poll
+
+
+# --------------------------------------------------------------------------- decode: full sizes, sampled
+FULL = [
+    ("fp16_407m", [(it, 0) for it in range(8)]),
+    ("int8_b16", [(0, 0), (3, 7), (7, 15)]),
+    ("int4_2b", [(0, 0), (4, 1), (7, 31)]),
+    ("int4_mixed", [(0, 0), (3, 15), (10, 20), (31, 47), (15, 33)]),
+]
+
+
+@pytest.mark.parametrize("name,samples", FULL, ids=[f[0] for f in FULL])
+def test_decode_full_size_sampled(name, samples):
+    import store_kv_attention_b200 as tl
+    w = get_workload(name)
+    dw = _dw(w)
+    dw.step()
+    torch.cuda.synchronize()
+    out = dw.out.cpu().numpy()
+    for it, b in samples:
+        assert it < w.loops[b]
+        _assert_close(out[it, b], _oracle_lane(w, it, b, form="absorbed"), f"{name} lane {b} it {it}")
+    # every active (lane, iteration) was written, every inactive one was not
+    act = np.array([[it < w.loops[b] for b in range(w.B)] for it in range(w.L_max)])
+    assert np.all(np.isfinite(out[act])) and np.all(np.isnan(out[~act]))
+    f = np.zeros(w.B, np.uint8)
+    fi = np.full(w.B, -1, np.int32)
+    for it in range(w.L_max):
+        f, fi, _ = oracle.residual_norm_check(w.residual(it), w.threshold, it, np.array(w.loops), f, fi)
+    assert np.array_equal(dw.flags.cpu().numpy(), f) and np.array_equal(dw.first.cpu().numpy(), fi)
+    assert tl.poll_status(dw.cache) == tl.TL_OK
