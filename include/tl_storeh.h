@@ -81,7 +81,7 @@ typedef enum {
 
 /*
  * Shape of one store-h cache.  Supported: head_dim in {64, 128};
- * d_model = n_heads * head_dim with d_model a multiple of 256 and at most 4096;
+ * d_model = n_heads * head_dim with d_model a multiple of 256 and at most 2048;
  * n_heads <= 16; 1 <= max_ctx <= 65536 counts every position including the newest token.
  */
 typedef struct {

@@ -208,6 +208,10 @@ class ProfileHook:
         import torch
         self.events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                        for _ in range(capacity)]
+        for b, e in self.events:      # torch creates the CUDA event on its first record
+            b.record()
+            e.record()
+        torch.cuda.synchronize()
         self._b = (ctypes.c_void_p * capacity)(*[e[0].cuda_event for e in self.events])
         self._e = (ctypes.c_void_p * capacity)(*[e[1].cuda_event for e in self.events])
         self.p = Profile(self._b, self._e, capacity, 0, 0)

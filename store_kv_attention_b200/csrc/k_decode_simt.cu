@@ -3,7 +3,7 @@
 //  Features, "Store-h KV cache", "Variable-L KV cache", "L-aware batching"]
 //
 // Absorbed form of K = W_k h, V = W_v h for one loop iteration i, layer n_pre+i:
-//   prologue : q = W_q h_new ; qt_j = W_k[j]^T q_j * log2(e)/sqrt(hd)   (fp16, workspace)
+//   prologue : q = W_q h_new ; qt_j = W_k[j]^T q_j * log2(e)/sqrt(hd)   (fp32, workspace)
 //   stream   : per (lane, split): s_cj = qt_j . h_c ; online softmax in base 2 ;
 //              U_j = sum_c 2^(s_cj - m_j) h_c  (partials m, l, U in the workspace)
 //   epilogue : merge the splits of a lane exactly ; u_j = U_j / l_j ; out_j = W_v[j] u_j
@@ -77,18 +77,18 @@ __global__ void __launch_bounds__(kQWarps * 32) q_kernel(Shape s, int iter, cons
 }
 
 // ------------------------------------------------------------------ prologue: qt
-// qt[b][j][c] = sum_{r<hd} W_k[j*hd + r][c] * q[b][j*hd + r], times log2(e)/sqrt(hd).
+// qt[b][j][c] = sum_{r<hd} W_k[j*hd + r][c] * q[b][j*hd + r], times log2(e)/sqrt(hd), in fp32.
 // Block (column block, head j); thread = column c.  Heads j >= H are written as 0.
 constexpr int kQtThreads = 256;
 
 __global__ void __launch_bounds__(kQtThreads) qt_kernel(Shape s, int iter, const int32_t* __restrict__ loops,
                                                         const int32_t* __restrict__ ctx_len,
                                                         const __half* __restrict__ Wk, const float* __restrict__ q,
-                                                        __half* __restrict__ qt, int n_lanes) {
+                                                        float* __restrict__ qt, int n_lanes) {
   const int c = blockIdx.x * kQtThreads + threadIdx.x;
   const int j = blockIdx.y;
   if (j >= s.H) {
-    for (int b = 0; b < n_lanes; ++b) qt[((size_t)b * kMaxHeads + j) * s.d + c] = __float2half_rn(0.0f);
+    for (int b = 0; b < n_lanes; ++b) qt[((size_t)b * kMaxHeads + j) * s.d + c] = 0.0f;
     return;
   }
   const float scale = 1.4426950408889634f / sqrtf((float)s.hd);
@@ -98,7 +98,7 @@ __global__ void __launch_bounds__(kQtThreads) qt_kernel(Shape s, int iter, const
     float acc = 0.0f;
     const float* qj = q + (size_t)b * s.d + j * s.hd;
     for (int r = 0; r < s.hd; ++r) acc = fmaf(__half2float(Wk[(size_t)(j * s.hd + r) * s.d + c]), qj[r], acc);
-    qt[((size_t)b * kMaxHeads + j) * s.d + c] = __float2half_rn(acc * scale);
+    qt[((size_t)b * kMaxHeads + j) * s.d + c] = acc * scale;
   }
 }
 
@@ -131,7 +131,7 @@ __device__ __forceinline__ void dequant_tile(const Shape& s, const uint8_t* code
 
 __global__ void __launch_bounds__(512) stream_kernel(Shape s, int iter, const int32_t* __restrict__ loops,
                               const int32_t* __restrict__ ctx_len, const uint8_t* __restrict__ codes,
-                              const uint8_t* __restrict__ scales, const __half* __restrict__ qt,
+                              const uint8_t* __restrict__ scales, const float* __restrict__ qt,
                               float* __restrict__ ml, float* __restrict__ U, int s_max, int T) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int split = blockIdx.x, b = blockIdx.y;
@@ -142,15 +142,15 @@ __global__ void __launch_bounds__(512) stream_kernel(Shape s, int iter, const in
   const int d = s.d, H = s.H;
   const int r_begin = split * kSplitRows, r_end = min(n, r_begin + kSplitRows);
 
-  __half* qt_sh = reinterpret_cast<__half*>(smem);                         // [16][d]
-  float* hrow = reinterpret_cast<float*>(smem + (size_t)kMaxHeads * d * 2);  // [T][d]
+  float* qt_sh = reinterpret_cast<float*>(smem);                           // [16][d]
+  float* hrow = qt_sh + (size_t)kMaxHeads * d;                             // [T][d]
   float* sc = hrow + (size_t)T * d;                                        // [T][16]
   float* m_sh = sc + T * kMaxHeads;                                        // [16]
   float* l_sh = m_sh + kMaxHeads;                                          // [16]
   float* a_sh = l_sh + kMaxHeads;                                          // [16]
 
-  for (int i = threadIdx.x; i < kMaxHeads * d / 8; i += blockDim.x)
-    reinterpret_cast<uint4*>(qt_sh)[i] = reinterpret_cast<const uint4*>(qt + (size_t)b * kMaxHeads * d)[i];
+  for (int i = threadIdx.x; i < kMaxHeads * d / 4; i += blockDim.x)
+    reinterpret_cast<float4*>(qt_sh)[i] = reinterpret_cast<const float4*>(qt + (size_t)b * kMaxHeads * d)[i];
   if (threadIdx.x < kMaxHeads) {
     m_sh[threadIdx.x] = -CUDART_INF_F;
     l_sh[threadIdx.x] = 0.0f;
@@ -182,7 +182,7 @@ __global__ void __launch_bounds__(512) stream_kernel(Shape s, int iter, const in
         const float h = hrow[rr * d + k];
 #pragma unroll
         for (int j = 0; j < kMaxHeads; ++j)
-          if (j < H) part[j] = fmaf(__half2float(qt_sh[j * d + k]), h, part[j]);
+          if (j < H) part[j] = fmaf(qt_sh[j * d + k], h, part[j]);
       }
 #pragma unroll
       for (int j = 0; j < kMaxHeads; ++j) {
@@ -327,7 +327,7 @@ __global__ void __launch_bounds__(kEpiThreads) epilogue_kernel(Shape s, int iter
 cudaError_t launch_prologue(const DecodeArgs& a, cudaStream_t st) {
   const Shape& s = a.s;
   float* q = reinterpret_cast<float*>(a.ws + a.wl.q_off);
-  __half* qt = reinterpret_cast<__half*>(a.ws + a.wl.qt_off);
+  float* qt = reinterpret_cast<float*>(a.ws + a.wl.qt_off);
   uint32_t* status = reinterpret_cast<uint32_t*>(a.ws + a.wl.status_off);
   q_kernel<<<(s.d + kQWarps - 1) / kQWarps, kQWarps * 32, 0, st>>>(s, a.iter, a.loops, a.ctx_len, a.h_new, a.Wq, q,
                                                                   a.n_lanes, status);
@@ -342,14 +342,14 @@ cudaError_t launch_prologue(const DecodeArgs& a, cudaStream_t st) {
 
 cudaError_t launch_stream(const DecodeArgs& a, cudaStream_t st) {
   const Shape& s = a.s;
-  const int T = s.d <= 2048 ? 8 : 4;
-  const size_t sm = (size_t)kMaxHeads * s.d * 2 + (size_t)T * s.d * 4 + (size_t)T * kMaxHeads * 4 + 3 * kMaxHeads * 4;
+  const int T = 8;
+  const size_t sm = (size_t)kMaxHeads * s.d * 4 + (size_t)T * s.d * 4 + (size_t)T * kMaxHeads * 4 + 3 * kMaxHeads * 4;
   cudaError_t e = cudaFuncSetAttribute(stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   dim3 grid(a.wl.s_max, a.n_lanes);
   stream_kernel<<<grid, s.d / 8, sm, st>>>(s, a.iter, a.loops, a.ctx_len, (const uint8_t*)a.codes,
                                            (const uint8_t*)a.scales,
-                                           reinterpret_cast<const __half*>(a.ws + a.wl.qt_off),
+                                           reinterpret_cast<const float*>(a.ws + a.wl.qt_off),
                                            reinterpret_cast<float*>(a.ws + a.wl.ml_off),
                                            reinterpret_cast<float*>(a.ws + a.wl.u_off), a.wl.s_max, T);
   count_launch();

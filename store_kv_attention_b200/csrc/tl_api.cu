@@ -34,8 +34,8 @@ tl_status check_desc(const tl_storeh_desc* d, tl::Shape* s) {
   if ((int64_t)d->n_heads * d->head_dim != d->d_model)
     return fail(TL_ERR_SHAPE, "d_model %d != n_heads %d * head_dim %d", d->d_model, d->n_heads, d->head_dim);
   if (d->head_dim != 64 && d->head_dim != 128) return fail(TL_ERR_UNSUPPORTED, "head_dim %d not in {64, 128}", d->head_dim);
-  if (d->d_model % 256 != 0 || d->d_model > 4096)
-    return fail(TL_ERR_UNSUPPORTED, "d_model %d must be a multiple of 256 and at most 4096", d->d_model);
+  if (d->d_model % 256 != 0 || d->d_model > 2048)
+    return fail(TL_ERR_UNSUPPORTED, "d_model %d must be a multiple of 256 and at most 2048", d->d_model);
   if (d->n_heads > tl::kMaxHeads) return fail(TL_ERR_UNSUPPORTED, "n_heads %d > %d", d->n_heads, tl::kMaxHeads);
   if (d->max_ctx > tl::kMaxCtx) return fail(TL_ERR_UNSUPPORTED, "max_ctx %d > %d", d->max_ctx, tl::kMaxCtx);
   if ((int64_t)(d->n_pre + d->L_max) * d->max_lanes * d->max_ctx > ((int64_t)1 << 40))

@@ -42,7 +42,7 @@ __host__ __device__ inline int splits_for_rows(int n_rows) { return (n_rows + kS
 struct Workspace {
   size_t status_off;   // uint32 status word (+ padding)
   size_t q_off;        // fp32 [n_lanes][d]       q = W_q h_new
-  size_t qt_off;       // fp16 [n_lanes][16][d]   absorbed query, scaled by log2(e)/sqrt(hd)
+  size_t qt_off;       // fp32 [n_lanes][16][d]   absorbed query, scaled by log2(e)/sqrt(hd)
   size_t ml_off;       // fp32 [n_lanes][S_max][16][2]   per-split running max and sum
   size_t u_off;        // fp32 [n_lanes][S_max][16][d]   per-split unnormalised sum_c p_c h_c
   size_t total;
@@ -60,7 +60,7 @@ inline Workspace workspace_layout(const Shape& s, int n_lanes) {
   w.q_off = off;
   off = align256(off + (size_t)n_lanes * s.d * 4);
   w.qt_off = off;
-  off = align256(off + (size_t)n_lanes * kMaxHeads * s.d * 2);
+  off = align256(off + (size_t)n_lanes * kMaxHeads * s.d * 4);
   w.ml_off = off;
   off = align256(off + (size_t)n_lanes * w.s_max * kMaxHeads * 2 * 4);
   w.u_off = off;

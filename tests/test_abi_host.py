@@ -67,7 +67,8 @@ def test_workspace_bytes(tl):
 @pytest.mark.parametrize("kw,status", [
     (dict(d_model=2048, n_heads=15), 2),          # d != H * hd -> TL_ERR_SHAPE
     (dict(head_dim=96, n_heads=16, d_model=1536), 4),
-    (dict(d_model=4352, n_heads=34, head_dim=128), 4),
+    (dict(d_model=2304, n_heads=18, head_dim=128), 4),
+    (dict(d_model=4096, n_heads=32, head_dim=128), 4),
     (dict(n_heads=32, head_dim=64, d_model=2048), 4),
     (dict(fmt=7), 1),
     (dict(max_ctx=0), 1),
