@@ -190,6 +190,38 @@ TL_API tl_status tl_residual_norm_check(const float* residual, int32_t n_lanes, 
                                  int32_t* first_abort_iter, float* norms_out, tl_stream_t stream);
 
 /*
+ * tl_storeh_attn_decode without a caller-supplied workspace, for callers that
+ * cannot allocate device memory (no cudaMalloc, no allocator of their own:
+ * plug-ins running inside a host application's memory budget, code that must
+ * not allocate once a stream or graph is set up, and similar).  The pages have
+ * no counterpart; this is a packaging variant of the decode above.
+ *
+ * Same arguments, meaning and results as tl_storeh_attn_decode, minus
+ * `workspace` / `workspace_bytes`.  The scratch is a 32 MiB array compiled into
+ * the library (a static __device__ variable): every GPU that loads the library
+ * holds those 32 MiB until the process exits.  Requests whose workspace
+ * (tl_storeh_workspace_bytes) would exceed 32 MiB are rejected with
+ * TL_ERR_CAPACITY before anything is launched.  The call allocates nothing: no
+ * cudaMalloc, cudaFree or allocating library routine.
+ *
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call before
+ * any stream capture.  All calls in the process share the one array and it
+ * keeps the previous call's contents (the call clears the part that must start
+ * at zero itself): two calls that may overlap on the GPU — on different streams
+ * without an ordering between them — race on it and give wrong results.
+ *   status_out  device uint32 or NULL: receives this call's device status word
+ *               (bit 0 = a lane's loops/ctx_len was out of range and the lane was
+ *               skipped, bit 1 = a bounded device wait gave up).
+ */
+TL_API tl_status tl_storeh_attn_decode_static_ws(const tl_storeh_desc* desc, tl_storeh_cache cache, int32_t iter,
+                                                 const int32_t* loops, const int32_t* ctx_len, const void* h_new,
+                                                 const void* W_q, const void* W_k, const void* W_v, float* out,
+                                                 const float* residual, float threshold, uint8_t* abort_flags,
+                                                 int32_t* first_abort_iter, float* norms_out, int32_t n_lanes,
+                                                 uint32_t* status_out, tl_stream_t stream);
+
+/*
  * Synchronises `stream`, then reads and clears the status word that kernels
  * of tl_storeh_attn_decode record in `workspace`.  Returns TL_OK,
  * TL_ERR_DEVICE_TIMEOUT (a bounded device wait gave up), TL_ERR_DEVICE_RANGE

@@ -34,7 +34,7 @@ TL_H_INT4_G64 = 2
 # every symbol include/tl_storeh.h declares
 EXPORTS = ["tl_storeh_cache_bytes", "tl_storeh_workspace_bytes", "tl_storeh_append", "tl_storeh_attn_decode",
            "tl_residual_norm_check", "tl_storeh_poll_status", "tl_status_string", "tl_last_error_message",
-           "tl_storeh_abi_version", "tl_set_profile"]
+           "tl_storeh_abi_version", "tl_set_profile", "tl_storeh_attn_decode_static_ws"]
 
 
 class TLError(RuntimeError):
@@ -87,6 +87,9 @@ def _load():
     L.tl_last_error_message.argtypes = []
     L.tl_last_error_message.restype = ctypes.c_char_p
     L.tl_storeh_abi_version.restype = ctypes.c_int32
+    L.tl_storeh_attn_decode_static_ws.argtypes = [P(Desc), Cache, i32, vp, vp, vp, vp, vp, vp, vp, vp, f32, vp,
+                                                  vp, vp, i32, vp, vp]
+    L.tl_storeh_attn_decode_static_ws.restype = ctypes.c_int
     L.tl_set_profile.argtypes = [P(Profile)]
     L.tl_set_profile.restype = ctypes.c_int
     _lib_handle = L
@@ -185,6 +188,19 @@ def attn_decode(cache: StoreHCache, it: int, loops, ctx_len, h_new, W_q, W_k, W_
                                      float(threshold), _ptr(abort_flags), _ptr(first_abort_iter), _ptr(norms_out),
                                      cache.workspace.data_ptr(), cache.ws_bytes, n_lanes, _stream(stream)),
            "tl_storeh_attn_decode")
+
+
+def attn_decode_static_ws(cache: StoreHCache, it: int, loops, ctx_len, h_new, W_q, W_k, W_v, out,
+                          residual=None, threshold: float = 0.0, abort_flags=None, first_abort_iter=None,
+                          norms_out=None, status_out=None, stream=None) -> None:
+    """attn_decode on the library's built-in scratch (for callers that cannot allocate)."""
+    n_lanes = int(h_new.shape[0])
+    _check(_load().tl_storeh_attn_decode_static_ws(ctypes.byref(cache.desc.c()), cache.c(), it, _ptr(loops),
+                                                   _ptr(ctx_len), _ptr(h_new), _ptr(W_q), _ptr(W_k), _ptr(W_v),
+                                                   _ptr(out), _ptr(residual), float(threshold), _ptr(abort_flags),
+                                                   _ptr(first_abort_iter), _ptr(norms_out), n_lanes,
+                                                   _ptr(status_out), _stream(stream)),
+           "tl_storeh_attn_decode_static_ws")
 
 
 def residual_norm_check(residual, threshold: float, it: int, loops, abort_flags, first_abort_iter,

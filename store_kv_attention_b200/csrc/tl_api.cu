@@ -56,6 +56,14 @@ tl_status check_cache(const tl::Shape& s, const tl_storeh_cache& c) {
 
 namespace tl {
 
+tl_status set_error(tl_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof g_msg, fmt, ap);
+  va_end(ap);
+  return st;
+}
+
 tl_profile*& current_profile() {
   thread_local tl_profile* p = nullptr;
   return p;

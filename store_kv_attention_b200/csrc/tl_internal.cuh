@@ -69,6 +69,9 @@ inline Workspace workspace_layout(const Shape& s, int n_lanes) {
   return w;
 }
 
+// Records a message for tl_last_error_message() and returns `st`.
+tl_status set_error(tl_status st, const char* fmt, ...);
+
 // ---------------------------------------------------------------- measurement hook
 tl_profile*& current_profile();                  // thread-local; NULL when not installed
 inline void count_launch(int n = 1) {
