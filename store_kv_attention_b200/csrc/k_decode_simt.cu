@@ -1,11 +1,12 @@
-// Store-h decode attention, CUDA-core kernels (prologue, split-context stream, epilogue).
+// Store-h decode attention, CUDA-core kernels: prologue (query, absorbed query) and epilogue
+// (split merge + W_v).  The context-streaming kernel between them is k_stream_tc.cu.
 // [Novel Contributions, "Novel Mechanism: Store-h KV Cache"; Architecture-Exclusive
 //  Features, "Store-h KV cache", "Variable-L KV cache", "L-aware batching"]
 //
 // Absorbed form of K = W_k h, V = W_v h for one loop iteration i, layer n_pre+i:
 //   prologue : q = W_q h_new ; qt_j = W_k[j]^T q_j * log2(e)/sqrt(hd)   (fp32, workspace)
-//   stream   : per (lane, split): s_cj = qt_j . h_c ; online softmax in base 2 ;
-//              U_j = sum_c 2^(s_cj - m_j) h_c  (partials m, l, U in the workspace)
+//   stream   : (tensor cores, k_stream_tc.cu) per (lane, split): s_cj = qt_j . h_c ;
+//              online softmax in base 2 ; U_j = sum_c 2^(s_cj - m_j) h_c  (partials m, l, U)
 //   epilogue : merge the splits of a lane exactly ; u_j = U_j / l_j ; out_j = W_v[j] u_j
 // The split plan depends only on the lane's own context length, so a lane's
 // result does not depend on which other lanes share its batch.
@@ -102,153 +103,6 @@ __global__ void __launch_bounds__(kQtThreads) qt_kernel(Shape s, int iter, const
   }
 }
 
-// ------------------------------------------------------------------ stream
-// Block = d/8 threads; thread t owns columns 8t .. 8t+7 of U for every head.
-// Tiles of T rows are dequantised to fp32 in shared memory.
-__device__ __forceinline__ void dequant_tile(const Shape& s, const uint8_t* codes_row0, const uint8_t* scales_row0,
-                                             int r0, int rows, int T, float* hrow) {
-  const int d = s.d;
-  for (int i = threadIdx.x; i < T * d; i += blockDim.x) {
-    const int rr = i / d, k = i % d;
-    float v = 0.0f;
-    if (rr < rows) {
-      const size_t row = (size_t)(r0 + rr);
-      if (s.fmt == TL_H_FP16) {
-        v = __half2float(reinterpret_cast<const __half*>(codes_row0)[row * d + k]);
-      } else if (s.fmt == TL_H_INT8_TOKEN) {
-        v = (float)reinterpret_cast<const int8_t*>(codes_row0)[row * d + k] *
-            reinterpret_cast<const float*>(scales_row0)[row];
-      } else {
-        const uint8_t byte = codes_row0[row * (d / 2) + k / 2];
-        int code = (k & 1) ? (byte >> 4) : (byte & 0xF);
-        code = code >= 8 ? code - 16 : code;
-        v = (float)code * __half2float(reinterpret_cast<const __half*>(scales_row0)[row * (d / kInt4Group) + k / kInt4Group]);
-      }
-    }
-    hrow[rr * d + k] = v;
-  }
-}
-
-__global__ void __launch_bounds__(512) stream_kernel(Shape s, int iter, const int32_t* __restrict__ loops,
-                              const int32_t* __restrict__ ctx_len, const uint8_t* __restrict__ codes,
-                              const uint8_t* __restrict__ scales, const float* __restrict__ qt,
-                              float* __restrict__ ml, float* __restrict__ U, int s_max, int T) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  const int split = blockIdx.x, b = blockIdx.y;
-  int n;
-  if (!lane_active(s, iter, loops, ctx_len, b, &n)) return;
-  const int S = splits_for_rows(n);
-  if (split >= S) return;
-  const int d = s.d, H = s.H;
-  const int r_begin = split * kSplitRows, r_end = min(n, r_begin + kSplitRows);
-
-  float* qt_sh = reinterpret_cast<float*>(smem);                           // [16][d]
-  float* hrow = qt_sh + (size_t)kMaxHeads * d;                             // [T][d]
-  float* sc = hrow + (size_t)T * d;                                        // [T][16]
-  float* m_sh = sc + T * kMaxHeads;                                        // [16]
-  float* l_sh = m_sh + kMaxHeads;                                          // [16]
-  float* a_sh = l_sh + kMaxHeads;                                          // [16]
-
-  for (int i = threadIdx.x; i < kMaxHeads * d / 4; i += blockDim.x)
-    reinterpret_cast<float4*>(qt_sh)[i] = reinterpret_cast<const float4*>(qt + (size_t)b * kMaxHeads * d)[i];
-  if (threadIdx.x < kMaxHeads) {
-    m_sh[threadIdx.x] = -CUDART_INF_F;
-    l_sh[threadIdx.x] = 0.0f;
-  }
-
-  const int layer = s.n_pre + iter;
-  const size_t row0 = ((size_t)layer * s.max_lanes + b) * s.max_ctx;
-  const uint8_t* crow = codes + row0 * s.row_code_bytes();
-  const uint8_t* srow = scales ? scales + row0 * s.row_scales() * s.scale_bytes() : nullptr;
-
-  float acc[kMaxHeads][8];
-#pragma unroll
-  for (int j = 0; j < kMaxHeads; ++j)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) acc[j][c] = 0.0f;
-
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  for (int r0 = r_begin; r0 < r_end; r0 += T) {
-    const int rows = min(T, r_end - r0);
-    __syncthreads();
-    dequant_tile(s, crow, srow, r0, rows, T, hrow);
-    __syncthreads();
-    // scores: warp per row
-    for (int rr = warp; rr < T; rr += nwarps) {
-      float part[kMaxHeads];
-#pragma unroll
-      for (int j = 0; j < kMaxHeads; ++j) part[j] = 0.0f;
-      for (int k = lane; k < d; k += 32) {
-        const float h = hrow[rr * d + k];
-#pragma unroll
-        for (int j = 0; j < kMaxHeads; ++j)
-          if (j < H) part[j] = fmaf(qt_sh[j * d + k], h, part[j]);
-      }
-#pragma unroll
-      for (int j = 0; j < kMaxHeads; ++j) {
-        float v = part[j];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0) sc[rr * kMaxHeads + j] = (rr < rows) ? v : -CUDART_INF_F;
-      }
-    }
-    __syncthreads();
-    if (threadIdx.x < kMaxHeads) {
-      const int j = threadIdx.x;
-      float mt = m_sh[j];
-      for (int rr = 0; rr < rows; ++rr) mt = fmaxf(mt, sc[rr * kMaxHeads + j]);
-      const float alpha = exp2f(m_sh[j] - mt);  // m_sh = -inf on the first tile -> 0
-      float lsum = l_sh[j] * alpha;
-      for (int rr = 0; rr < T; ++rr) {
-        const float p = rr < rows ? exp2f(sc[rr * kMaxHeads + j] - mt) : 0.0f;
-        sc[rr * kMaxHeads + j] = p;
-        lsum += p;
-      }
-      m_sh[j] = mt;
-      l_sh[j] = lsum;
-      a_sh[j] = alpha;
-    }
-    __syncthreads();
-    const int col0 = threadIdx.x * 8;
-#pragma unroll
-    for (int j = 0; j < kMaxHeads; ++j) {
-      if (j < H) {
-        const float alpha = a_sh[j];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) acc[j][c] *= alpha;
-      }
-    }
-    for (int rr = 0; rr < rows; ++rr) {
-      float h[8];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) h[c] = hrow[rr * d + col0 + c];
-#pragma unroll
-      for (int j = 0; j < kMaxHeads; ++j) {
-        if (j < H) {
-          const float p = sc[rr * kMaxHeads + j];
-#pragma unroll
-          for (int c = 0; c < 8; ++c) acc[j][c] = fmaf(p, h[c], acc[j][c]);
-        }
-      }
-    }
-  }
-  __syncthreads();
-  const size_t part = (size_t)b * s_max + split;
-  if (threadIdx.x < kMaxHeads) {
-    ml[(part * kMaxHeads + threadIdx.x) * 2 + 0] = m_sh[threadIdx.x];
-    ml[(part * kMaxHeads + threadIdx.x) * 2 + 1] = l_sh[threadIdx.x];
-  }
-  const int col0 = threadIdx.x * 8;
-#pragma unroll
-  for (int j = 0; j < kMaxHeads; ++j) {
-    if (j < H) {
-      float4* dst = reinterpret_cast<float4*>(U + (part * kMaxHeads + j) * d + col0);
-      dst[0] = make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
-      dst[1] = make_float4(acc[j][4], acc[j][5], acc[j][6], acc[j][7]);
-    }
-  }
-}
-
 // ------------------------------------------------------------------ epilogue
 // Block (head j, group of 8 lanes): merge the lane's splits exactly into
 // u = sum_s 2^(m_s - M) U_s / sum_s 2^(m_s - M) l_s, then out_j = W_v[j] u.
@@ -336,22 +190,6 @@ cudaError_t launch_prologue(const DecodeArgs& a, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   qt_kernel<<<dim3(s.d / kQtThreads, kMaxHeads), kQtThreads, 0, st>>>(s, a.iter, a.loops, a.ctx_len, a.Wk, q, qt,
                                                                         a.n_lanes);
-  count_launch();
-  return cudaGetLastError();
-}
-
-cudaError_t launch_stream(const DecodeArgs& a, cudaStream_t st) {
-  const Shape& s = a.s;
-  const int T = 8;
-  const size_t sm = (size_t)kMaxHeads * s.d * 4 + (size_t)T * s.d * 4 + (size_t)T * kMaxHeads * 4 + 3 * kMaxHeads * 4;
-  cudaError_t e = cudaFuncSetAttribute(stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-  if (e != cudaSuccess) return e;
-  dim3 grid(a.wl.s_max, a.n_lanes);
-  stream_kernel<<<grid, s.d / 8, sm, st>>>(s, a.iter, a.loops, a.ctx_len, (const uint8_t*)a.codes,
-                                           (const uint8_t*)a.scales,
-                                           reinterpret_cast<const float*>(a.ws + a.wl.qt_off),
-                                           reinterpret_cast<float*>(a.ws + a.wl.ml_off),
-                                           reinterpret_cast<float*>(a.ws + a.wl.u_off), a.wl.s_max, T);
   count_launch();
   return cudaGetLastError();
 }
