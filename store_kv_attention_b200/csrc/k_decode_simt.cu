@@ -4,7 +4,7 @@
 //  Features, "Store-h KV cache", "Variable-L KV cache", "L-aware batching"]
 //
 // Absorbed form of K = W_k h, V = W_v h for one loop iteration i, layer n_pre+i:
-//   prologue : q = W_q h_new ; qt_j = W_k[j]^T q_j * log2(e)/sqrt(hd)   (fp32, workspace)
+//   prologue : q = W_q h_new ; qt_j = W_k[j]^T q_j * log2(e)/sqrt(hd)   (fp16 operand image, workspace)
 //   stream   : (tensor cores, k_stream_tc.cu) per (lane, split): s_cj = qt_j . h_c ;
 //              online softmax in base 2 ; U_j = sum_c 2^(s_cj - m_j) h_c  (partials m, l, U)
 //   epilogue : merge the splits of a lane exactly ; u_j = U_j / l_j ; out_j = W_v[j] u_j
@@ -78,28 +78,35 @@ __global__ void __launch_bounds__(kQWarps * 32) q_kernel(Shape s, int iter, cons
 }
 
 // ------------------------------------------------------------------ prologue: qt
-// qt[b][j][c] = sum_{r<hd} W_k[j*hd + r][c] * q[b][j*hd + r], times log2(e)/sqrt(hd), in fp32.
-// Block (column block, head j); thread = column c.  Heads j >= H are written as 0.
+// qt[b][j][c] = sum_{r<hd} W_k[j*hd + r][c] * q[b][j*hd + r], times log2(e)/sqrt(hd), in fp32,
+// written as the fp16 B-operand image of the tensor-core scores: row j = fp16(qt), and when the
+// operands are split, row 16 + j = fp16(qt - fp16(qt)); columns in the dequantised position order,
+// 128-byte swizzled atom-columns.  Heads j >= H are zero rows.
 constexpr int kQtThreads = 256;
 
 __global__ void __launch_bounds__(kQtThreads) qt_kernel(Shape s, int iter, const int32_t* __restrict__ loops,
                                                         const int32_t* __restrict__ ctx_len,
                                                         const __half* __restrict__ Wk, const float* __restrict__ q,
-                                                        float* __restrict__ qt, int n_lanes) {
+                                                        uint8_t* __restrict__ qimg, int n_lanes) {
   const int c = blockIdx.x * kQtThreads + threadIdx.x;
   const int j = blockIdx.y;
-  if (j >= s.H) {
-    for (int b = 0; b < n_lanes; ++b) qt[((size_t)b * kMaxHeads + j) * s.d + c] = 0.0f;
-    return;
-  }
+  const int rows = qimg_rows(s.d);
+  const bool split = split_operands(s.d);
+  const int pos = phys_pos(s.fmt, c);
   const float scale = 1.4426950408889634f / sqrtf((float)s.hd);
   for (int b = 0; b < n_lanes; ++b) {
     int n;
     if (!lane_active(s, iter, loops, ctx_len, b, &n)) continue;
     float acc = 0.0f;
-    const float* qj = q + (size_t)b * s.d + j * s.hd;
-    for (int r = 0; r < s.hd; ++r) acc = fmaf(__half2float(Wk[(size_t)(j * s.hd + r) * s.d + c]), qj[r], acc);
-    qt[((size_t)b * kMaxHeads + j) * s.d + c] = acc * scale;
+    if (j < s.H) {
+      const float* qj = q + (size_t)b * s.d + j * s.hd;
+      for (int r = 0; r < s.hd; ++r) acc = fmaf(__half2float(Wk[(size_t)(j * s.hd + r) * s.d + c]), qj[r], acc);
+      acc *= scale;
+    }
+    uint8_t* img = qimg + (size_t)b * qimg_bytes(s.d);
+    const __half hi = __float2half_rn(acc);
+    *reinterpret_cast<__half*>(img + kmajor_offset(j, pos, rows)) = hi;
+    if (split) *reinterpret_cast<__half*>(img + kmajor_offset(16 + j, pos, rows)) = __float2half_rn(acc - __half2float(hi));
   }
 }
 
@@ -181,7 +188,7 @@ __global__ void __launch_bounds__(kEpiThreads) epilogue_kernel(Shape s, int iter
 cudaError_t launch_prologue(const DecodeArgs& a, cudaStream_t st) {
   const Shape& s = a.s;
   float* q = reinterpret_cast<float*>(a.ws + a.wl.q_off);
-  float* qt = reinterpret_cast<float*>(a.ws + a.wl.qt_off);
+  uint8_t* qt = a.ws + a.wl.qt_off;
   uint32_t* status = reinterpret_cast<uint32_t*>(a.ws + a.wl.status_off);
   q_kernel<<<(s.d + kQWarps - 1) / kQWarps, kQWarps * 32, 0, st>>>(s, a.iter, a.loops, a.ctx_len, a.h_new, a.Wq, q,
                                                                   a.n_lanes, status);

@@ -13,11 +13,14 @@
 // U^T accumulates in TMEM over the whole split; the (m, l, U) partial goes to
 // the workspace and is merged exactly by the epilogue kernel.
 //
-// Warp roles (192 threads): warp 0 = TMA producer, warp 1 = MMA issuer (and TMEM
-// owner), warps 2-5 = 128 math threads, one per tile row / TMEM lane, which
-// dequantise (twice: once into TMEM for the scores, once into shared memory
-// for P.V, re-reading the codes tile, which is then still in L2), run the
-// online softmax in base 2, and write the partial at the end.
+// Warp roles (320 threads): warp 0 = TMA producer, warp 1 = MMA issuer (and TMEM
+// owner), warps 2-9 = math: two warps per TMEM lane quarter, one for the even and
+// one for the odd 128-value units of every row and for heads 0-7 / 8-15 in the
+// softmax.  The math warps dequantise each tile twice (into TMEM for the scores,
+// into shared memory for P.V, re-reading the codes tile, which is then still in
+// L2), run the online softmax in base 2, and write the partial at the end.
+// The absorbed query arrives as a ready-made fp16 operand image (written by the
+// prologue) through one bulk copy.
 //
 // Codes tiles arrive through a ring of 16 KB slots (128 rows x 128 bytes,
 // 128-byte swizzle) loaded by TMA; every row of a slot is read by its own
@@ -52,13 +55,15 @@ namespace {
 
 using namespace ptx;
 
-constexpr int kMathThreads = 128;
+constexpr int kMathWarps = 8;                  // two per TMEM lane quarter
+constexpr int kMathThreads = 32 * kMathWarps;
 constexpr int kThreads = 64 + kMathThreads;
-constexpr int kSlotBytes = 128 * 128;    // one ring slot: 128 rows x 128 bytes
-constexpr int kPvStageBytes = 128 * 256; // 128 rows x 128 fp16 values
-constexpr int kScaleRowWords = 17;          // 16 words of INT4 group scales (d <= 2048) + 1 of padding
-constexpr int kScaleBytes = 128 * kScaleRowWords * 4;
-constexpr long long kWaitLimit = 4000000000ll;  // ~2 s of SM clocks, far beyond any legitimate wait
+constexpr int kRing = 4;                       // codes ring slots
+constexpr int kSlotBytes = 128 * 128;          // one ring slot: 128 rows x 128 bytes
+constexpr int kPvStageBytes = 128 * 256;       // 128 rows x 128 fp16 values
+constexpr int kScaleRowWords = 17;             // 16 words of INT4 group scales (d <= 2048) + 1 of padding
+constexpr int kScaleBytes = 2 * 128 * kScaleRowWords * 4;  // one copy per half
+constexpr long long kWaitLimit = 4000000000ll; // ~2 s of SM clocks, far beyond any legitimate wait
 
 template <int FMT>
 struct Fmt {
@@ -71,31 +76,40 @@ struct StreamParams {
   const int32_t* loops;
   const int32_t* ctx_len;
   const uint8_t* scales;
-  const float* qt;   // fp32 [n_lanes][16][d]
-  float* ml;         // [n_lanes][s_max][16][2]
-  float* U;          // [n_lanes][s_max][16][d]
+  const uint8_t* qimg;  // [n_lanes][qimg_bytes(d)] absorbed-query operand images
+  float* ml;            // [n_lanes][s_max][16][2]
+  float* U;             // [n_lanes][s_max][16][d]
   uint32_t* status;
   int s_max;
-  int ring;          // ring slots
 };
 
 struct __align__(8) Bars {
-  uint64_t ring_full[8], ring_empty[8];
+  uint64_t ring_full[kRing], ring_empty[kRing];
   uint64_t stg_full[2], stg_empty[2];
   uint64_t pv_full[2], pv_empty[2];
-  uint64_t s_full, s_empty, p_full, p_empty, u_done, fin;
+  uint64_t q_full, s_full, s_empty, p_full, p_empty, u_done, fin;
 };
-
-// Position p (0..7) inside an INT4 word holds element e = (p >> 1) + 4 * (p & 1).
-template <int FMT>
-__device__ __forceinline__ int logical_d(int pos) {
-  if (FMT != TL_H_INT4_G64) return pos;
-  const int p = pos & 7;
-  return (pos & ~7) + (p >> 1) + 4 * (p & 1);
-}
 
 __device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 bits_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t* v) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+               : "r"(taddr)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(v[0]),
+               "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
+}
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_addr(dst)),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_addr(bar))
+               : "memory");
+}
 
 // Dequantise one 16-byte vector of codes into fp16 pairs.
 // FP16: 8 values -> 4 regs; INT8: 16 values -> 8 regs; INT4: 32 values -> 16 regs.
@@ -135,23 +149,20 @@ __device__ __forceinline__ void dequant_vec(const uint4 v, uint32_t* out, __half
   }
 }
 
-// Byte address of K-position `pos` of row `row` in a K-major, 128-byte-swizzled
-// operand made of atom-columns of 64 fp16 values, each atom-column `rows` high.
-__device__ __forceinline__ uint32_t kmajor_offset(int row, int pos, int rows) {
-  const int a = pos >> 6, c = pos & 63;
-  return (uint32_t)(a * rows * 128 + row * 128 + ((((c >> 3) ^ (row & 7)) << 4) | ((c & 7) << 1)));
-}
-
 template <int FMT, bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
     stream_tc_kernel(const __grid_constant__ CUtensorMap tmap, const StreamParams p) {
   constexpr int NS = SPLIT ? 32 : 16;  // score columns (heads, or hi/lo x heads)
   constexpr int NP = SPLIT ? 32 : 16;  // P.V columns
   constexpr int kVals = Fmt<FMT>::kVals;
+  constexpr int kRegsPerVec = kVals / 16;  // fp16 pairs per 16-byte code vector
+  // ring-slot readers: an INT4 chunk holds two units, one per half; other formats: one half reads it
+  constexpr int kSlotReaders = FMT == TL_H_INT4_G64 ? kMathWarps : kMathWarps / 2;
+  constexpr int kChunksPerUnit = FMT == TL_H_FP16 ? 2 : 1;
+  constexpr int kVecs = FMT == TL_H_INT4_G64 ? 4 : 8;  // vectors of one chunk used by one unit
   constexpr uint32_t kIdS = idesc_f16_f32(128, NS, false, false);
   constexpr uint32_t kIdP = idesc_f16_f32(128, NP, true, false);
-  // TMEM columns
-  constexpr uint32_t kColS = 0, kColStg = 64, kColU = 256;
+  constexpr uint32_t kColS = 0, kColStg = 64, kColU = 256;  // TMEM columns
 
   const Shape& s = p.s;
   const int D = s.d;
@@ -165,28 +176,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (r_begin >= n) return;
   const int r_end = min(n, r_begin + kSplitRows);
   const int n_tiles = (r_end - r_begin + 127) >> 7;
-  const int n_units = D >> 7;
+  const int n_units = D >> 7;  // even: d is a multiple of 256
   const int n_chunks = D / kVals;
   const int layer = s.n_pre + p.iter;
   const int row_base = (layer * s.max_lanes + b) * s.max_ctx;
+  const uint32_t qbytes = (uint32_t)(NS * D * 2);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
   uint8_t* ring = base;
-  uint8_t* qs = ring + p.ring * kSlotBytes;   // NS x D fp16, K-major swizzled atom-columns
-  uint8_t* pvs = qs + NS * D * 2;            // 2 x [128 rows x 128 fp16]
+  uint8_t* qs = ring + kRing * kSlotBytes;    // NS x D fp16, K-major swizzled atom-columns
+  uint8_t* pvs = qs + qbytes;                // 2 x [128 rows x 128 fp16]
   uint8_t* ps = pvs + 2 * kPvStageBytes;     // NP x 128 fp16, K-major swizzled
-  uint32_t* scs = reinterpret_cast<uint32_t*>(ps + NP * 256);  // INT4: [128][17] words of group scales
+  uint32_t* scs = reinterpret_cast<uint32_t*>(ps + NP * 256);  // INT4: [2][128][17] words of group scales
   __shared__ Bars bars;
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
-  __shared__ float red[4][16];
+  __shared__ float red[2][4][8];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < p.ring; ++i) {
+    for (int i = 0; i < kRing; ++i) {
       mbar_init(&bars.ring_full[i], 1);
-      mbar_init(&bars.ring_empty[i], 4);
+      mbar_init(&bars.ring_empty[i], kSlotReaders);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.stg_full[i], 4);
@@ -194,9 +206,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars.pv_full[i], 4);
       mbar_init(&bars.pv_empty[i], 1);
     }
+    mbar_init(&bars.q_full, 1);
     mbar_init(&bars.s_full, 1);
-    mbar_init(&bars.s_empty, 4);
-    mbar_init(&bars.p_full, 4);
+    mbar_init(&bars.s_empty, kMathWarps);
+    mbar_init(&bars.p_full, kMathWarps);
     mbar_init(&bars.p_empty, 1);
     mbar_init(&bars.u_done, 1);
     mbar_init(&bars.fin, 1);
@@ -217,37 +230,41 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
+      // the lane's absorbed-query operand image, straight into place
+      mbar_expect_tx(&bars.q_full, qbytes);
+      const uint8_t* qsrc = p.qimg + (size_t)b * qbytes;
+      for (uint32_t off = 0; off < qbytes; off += 16384) bulk_load(qs + off, qsrc + off, 16384, &bars.q_full);
       // first pass over a tile: keep it in L2 for the second (P.V) pass; second pass: last use
-      const uint64_t pol_first = l2_policy_evict_first();
-      const uint64_t pol_normal = l2_policy_evict_normal();
-      int slot = 0, use = 0, issued = 0;
+      const uint64_t pol_last_use = l2_policy_evict_first();
+      const uint64_t pol_keep = l2_policy_evict_normal();
+      int issued = 0;
       bool ok = true;
       for (int t = 0; t < n_tiles && ok; ++t) {
         const int gy = row_base + r_begin + t * 128;
         for (int ph = 0; ph < 2 && ok; ++ph) {
-          for (int c = 0; c < n_chunks; ++c) {
+          for (int c = 0; c < n_chunks; ++c, ++issued) {
+            const int slot = issued & (kRing - 1), use = issued / kRing;
             if (use > 0 && !mbar_wait(&bars.ring_empty[slot], (use - 1) & 1, abort_p, kWaitLimit)) {
               ok = false;
               break;
             }
             mbar_expect_tx(&bars.ring_full[slot], kSlotBytes);
             tma_load_2d(ring + slot * kSlotBytes, &tmap, c * 128, gy, &bars.ring_full[slot],
-                        ph == 0 ? pol_normal : pol_first);
-            ++issued;
-            if (++slot == p.ring) {
-              slot = 0;
-              ++use;
-            }
+                        ph == 0 ? pol_keep : pol_last_use);
           }
         }
       }
+      {
+        // every load issued must land before the CTA's shared memory goes away
+        const long long t0 = clock64();
+        while (!mbar_try_wait(&bars.q_full, 0) && clock64() - t0 < kWaitLimit) {
+        }
+      }
       if (!ok) {
-        // let the loads already issued land before the CTA's shared memory goes away
-        const int first = issued > p.ring ? issued - p.ring : 0;
+        const int first = issued > kRing ? issued - kRing : 0;
         for (int g = first; g < issued; ++g) {
-          const int sl = g % p.ring, u = g / p.ring;
           const long long t0 = clock64();
-          while (!mbar_try_wait(&bars.ring_full[sl], u & 1) && clock64() - t0 < kWaitLimit) {
+          while (!mbar_try_wait(&bars.ring_full[g & (kRing - 1)], (g / kRing) & 1) && clock64() - t0 < kWaitLimit) {
           }
         }
       }
@@ -256,13 +273,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t qs_a = smem_addr(qs), pvs_a = smem_addr(pvs), ps_a = smem_addr(ps);
-      int gs = 0, gp = 0;  // staging buffer counters (scores, P.V)
-      bool ok = true;
+      bool ok = mbar_wait(&bars.q_full, 0, abort_p, kWaitLimit);
       bool issued_any = false;
       for (int t = 0; t < n_tiles && ok; ++t) {
         if (t > 0 && !mbar_wait(&bars.s_empty, (t - 1) & 1, abort_p, kWaitLimit)) { ok = false; break; }
-        for (int u = 0; u < n_units; ++u, ++gs) {
-          const int x = gs & 1;
+        for (int u = 0; u < n_units; ++u) {
+          const int gs = t * n_units + u, x = u & 1;
           if (!mbar_wait(&bars.stg_full[x], (gs >> 1) & 1, abort_p, kWaitLimit)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
@@ -279,8 +295,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(&bars.s_full);
         if (!mbar_wait(&bars.p_full, t & 1, abort_p, kWaitLimit)) { ok = false; break; }
         tc_fence_after();
-        for (int u = 0; u < n_units; ++u, ++gp) {
-          const int x = gp & 1;
+        for (int u = 0; u < n_units; ++u) {
+          const int gp = t * n_units + u, x = u & 1;
           if (!mbar_wait(&bars.pv_full[x], (gp >> 1) & 1, abort_p, kWaitLimit)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
@@ -306,90 +322,91 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ math warps
+    // half 0 (warps 2-5) takes the even units and heads 0-7, half 1 (warps 6-9) the odd
+    // units and heads 8-15; in each half, warp w owns TMEM lanes / tile rows 32*(w%4) ..
     const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;          // tile row == TMEM lane of this thread
+    const int half = (warp - 2) >> 2;
+    const int r = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const float* qt = p.qt + (size_t)b * kMaxHeads * D;
-    uint32_t* sc_row = scs + r * kScaleRowWords;
-    // absorbed query -> shared memory (fp16, or hi + lo), positions in the dequantised order
-    for (int i = r; i < 16 * D; i += kMathThreads) {
-      const int j = i / D, pos = i % D;
-      const float v = qt[(size_t)j * D + logical_d<FMT>(pos)];
-      const __half hi = __float2half_rn(v);
-      *reinterpret_cast<__half*>(qs + kmajor_offset(j, pos, NS)) = hi;
-      if (SPLIT) *reinterpret_cast<__half*>(qs + kmajor_offset(16 + j, pos, NS)) = __float2half_rn(v - __half2float(hi));
-    }
-    fence_proxy_async_smem();
+    const int h0 = half * 8;  // first head of this half
+    uint32_t* sc_row = scs + (half * 128 + r) * kScaleRowWords;
+    const uint8_t* my_row = ring + r * 128;
+    const int xr = r & 7;
 
-    float m_used[16], l_part[16];
+    float m_used[8], l_part[8];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
+    for (int j = 0; j < 8; ++j) {
       m_used[j] = -CUDART_INF_F;
       l_part[j] = 0.0f;
     }
-    int slot = 0, use = 0;  // ring consumer position
-    int gs = 0, gp = 0;
     bool ok = true;
-    const uint8_t* scales_row0 = p.scales;
+
+    // scales of a tile's rows (INT8: one fp32; INT4: d/64 fp16, up to 16 words), fetched a tile ahead
+    float scale_next = 0.0f;
+    uint4 scv_next[4];
+    auto fetch_scales = [&](int t_next) {
+      const int row0n = r_begin + t_next * 128;
+      const bool vn = r < (r_end - row0n);
+      const size_t grown = (size_t)row_base + row0n + r;
+      if (FMT == TL_H_INT8_TOKEN) scale_next = vn ? reinterpret_cast<const float*>(p.scales)[grown] : 0.0f;
+      if (FMT == TL_H_INT4_G64) {
+        const uint4* src = reinterpret_cast<const uint4*>(p.scales + grown * (size_t)(D / kInt4Group) * 2);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) scv_next[i] = (vn && i * 8 < D / kInt4Group) ? src[i] : make_uint4(0, 0, 0, 0);
+      }
+    };
+    fetch_scales(0);
 
     for (int t = 0; t < n_tiles && ok; ++t) {
       const int row0 = r_begin + t * 128;
       const bool valid = r < (r_end - row0);
-      const size_t grow = (size_t)row_base + row0 + r;
-      // row scale(s)
-      float scale_row = 0.0f;
-      if (FMT == TL_H_INT8_TOKEN) {
-        scale_row = valid ? reinterpret_cast<const float*>(scales_row0)[grow] : 0.0f;
-      }
+      const float scale_row = scale_next;
       if (FMT == TL_H_INT4_G64) {
-        // this row's fp16 group scales, two per word, into the thread's own padded smem row
-        const uint4* src = reinterpret_cast<const uint4*>(scales_row0 + grow * (size_t)(D / kInt4Group) * 2);
-        const int nvec = D / (kInt4Group * 8);  // 16-byte vectors of scales per row
-        for (int i = 0; i < nvec; ++i) {
-          const uint4 v = valid ? src[i] : make_uint4(0, 0, 0, 0);
-          sc_row[4 * i + 0] = v.x;
-          sc_row[4 * i + 1] = v.y;
-          sc_row[4 * i + 2] = v.z;
-          sc_row[4 * i + 3] = v.w;
+        // into this thread's own padded smem row (read back one word per unit)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          sc_row[4 * i + 0] = scv_next[i].x;
+          sc_row[4 * i + 1] = scv_next[i].y;
+          sc_row[4 * i + 2] = scv_next[i].z;
+          sc_row[4 * i + 3] = scv_next[i].w;
         }
       }
 
       for (int ph = 0; ph < 2 && ok; ++ph) {
         if (ph == 1) {
-          // ------------------------------------------------ softmax of this tile, then P
+          // ------------------------------------------------ softmax of this tile (this half's heads), then P
           if (!mbar_wait(&bars.s_full, t & 1, abort_p, kWaitLimit)) { ok = false; break; }
           tc_fence_after();
-          uint32_t sv[32];
-          tmem_ld16(tbase + lane_off + kColS, sv);
-          if (NS == 32) tmem_ld16(tbase + lane_off + kColS + 16, sv + 16);
+          uint32_t sv[16];
+          tmem_ld8(tbase + lane_off + kColS + h0, sv);
+          if (NS == 32) tmem_ld8(tbase + lane_off + kColS + 16 + h0, sv + 8);
           tmem_ld_wait();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&bars.s_empty);
-          float sc[16];
+          float sc[8];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
+          for (int j = 0; j < 8; ++j) {
             float v = __uint_as_float(sv[j]);
-            if (NS == 32) v += __uint_as_float(sv[16 + j]);
+            if (NS == 32) v += __uint_as_float(sv[8 + j]);
             if (FMT == TL_H_INT8_TOKEN) v *= scale_row;
             sc[j] = valid ? v : -CUDART_INF_F;
           }
-          // tile maximum per head over the 128 rows
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
+          for (int j = 0; j < 8; ++j) {
             float v = sc[j];
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-            if (lane == 0) red[quarter][j] = v;
+            if (lane == 0) red[half][quarter][j] = v;
           }
-          named_bar_sync(1, kMathThreads);
-          float alpha[16];
+          named_bar_sync(1 + half, 128);
+          float alpha[8];
           bool rescale = false;
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float tm = fmaxf(fmaxf(red[0][j], red[1][j]), fmaxf(red[2][j], red[3][j]));
+          for (int j = 0; j < 8; ++j) {
+            const float tm = fmaxf(fmaxf(red[half][0][j], red[half][1][j]), fmaxf(red[half][2][j], red[half][3][j]));
             alpha[j] = 1.0f;
-            if (tm > m_used[j] + 8.0f) {  // lazy rescale: P stays <= 2^8 otherwise
+            if (tm > m_used[j] + 8.0f) {  // lazy rescale: P stays below 2^8 otherwise
               if (m_used[j] != -CUDART_INF_F) {
                 alpha[j] = exp2f(m_used[j] - tm);
                 rescale = true;
@@ -397,10 +414,10 @@ __global__ void __launch_bounds__(kThreads, 1)
               m_used[j] = tm;
             }
           }
-          named_bar_sync(1, kMathThreads);  // red is reused by the next tile
-          float pr[16];
+          named_bar_sync(1 + half, 128);  // red is rewritten by the next tile
+          float pr[8];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
+          for (int j = 0; j < 8; ++j) {
             pr[j] = valid ? exp2f(sc[j] - m_used[j]) : 0.0f;
             l_part[j] = l_part[j] * alpha[j] + pr[j];
           }
@@ -408,73 +425,69 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (t > 0 && !mbar_wait(&bars.p_empty, (t - 1) & 1, abort_p, kWaitLimit)) { ok = false; break; }
           tc_fence_after();
           if (rescale) {
-            // rare: the running maximum rose by more than 2^8; rescale U^T in TMEM
+            // rare: the running maximum rose by more than 2^8; rescale this half's columns of U^T
             for (int u = 0; u < n_units; ++u) {
-              uint32_t uv[32];
-              tmem_ld16(tbase + lane_off + kColU + u * NP, uv);
-              if (NP == 32) tmem_ld16(tbase + lane_off + kColU + u * NP + 16, uv + 16);
+              uint32_t uv[16];
+              tmem_ld8(tbase + lane_off + kColU + u * NP + h0, uv);
+              if (NP == 32) tmem_ld8(tbase + lane_off + kColU + u * NP + 16 + h0, uv + 8);
               tmem_ld_wait();
 #pragma unroll
-              for (int c = 0; c < NP; ++c) uv[c] = __float_as_uint(__uint_as_float(uv[c]) * alpha[c & 15]);
-              tmem_st16(tbase + lane_off + kColU + u * NP, uv);
-              if (NP == 32) tmem_st16(tbase + lane_off + kColU + u * NP + 16, uv + 16);
+              for (int c = 0; c < 16; ++c) uv[c] = __float_as_uint(__uint_as_float(uv[c]) * alpha[c & 7]);
+              tmem_st8(tbase + lane_off + kColU + u * NP + h0, uv);
+              if (NP == 32) tmem_st8(tbase + lane_off + kColU + u * NP + 16 + h0, uv + 8);
             }
             tmem_st_wait();
           }
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
+          for (int j = 0; j < 8; ++j) {
             const float v = FMT == TL_H_INT8_TOKEN ? pr[j] * scale_row : pr[j];
             const __half hi = __float2half_rn(v);
-            *reinterpret_cast<__half*>(ps + kmajor_offset(j, r, NP)) = hi;
-            if (NP == 32) *reinterpret_cast<__half*>(ps + kmajor_offset(16 + j, r, NP)) = __float2half_rn(v - __half2float(hi));
+            *reinterpret_cast<__half*>(ps + kmajor_offset(h0 + j, r, NP)) = hi;
+            if (NP == 32)
+              *reinterpret_cast<__half*>(ps + kmajor_offset(16 + h0 + j, r, NP)) = __float2half_rn(v - __half2float(hi));
           }
           fence_proxy_async_smem();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&bars.p_full);
+          if (t + 1 < n_tiles) fetch_scales(t + 1);  // lands while this tile's P.V operands are made
         }
 
-        // ------------------------------------------------ dequantise the tile, unit by unit
-        for (int u = 0; u < n_units && ok; ++u) {
+        // ------------------------------------------------ dequantise this half's units of the tile
+        const int gbase = (t * 2 + ph) * n_chunks;  // producer's load index of chunk 0 of this pass
+        for (int u = half; u < n_units && ok; u += 2) {
           uint32_t h[64];
-          constexpr int kVecPerUnit = 1024 / kVals;  // 16-byte vectors of codes per 128 values
-          // FP16: 16 vectors over 2 chunks; INT8: 8 vectors (1 chunk); INT4: 4 vectors (half a chunk)
+          uint32_t scw = 0;
+          if (FMT == TL_H_INT4_G64) scw = sc_row[u];  // fp16 scales of groups 2u (low) and 2u+1 (high)
 #pragma unroll
-          for (int v = 0; v < kVecPerUnit; ++v) {
-            const int vglob = u * kVecPerUnit + v;           // vector index within the row
-            const int vin = vglob & 7;                       // vector within its chunk
-            if (vin == 0 || v == 0) {
-              if (!mbar_wait(&bars.ring_full[slot], use & 1, abort_p, kWaitLimit)) { ok = false; break; }
-            }
-            const uint8_t* row = ring + slot * kSlotBytes + r * 128;
-            const uint4 cv = *reinterpret_cast<const uint4*>(row + ((vin ^ (r & 7)) << 4));
-            __half2 s2 = __halves2half2(__float2half_rn(1.0f), __float2half_rn(1.0f));
-            if (FMT == TL_H_INT4_G64) {
-              const int g = vglob >> 1;  // 32 values per vector, 64 per group
-              const uint32_t pair = sc_row[g >> 1];
-              const uint16_t sbits = (g & 1) ? (uint16_t)(pair >> 16) : (uint16_t)(pair & 0xFFFF);
-              s2 = bits_h2((uint32_t)sbits | ((uint32_t)sbits << 16));
-            }
-            constexpr int kRegsPerVec = 64 / kVecPerUnit;
-            dequant_vec<FMT>(cv, h + v * kRegsPerVec, s2);
-            if (vin == 7) {
-              // this thread is done with the slot
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&bars.ring_empty[slot]);
-              if (++slot == p.ring) {
-                slot = 0;
-                ++use;
+          for (int cc = 0; cc < kChunksPerUnit; ++cc) {
+            const int c = FMT == TL_H_INT4_G64 ? (u >> 1) : FMT == TL_H_INT8_TOKEN ? u : 2 * u + cc;
+            const int g = gbase + c;
+            const int slot = g & (kRing - 1);
+            if (!mbar_wait(&bars.ring_full[slot], (g / kRing) & 1, abort_p, kWaitLimit)) { ok = false; break; }
+            const uint8_t* src = my_row + slot * kSlotBytes;
+            const int v0 = FMT == TL_H_INT4_G64 ? (u & 1) * 4 : 0;
+#pragma unroll
+            for (int v = 0; v < kVecs; ++v) {
+              const uint4 cv = *reinterpret_cast<const uint4*>(src + (((v0 + v) ^ xr) << 4));
+              __half2 s2 = __halves2half2(__float2half_rn(1.0f), __float2half_rn(1.0f));
+              if (FMT == TL_H_INT4_G64) {
+                const uint32_t sbits = (v < 2) ? (scw & 0xFFFFu) : (scw >> 16);
+                s2 = bits_h2(sbits | (sbits << 16));
               }
+              dequant_vec<FMT>(cv, h + (cc * kVecs + v) * kRegsPerVec, s2);
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars.ring_empty[slot]);
           }
           if (!ok) break;
           if (!valid) {
 #pragma unroll
             for (int i = 0; i < 64; ++i) h[i] = 0u;
           }
+          const int gu = t * n_units + u, x = half;
           if (ph == 0) {
-            const int x = gs & 1;
-            if (gs >= 2 && !mbar_wait(&bars.stg_empty[x], ((gs >> 1) - 1) & 1, abort_p, kWaitLimit)) { ok = false; break; }
+            if (gu >= 2 && !mbar_wait(&bars.stg_empty[x], ((gu >> 1) - 1) & 1, abort_p, kWaitLimit)) { ok = false; break; }
             tc_fence_after();
             const uint32_t ta = tbase + lane_off + kColStg + x * 64;
             tmem_st16(ta + 0, h + 0);
@@ -485,53 +498,51 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars.stg_full[x]);
-            ++gs;
           } else {
-            const int x = gp & 1;
-            if (gp >= 2 && !mbar_wait(&bars.pv_empty[x], ((gp >> 1) - 1) & 1, abort_p, kWaitLimit)) { ok = false; break; }
+            if (gu >= 2 && !mbar_wait(&bars.pv_empty[x], ((gu >> 1) - 1) & 1, abort_p, kWaitLimit)) { ok = false; break; }
             uint8_t* st = pvs + x * kPvStageBytes + r * 128;
 #pragma unroll
             for (int v = 0; v < 16; ++v) {
-              uint4 val = make_uint4(h[4 * v], h[4 * v + 1], h[4 * v + 2], h[4 * v + 3]);
-              *reinterpret_cast<uint4*>(st + (v >> 3) * 16384 + (((v & 7) ^ (r & 7)) << 4)) = val;
+              const uint4 val = make_uint4(h[4 * v], h[4 * v + 1], h[4 * v + 2], h[4 * v + 3]);
+              *reinterpret_cast<uint4*>(st + (v >> 3) * 16384 + (((v & 7) ^ xr) << 4)) = val;
             }
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars.pv_full[x]);
-            ++gp;
           }
         }
       }
     }
 
-    // ------------------------------------------------ partial (m, l, U) of this split
+    // ------------------------------------------------ partial (m, l, U) of this split, this half's heads
     if (ok && mbar_wait(&bars.u_done, 0, abort_p, kWaitLimit)) {
       tc_fence_after();
       const size_t part = (size_t)b * p.s_max + split;
       for (int u = 0; u < n_units; ++u) {
-        uint32_t uv[32];
-        tmem_ld16(tbase + lane_off + kColU + u * NP, uv);
-        if (NP == 32) tmem_ld16(tbase + lane_off + kColU + u * NP + 16, uv + 16);
+        uint32_t uv[16];
+        tmem_ld8(tbase + lane_off + kColU + u * NP + h0, uv);
+        if (NP == 32) tmem_ld8(tbase + lane_off + kColU + u * NP + 16 + h0, uv + 8);
         tmem_ld_wait();
-        const int d = logical_d<FMT>(u * 128 + r);
+        const int d = logical_of_pos(FMT, u * 128 + r);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
+        for (int j = 0; j < 8; ++j) {
           float v = __uint_as_float(uv[j]);
-          if (NP == 32) v += __uint_as_float(uv[16 + j]);
-          if (j < s.H) p.U[(part * kMaxHeads + j) * D + d] = v;
+          if (NP == 32) v += __uint_as_float(uv[8 + j]);
+          if (h0 + j < s.H) p.U[(part * kMaxHeads + h0 + j) * D + d] = v;
         }
       }
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
+      for (int j = 0; j < 8; ++j) {
         float v = l_part[j];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0) red[quarter][j] = v;
+        if (lane == 0) red[half][quarter][j] = v;
       }
-      named_bar_sync(1, kMathThreads);
-      if (r < 16) {
-        p.ml[(part * kMaxHeads + r) * 2 + 0] = m_used[r];
-        p.ml[(part * kMaxHeads + r) * 2 + 1] = red[0][r] + red[1][r] + red[2][r] + red[3][r];
+      named_bar_sync(1 + half, 128);
+      if (r < 8) {
+        p.ml[(part * kMaxHeads + h0 + r) * 2 + 0] = m_used[r];
+        p.ml[(part * kMaxHeads + h0 + r) * 2 + 1] =
+            red[half][0][r] + red[half][1][r] + red[half][2][r] + red[half][3][r];
       }
     }
   }
@@ -562,13 +573,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 template <int FMT, bool SPLIT>
 cudaError_t launch_fmt(const DecodeArgs& a, const CUtensorMap& tmap, cudaStream_t st) {
   const Shape& s = a.s;
-  constexpr int NS = SPLIT ? 32 : 16, NP = SPLIT ? 32 : 16;
-  const size_t fixed = (size_t)NS * s.d * 2 + 2 * kPvStageBytes + (size_t)NP * 256 + kScaleBytes + 1024;  // + align
-  const size_t budget = 225 * 1024;  // 227 KB minus the static shared variables
-  int ring = (int)((budget - fixed) / kSlotBytes);
-  ring = ring > 8 ? 8 : ring;
-  if (ring < 2) return cudaErrorInvalidConfiguration;
-  const size_t smem = fixed + (size_t)ring * kSlotBytes;
+  constexpr int NP = SPLIT ? 32 : 16;
+  const size_t smem = qimg_bytes(s.d) + 2 * kPvStageBytes + (size_t)NP * 256 + kScaleBytes + 1024 +  // + align
+                      (size_t)kRing * kSlotBytes;
+  if (smem > 225 * 1024) return cudaErrorInvalidConfiguration;
   cudaError_t e = cudaFuncSetAttribute(stream_tc_kernel<FMT, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
@@ -577,12 +585,11 @@ cudaError_t launch_fmt(const DecodeArgs& a, const CUtensorMap& tmap, cudaStream_
                  a.loops,
                  a.ctx_len,
                  (const uint8_t*)a.scales,
-                 reinterpret_cast<const float*>(a.ws + a.wl.qt_off),
+                 a.ws + a.wl.qt_off,
                  reinterpret_cast<float*>(a.ws + a.wl.ml_off),
                  reinterpret_cast<float*>(a.ws + a.wl.u_off),
                  reinterpret_cast<uint32_t*>(a.ws + a.wl.status_off),
-                 a.wl.s_max,
-                 ring};
+                 a.wl.s_max};
   dim3 grid(a.wl.s_max, a.n_lanes);
   stream_tc_kernel<FMT, SPLIT><<<grid, kThreads, smem, st>>>(tmap, p);
   count_launch();

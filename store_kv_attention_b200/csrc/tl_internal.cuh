@@ -35,6 +35,34 @@ struct Shape {
   __host__ __device__ size_t rows_total() const { return (size_t)layers() * max_lanes * max_ctx; }
 };
 
+// Operand precision of the tensor-core path: when d <= 1024 the absorbed query and
+// P are split into fp16 hi + lo parts (32 MMA columns instead of 16).
+__host__ __device__ inline bool split_operands(int d) { return d <= 1024; }
+__host__ __device__ inline int qimg_rows(int d) { return split_operands(d) ? 32 : 16; }
+__host__ __device__ inline size_t qimg_bytes(int d) { return (size_t)qimg_rows(d) * d * 2; }
+
+// Physical K position of logical d-index c in the dequantised operand order.
+// INT4 words are unpacked as pairs (e0,e4),(e1,e5),(e2,e6),(e3,e7): position p of a
+// group of 8 holds element (p >> 1) + 4 * (p & 1), so element e sits at 2 * (e & 3) + (e >> 2).
+__host__ __device__ inline int phys_pos(int fmt, int c) {
+  if (fmt != TL_H_INT4_G64) return c;
+  const int e = c & 7;
+  return (c & ~7) + 2 * (e & 3) + (e >> 2);
+}
+__host__ __device__ inline int logical_of_pos(int fmt, int pos) {
+  if (fmt != TL_H_INT4_G64) return pos;
+  const int p = pos & 7;
+  return (pos & ~7) + (p >> 1) + 4 * (p & 1);
+}
+
+// Byte offset of K-position `pos` of row `row` in a K-major, 128-byte-swizzled fp16
+// operand made of atom-columns of 64 values, each atom-column `rows` high
+// (the canonical layout of a UMMA operand with SWIZZLE_128B).
+__host__ __device__ inline uint32_t kmajor_offset(int row, int pos, int rows) {
+  const int a = pos >> 6, c = pos & 63;
+  return (uint32_t)(a * rows * 128 + row * 128 + ((((c >> 3) ^ (row & 7)) << 4) | ((c & 7) << 1)));
+}
+
 __host__ __device__ inline int splits_for_rows(int n_rows) { return (n_rows + kSplitRows - 1) / kSplitRows; }
 
 // ---------------------------------------------------------------- workspace layout
@@ -42,7 +70,7 @@ __host__ __device__ inline int splits_for_rows(int n_rows) { return (n_rows + kS
 struct Workspace {
   size_t status_off;   // uint32 status word (+ padding)
   size_t q_off;        // fp32 [n_lanes][d]       q = W_q h_new
-  size_t qt_off;       // fp32 [n_lanes][16][d]   absorbed query, scaled by log2(e)/sqrt(hd)
+  size_t qt_off;       // fp16 [n_lanes][qimg_rows(d) x d] absorbed query image (see k_stream_tc.cu)
   size_t ml_off;       // fp32 [n_lanes][S_max][16][2]   per-split running max and sum
   size_t u_off;        // fp32 [n_lanes][S_max][16][d]   per-split unnormalised sum_c p_c h_c
   size_t total;
@@ -60,7 +88,7 @@ inline Workspace workspace_layout(const Shape& s, int n_lanes) {
   w.q_off = off;
   off = align256(off + (size_t)n_lanes * s.d * 4);
   w.qt_off = off;
-  off = align256(off + (size_t)n_lanes * kMaxHeads * s.d * 4);
+  off = align256(off + (size_t)n_lanes * qimg_bytes(s.d));
   w.ml_off = off;
   off = align256(off + (size_t)n_lanes * w.s_max * kMaxHeads * 2 * 4);
   w.u_off = off;
