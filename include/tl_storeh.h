@@ -115,7 +115,8 @@ TL_API tl_status tl_storeh_cache_bytes(const tl_storeh_desc* desc, size_t* codes
 
 /* Bytes of device workspace tl_storeh_attn_decode needs for up to `n_lanes`
  * lanes (256-byte aligned, contents need no initialisation, must not be shared
- * by two calls in flight at once). */
+ * by two calls in flight at once).  One decode call takes at most 64 lanes
+ * (TL_ERR_UNSUPPORTED above); larger batches are split into several calls. */
 TL_API tl_status tl_storeh_workspace_bytes(const tl_storeh_desc* desc, int32_t n_lanes, size_t* bytes);
 
 /*

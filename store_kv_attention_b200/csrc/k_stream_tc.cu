@@ -272,7 +272,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t qs_a = smem_addr(qs), pvs_a = smem_addr(pvs), ps_a = smem_addr(ps);
+      // base descriptors; the address field is the low 14 bits of (address >> 4), so adding
+      // (byte offset >> 4) to a descriptor moves it within shared memory
+      const uint64_t q_desc0 = sdesc_sw128(smem_addr(qs), 16, 1024);
+      const uint64_t pv_desc0 = sdesc_sw128(smem_addr(pvs), 16384, 1024);
+      const uint64_t p_desc0 = sdesc_sw128(smem_addr(ps), 16, 1024);
       bool ok = mbar_wait(&bars.q_full, 0, abort_p, kWaitLimit);
       bool issued_any = false;
       for (int t = 0; t < n_tiles && ok; ++t) {
@@ -281,13 +285,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int gs = t * n_units + u, x = u & 1;
           if (!mbar_wait(&bars.stg_full[x], (gs >> 1) & 1, abort_p, kWaitLimit)) { ok = false; break; }
           tc_fence_after();
+          // descriptors of this unit's 8 K-steps differ from the first by compile-time byte offsets
+          const uint64_t bd = q_desc0 + (uint64_t)((u * 2 * NS * 128) >> 4);
+          const uint32_t ta = tbase + kColStg + x * 64;
+          if (u == 0)
+            mma_ts_first(tbase + kColS, ta, bd, kIdS);
+          else
+            mma_ts_acc(tbase + kColS, ta, bd, kIdS);
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const int pos = u * 128 + k * 16;
-            const uint32_t baddr = qs_a + (pos >> 6) * (NS * 128) + (pos & 63) * 2;
-            mma_ts(tbase + kColS, tbase + kColStg + x * 64 + k * 8, sdesc_sw128(baddr, 16, 1024), kIdS,
-                   (u > 0 || k > 0) ? 1u : 0u);
-          }
+          for (int k = 1; k < 8; ++k)
+            mma_ts_acc(tbase + kColS, ta + k * 8, bd + (uint64_t)(((k >> 2) * NS * 128 + (k & 3) * 32) >> 4), kIdS);
           issued_any = true;
           mma_commit(&bars.stg_empty[x]);
         }
@@ -299,13 +306,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int gp = t * n_units + u, x = u & 1;
           if (!mbar_wait(&bars.pv_full[x], (gp >> 1) & 1, abort_p, kWaitLimit)) { ok = false; break; }
           tc_fence_after();
+          const uint64_t ad = pv_desc0 + (uint64_t)((x * kPvStageBytes) >> 4);
+          const uint32_t du = tbase + kColU + u * NP;
+          if (t == 0)
+            mma_ss_first(du, ad, p_desc0, kIdP);
+          else
+            mma_ss_acc(du, ad, p_desc0, kIdP);
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const uint32_t aaddr = pvs_a + x * kPvStageBytes + k * 2048;
-            const uint32_t baddr = ps_a + ((k * 16) >> 6) * (NP * 128) + ((k * 16) & 63) * 2;
-            mma_ss(tbase + kColU + u * NP, sdesc_sw128(aaddr, 16384, 1024), sdesc_sw128(baddr, 16, 1024), kIdP,
-                   (t > 0 || k > 0) ? 1u : 0u);
-          }
+          for (int k = 1; k < 8; ++k)
+            mma_ss_acc(du, ad + (uint64_t)((k * 2048) >> 4),
+                       p_desc0 + (uint64_t)((((k * 16) >> 6) * NP * 128 + ((k * 16) & 63) * 2) >> 4), kIdP);
           mma_commit(&bars.pv_empty[x]);
         }
         if (!ok) break;

@@ -125,6 +125,8 @@ tl_status tl_storeh_workspace_bytes(const tl_storeh_desc* desc, int32_t n_lanes,
   if (!bytes) return fail(TL_ERR_INVALID_ARG, "bytes is NULL");
   if (n_lanes <= 0) return fail(TL_ERR_INVALID_ARG, "n_lanes %d <= 0", n_lanes);
   if (n_lanes > s.max_lanes) return fail(TL_ERR_CAPACITY, "n_lanes %d > max_lanes %d", n_lanes, s.max_lanes);
+  if (n_lanes > tl::kMaxGemmLanes)
+    return fail(TL_ERR_UNSUPPORTED, "n_lanes %d > %d lanes per decode call", n_lanes, tl::kMaxGemmLanes);
   *bytes = tl::workspace_layout(s, n_lanes).total;
   return TL_OK;
 }
@@ -180,6 +182,8 @@ tl_status tl_storeh_attn_decode(const tl_storeh_desc* desc, tl_storeh_cache cach
   if (n_lanes <= 0) return fail(TL_ERR_INVALID_ARG, "n_lanes %d <= 0", n_lanes);
   if (n_lanes > s.max_lanes) return fail(TL_ERR_CAPACITY, "n_lanes %d > max_lanes %d", n_lanes, s.max_lanes);
   if (iter < 0 || iter >= s.L_max) return fail(TL_ERR_CAPACITY, "iter %d outside [0, L_max=%d)", iter, s.L_max);
+  if (n_lanes > tl::kMaxGemmLanes)
+    return fail(TL_ERR_UNSUPPORTED, "n_lanes %d > %d lanes per decode call", n_lanes, tl::kMaxGemmLanes);
   if (residual && (!abort_flags || !first_abort_iter))
     return fail(TL_ERR_INVALID_ARG, "residual given without abort_flags / first_abort_iter");
   if (residual && !(threshold >= 0.0f)) return fail(TL_ERR_INVALID_ARG, "threshold must be a non-negative number");
