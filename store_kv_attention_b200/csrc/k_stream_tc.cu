@@ -13,18 +13,25 @@
 // U^T accumulates in TMEM over the whole split; the (m, l, U) partial goes to
 // the workspace and is merged exactly by the epilogue kernel.
 //
-// Warp roles (320 threads): warp 0 = TMA producer, warp 1 = MMA issuer (and TMEM
-// owner), warps 2-9 = math: two warps per TMEM lane quarter, one for the even and
-// one for the odd 128-value units of every row and for heads 0-7 / 8-15 in the
-// softmax.  The math warps dequantise each tile twice (into TMEM for the scores,
-// into shared memory for P.V, re-reading the codes tile, which is then still in
-// L2), run the online softmax in base 2, and write the partial at the end.
+// Warp roles (608 threads): warp 0 = TMA producer; warp 1 = score-MMA issuer
+// (and TMEM owner); warp 2 = P.V-MMA issuer; warps 3-10 = score group; warps
+// 11-18 = P.V group.  The two groups work on different tiles at the same time:
+// while the score group dequantises tile t+1 into TMEM (the A operand of the
+// score MMAs) and runs its online softmax, the P.V group dequantises tile t into
+// shared memory (the A operand of the P.V MMAs, which take tile t's P).  P is
+// double-buffered across tiles; the scores S are double-buffered in TMEM.
+// Score group: two warps per TMEM lane quarter, one for the even and one for the
+// odd 128-value units of each row, and for heads 0-7 / 8-15 in the softmax.
+// P.V group: two warps per 32-row block, one per 64-value half of every unit.
+// Each group reads the codes of a tile through its own TMA ring; the second
+// read of a tile (P.V) finds it in L2.  The online softmax runs in base 2 and
+// each split writes its partial (m, l, U) at the end.
 // The absorbed query arrives as a ready-made fp16 operand image (written by the
-// prologue) through one bulk copy.
+// prologue) through bulk copies.
 //
-// Codes tiles arrive through a ring of 16 KB slots (128 rows x 128 bytes,
-// 128-byte swizzle) loaded by TMA; every row of a slot is read by its own
-// math thread, conflict-free thanks to the swizzle.
+// Codes tiles arrive in 16 KB slots (128 rows x 128 bytes, 128-byte swizzle)
+// loaded by TMA; every row of a slot is read by its own thread, conflict-free
+// thanks to the swizzle.
 //
 // Precision: dequantised h is fp16 (INT8 keeps the exact integer codes and
 // applies the per-row scale to the scores and to P instead).  When the
@@ -45,6 +52,7 @@
 #include <cudaTypedefs.h>
 #include <math_constants.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "tc_ptx.cuh"
@@ -55,19 +63,32 @@ namespace {
 
 using namespace ptx;
 
-constexpr int kMathWarps = 8;                  // two per TMEM lane quarter
-constexpr int kMathThreads = 32 * kMathWarps;
-constexpr int kThreads = 64 + kMathThreads;
-constexpr int kRing = 4;                       // codes ring slots
-constexpr int kSlotBytes = 128 * 128;          // one ring slot: 128 rows x 128 bytes
-constexpr int kPvStageBytes = 128 * 256;       // 128 rows x 128 fp16 values
-constexpr int kScaleRowWords = 17;             // 16 words of INT4 group scales (d <= 2048) + 1 of padding
-constexpr int kScaleBytes = 2 * 128 * kScaleRowWords * 4;  // one copy per half
-constexpr long long kWaitLimit = 4000000000ll; // ~2 s of SM clocks, far beyond any legitimate wait
+constexpr int kSWarps = 8;                      // score group: two warps per TMEM lane quarter
+constexpr int kVWarps = 8;                      // P.V group: two warps per 32-row block
+constexpr int kWarpS0 = 3;                      // first score warp
+constexpr int kWarpV0 = kWarpS0 + kSWarps;      // first P.V warp
+constexpr int kThreads = 32 * (kWarpV0 + kVWarps);
+constexpr int kSlotBytes = 128 * 128;           // one ring slot: 128 rows x 128 bytes of codes
+constexpr int kPvStageBytes = 128 * 256;        // P.V operand staging: 128 rows x 128 fp16 values
+constexpr int kMaxRing = 4;                     // slots per ring at most
+constexpr long long kWaitLimit = 4000000000ll;  // ~2 s of SM clocks, far beyond any legitimate wait
 
 template <int FMT>
 struct Fmt {
   static constexpr int kVals = FMT == TL_H_FP16 ? 64 : FMT == TL_H_INT8_TOKEN ? 128 : 256;  // d-values per 128 B
+  // half-unit (64 values) hh of unit u: ring chunk, first 16-byte vector in it, vectors
+  __device__ static int chunk(int u, int hh) {
+    return FMT == TL_H_INT4_G64 ? (u >> 1) : FMT == TL_H_INT8_TOKEN ? u : 2 * u + hh;
+  }
+  __device__ static int vec0(int u, int hh) {
+    return FMT == TL_H_INT4_G64 ? (u & 1) * 4 + hh * 2 : FMT == TL_H_INT8_TOKEN ? hh * 4 : 0;
+  }
+  static constexpr int kVecs = FMT == TL_H_INT4_G64 ? 2 : FMT == TL_H_INT8_TOKEN ? 4 : 8;
+  // A score warp reads both halves of its own units: its last read of a chunk is half 1
+  // (FP16: every half is a chunk of its own).
+  __device__ static bool score_releases(int hh) { return FMT == TL_H_FP16 || hh == 1; }
+  // A P.V warp reads one half of every unit: INT4 chunks hold two units.
+  __device__ static bool pv_releases(int u) { return FMT != TL_H_INT4_G64 || (u & 1); }
 };
 
 struct StreamParams {
@@ -81,18 +102,34 @@ struct StreamParams {
   float* U;             // [n_lanes][s_max][16][d]
   uint32_t* status;
   int s_max;
+  int s_ring, v_ring;   // slots of the score-side and P.V-side rings
 };
 
 struct __align__(8) Bars {
-  uint64_t ring_full[kRing], ring_empty[kRing];
-  uint64_t stg_full[2], stg_empty[2];
-  uint64_t pv_full[2], pv_empty[2];
-  uint64_t q_full, s_full, s_empty, p_full, p_empty, u_done, fin;
+  uint64_t s_full[kMaxRing], s_empty[kMaxRing];  // score-side codes ring
+  uint64_t v_full[kMaxRing], v_empty[kMaxRing];  // P.V-side codes ring
+  uint64_t stg_full[2], stg_empty[2];            // TMEM staging of the score A operand, per score half
+  uint64_t pv_full[2], pv_empty[2];              // shared-memory staging of the P.V A operand
+  uint64_t sc_full[2], sc_empty[2];              // scores S in TMEM, per tile parity
+  uint64_t p_full[2], p_empty[2];                // P, per tile parity
+  uint64_t red[2];                               // cross-warp reductions of each score half
+  uint64_t q_full, u_done, fin_s, fin_v;
 };
 
 __device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 bits_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+__device__ __forceinline__ __half2 splat_h(uint32_t bits16) { return bits_h2(bits16 | (bits16 << 16)); }
 
+// Non-blocking test of a phase (the producer polls two rings).
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t* v) {
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
                : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
@@ -110,6 +147,15 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_addr(bar))
                : "memory");
 }
+__device__ __forceinline__ void prefetch_l1(const void* p) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
+}
+// Bounded wait used only on exit paths: gives up silently after the limit.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity) && clock64() - t0 < kWaitLimit) {
+  }
+}
 
 // Dequantise one 16-byte vector of codes into fp16 pairs.
 // FP16: 8 values -> 4 regs; INT8: 16 values -> 8 regs; INT4: 32 values -> 16 regs.
@@ -123,9 +169,9 @@ __device__ __forceinline__ void dequant_vec(const uint4 v, uint32_t* out, __half
     const __half2 bias = __halves2half2(__float2half_rn(1152.0f), __float2half_rn(1152.0f));
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint32_t x = w[i] ^ 0x80808080u;                 // offset binary: code + 128
-      const uint32_t a = prmt(x, 0x64646464u, 0x5140u);      // halves 0x64|b0, 0x64|b1 = 1024 + (code + 128)
-      const uint32_t b = prmt(x, 0x64646464u, 0x7362u);      // b2, b3
+      const uint32_t x = w[i] ^ 0x80808080u;             // offset binary: code + 128
+      const uint32_t a = prmt(x, 0x64646464u, 0x5140u);  // halves 0x64|b0, 0x64|b1 = 1024 + (code + 128)
+      const uint32_t b = prmt(x, 0x64646464u, 0x7362u);  // b2, b3
       out[2 * i + 0] = h2_bits(__hsub2(bits_h2(a), bias));
       out[2 * i + 1] = h2_bits(__hsub2(bits_h2(b), bias));
     }
@@ -149,20 +195,32 @@ __device__ __forceinline__ void dequant_vec(const uint4 v, uint32_t* out, __half
   }
 }
 
+// Dequantise half-unit hh (64 values) of unit u from a codes slot row into h[32].
+// INT4: the scale of group 2u + hh comes in `sbits` (fp16 bits).
+template <int FMT>
+__device__ __forceinline__ void dequant_half(const uint8_t* row, int xr, int u, int hh, uint32_t sbits, uint32_t* h) {
+  using F = Fmt<FMT>;
+  constexpr int kRegsPerVec = F::kVals / 16;
+  const __half2 s2 = FMT == TL_H_INT4_G64 ? splat_h(sbits) : __halves2half2(__float2half_rn(1.0f), __float2half_rn(1.0f));
+  const int v0 = F::vec0(u, hh);
+#pragma unroll
+  for (int v = 0; v < F::kVecs; ++v) {
+    const uint4 cv = *reinterpret_cast<const uint4*>(row + (((v0 + v) ^ xr) << 4));
+    dequant_vec<FMT>(cv, h + v * kRegsPerVec, s2);
+  }
+}
+
 template <int FMT, bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
     stream_tc_kernel(const __grid_constant__ CUtensorMap tmap, const StreamParams p) {
+  using F = Fmt<FMT>;
   constexpr int NS = SPLIT ? 32 : 16;  // score columns (heads, or hi/lo x heads)
   constexpr int NP = SPLIT ? 32 : 16;  // P.V columns
-  constexpr int kVals = Fmt<FMT>::kVals;
-  constexpr int kRegsPerVec = kVals / 16;  // fp16 pairs per 16-byte code vector
-  // ring-slot readers: an INT4 chunk holds two units, one per half; other formats: one half reads it
-  constexpr int kSlotReaders = FMT == TL_H_INT4_G64 ? kMathWarps : kMathWarps / 2;
-  constexpr int kChunksPerUnit = FMT == TL_H_FP16 ? 2 : 1;
-  constexpr int kVecs = FMT == TL_H_INT4_G64 ? 4 : 8;  // vectors of one chunk used by one unit
+  constexpr int kSReaders = FMT == TL_H_INT4_G64 ? kSWarps : kSWarps / 2;  // score warps reading a slot
+  constexpr int kVReaders = FMT == TL_H_FP16 ? kVWarps / 2 : kVWarps;      // P.V warps reading a slot
   constexpr uint32_t kIdS = idesc_f16_f32(128, NS, false, false);
   constexpr uint32_t kIdP = idesc_f16_f32(128, NP, true, false);
-  constexpr uint32_t kColS = 0, kColStg = 64, kColU = 256;  // TMEM columns
+  constexpr uint32_t kColS = 0, kColStg = 64, kColU = 256;  // TMEM columns: S[2] x 32, staging[2] x 64, U^T
 
   const Shape& s = p.s;
   const int D = s.d;
@@ -177,42 +235,50 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int r_end = min(n, r_begin + kSplitRows);
   const int n_tiles = (r_end - r_begin + 127) >> 7;
   const int n_units = D >> 7;  // even: d is a multiple of 256
-  const int n_chunks = D / kVals;
+  const int n_chunks = D / F::kVals;
   const int layer = s.n_pre + p.iter;
   const int row_base = (layer * s.max_lanes + b) * s.max_ctx;
   const uint32_t qbytes = (uint32_t)(NS * D * 2);
+  const int SR = p.s_ring, VR = p.v_ring;
+  const int scale_words = D / (2 * kInt4Group);  // INT4: fp16 group scales of a row, two per word
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
-  uint8_t* ring = base;
-  uint8_t* qs = ring + kRing * kSlotBytes;    // NS x D fp16, K-major swizzled atom-columns
-  uint8_t* pvs = qs + qbytes;                // 2 x [128 rows x 128 fp16]
-  uint8_t* ps = pvs + 2 * kPvStageBytes;     // NP x 128 fp16, K-major swizzled
-  uint32_t* scs = reinterpret_cast<uint32_t*>(ps + NP * 256);  // INT4: [2][128][17] words of group scales
+  uint8_t* sring = base;                      // SR slots
+  uint8_t* vring = sring + SR * kSlotBytes;   // VR slots
+  uint8_t* qs = vring + VR * kSlotBytes;      // NS x D fp16, K-major swizzled atom-columns
+  uint8_t* pvs = qs + qbytes;                 // 2 x [128 rows x 128 fp16], MN-major swizzled
+  uint8_t* ps = pvs + 2 * kPvStageBytes;      // 2 x [NP x 128 fp16], K-major swizzled
   __shared__ Bars bars;
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
-  __shared__ float red[2][4][8];
+  __shared__ float red[2][2][4][8];  // [parity][score half][quarter][head]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kRing; ++i) {
-      mbar_init(&bars.ring_full[i], 1);
-      mbar_init(&bars.ring_empty[i], kSlotReaders);
+    for (int i = 0; i < SR; ++i) {
+      mbar_init(&bars.s_full[i], 1);
+      mbar_init(&bars.s_empty[i], kSReaders);
+    }
+    for (int i = 0; i < VR; ++i) {
+      mbar_init(&bars.v_full[i], 1);
+      mbar_init(&bars.v_empty[i], kVReaders);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.stg_full[i], 4);
       mbar_init(&bars.stg_empty[i], 1);
-      mbar_init(&bars.pv_full[i], 4);
+      mbar_init(&bars.pv_full[i], kVWarps);
       mbar_init(&bars.pv_empty[i], 1);
+      mbar_init(&bars.sc_full[i], 1);
+      mbar_init(&bars.sc_empty[i], kSWarps);
+      mbar_init(&bars.p_full[i], kSWarps);
+      mbar_init(&bars.p_empty[i], 1);
+      mbar_init(&bars.red[i], 4);
     }
     mbar_init(&bars.q_full, 1);
-    mbar_init(&bars.s_full, 1);
-    mbar_init(&bars.s_empty, kMathWarps);
-    mbar_init(&bars.p_full, kMathWarps);
-    mbar_init(&bars.p_empty, 1);
     mbar_init(&bars.u_done, 1);
-    mbar_init(&bars.fin, 1);
+    mbar_init(&bars.fin_s, 1);
+    mbar_init(&bars.fin_v, 1);
     abort_flag = 0;
     mbar_fence_init();
     tma_prefetch_desc(&tmap);
@@ -228,80 +294,102 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_p = &abort_flag;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------ TMA producer (both rings)
     if (lane == 0) {
       // the lane's absorbed-query operand image, straight into place
       mbar_expect_tx(&bars.q_full, qbytes);
       const uint8_t* qsrc = p.qimg + (size_t)b * qbytes;
-      for (uint32_t off = 0; off < qbytes; off += 16384) bulk_load(qs + off, qsrc + off, 16384, &bars.q_full);
-      // first pass over a tile: keep it in L2 for the second (P.V) pass; second pass: last use
-      const uint64_t pol_last_use = l2_policy_evict_first();
+      for (uint32_t off = 0; off < qbytes; off += 16384)
+        bulk_load(qs + off, qsrc + off, min(16384u, qbytes - off), &bars.q_full);
+      // the score pass keeps a tile in L2 for the P.V pass, which is its last use
       const uint64_t pol_keep = l2_policy_evict_normal();
-      int issued = 0;
-      bool ok = true;
-      for (int t = 0; t < n_tiles && ok; ++t) {
-        const int gy = row_base + r_begin + t * 128;
-        for (int ph = 0; ph < 2 && ok; ++ph) {
-          for (int c = 0; c < n_chunks; ++c, ++issued) {
-            const int slot = issued & (kRing - 1), use = issued / kRing;
-            if (use > 0 && !mbar_wait(&bars.ring_empty[slot], (use - 1) & 1, abort_p, kWaitLimit)) {
-              ok = false;
-              break;
-            }
-            mbar_expect_tx(&bars.ring_full[slot], kSlotBytes);
-            tma_load_2d(ring + slot * kSlotBytes, &tmap, c * 128, gy, &bars.ring_full[slot],
-                        ph == 0 ? pol_keep : pol_last_use);
+      const uint64_t pol_last_use = l2_policy_evict_first();
+      const int total = n_tiles * n_chunks;
+      int si = 0, vi = 0;
+      long long t_idle = clock64();
+      while ((si < total || vi < total) && !*abort_p) {
+        bool progress = false;
+        if (si < total) {
+          const int slot = si % SR, use = si / SR;
+          if (use == 0 || mbar_test(&bars.s_empty[slot], (use - 1) & 1)) {
+            mbar_expect_tx(&bars.s_full[slot], kSlotBytes);
+            tma_load_2d(sring + slot * kSlotBytes, &tmap, (si % n_chunks) * 128,
+                        row_base + r_begin + (si / n_chunks) * 128, &bars.s_full[slot], pol_keep);
+            ++si;
+            progress = true;
           }
         }
-      }
-      {
-        // every load issued must land before the CTA's shared memory goes away
-        const long long t0 = clock64();
-        while (!mbar_try_wait(&bars.q_full, 0) && clock64() - t0 < kWaitLimit) {
-        }
-      }
-      if (!ok) {
-        const int first = issued > kRing ? issued - kRing : 0;
-        for (int g = first; g < issued; ++g) {
-          const long long t0 = clock64();
-          while (!mbar_try_wait(&bars.ring_full[g & (kRing - 1)], (g / kRing) & 1) && clock64() - t0 < kWaitLimit) {
+        if (vi < si) {  // the P.V read of a chunk never overtakes its score read
+          const int slot = vi % VR, use = vi / VR;
+          if (use == 0 || mbar_test(&bars.v_empty[slot], (use - 1) & 1)) {
+            mbar_expect_tx(&bars.v_full[slot], kSlotBytes);
+            tma_load_2d(vring + slot * kSlotBytes, &tmap, (vi % n_chunks) * 128,
+                        row_base + r_begin + (vi / n_chunks) * 128, &bars.v_full[slot], pol_last_use);
+            ++vi;
+            progress = true;
           }
         }
+        if (progress) {
+          t_idle = clock64();
+        } else if (clock64() - t_idle > kWaitLimit) {
+          *abort_p = 1;
+        }
       }
+      // every copy issued lands before the CTA's shared memory goes away
+      drain_wait(&bars.q_full, 0);
+      for (int g = si > SR ? si - SR : 0; g < si; ++g) drain_wait(&bars.s_full[g % SR], (g / SR) & 1);
+      for (int g = vi > VR ? vi - VR : 0; g < vi; ++g) drain_wait(&bars.v_full[g % VR], (g / VR) & 1);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ score-MMA issuer
     if (lane == 0) {
-      // base descriptors; the address field is the low 14 bits of (address >> 4), so adding
-      // (byte offset >> 4) to a descriptor moves it within shared memory
+      // the address field of a descriptor is (address >> 4), so adding (byte offset >> 4)
+      // moves it within shared memory
       const uint64_t q_desc0 = sdesc_sw128(smem_addr(qs), 16, 1024);
-      const uint64_t pv_desc0 = sdesc_sw128(smem_addr(pvs), 16384, 1024);
-      const uint64_t p_desc0 = sdesc_sw128(smem_addr(ps), 16, 1024);
       bool ok = mbar_wait(&bars.q_full, 0, abort_p, kWaitLimit);
-      bool issued_any = false;
+      bool issued = false;
       for (int t = 0; t < n_tiles && ok; ++t) {
-        if (t > 0 && !mbar_wait(&bars.s_empty, (t - 1) & 1, abort_p, kWaitLimit)) { ok = false; break; }
+        const int sb = t & 1;
+        if (t >= 2 && !mbar_wait(&bars.sc_empty[sb], ((t >> 1) - 1) & 1, abort_p, kWaitLimit)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t dS = tbase + kColS + sb * 32;
         for (int u = 0; u < n_units; ++u) {
-          const int gs = t * n_units + u, x = u & 1;
-          if (!mbar_wait(&bars.stg_full[x], (gs >> 1) & 1, abort_p, kWaitLimit)) { ok = false; break; }
+          const int x = u & 1, k_use = t * (n_units >> 1) + (u >> 1);
+          if (!mbar_wait(&bars.stg_full[x], k_use & 1, abort_p, kWaitLimit)) { ok = false; break; }
           tc_fence_after();
-          // descriptors of this unit's 8 K-steps differ from the first by compile-time byte offsets
+          // the unit's 8 K-steps: A = 8 TMEM columns each, B = 32 bytes within an atom-column
           const uint64_t bd = q_desc0 + (uint64_t)((u * 2 * NS * 128) >> 4);
           const uint32_t ta = tbase + kColStg + x * 64;
           if (u == 0)
-            mma_ts_first(tbase + kColS, ta, bd, kIdS);
+            mma_ts_first(dS, ta, bd, kIdS);
           else
-            mma_ts_acc(tbase + kColS, ta, bd, kIdS);
+            mma_ts_acc(dS, ta, bd, kIdS);
 #pragma unroll
           for (int k = 1; k < 8; ++k)
-            mma_ts_acc(tbase + kColS, ta + k * 8, bd + (uint64_t)(((k >> 2) * NS * 128 + (k & 3) * 32) >> 4), kIdS);
-          issued_any = true;
+            mma_ts_acc(dS, ta + k * 8, bd + (uint64_t)(((k >> 2) * NS * 128 + (k & 3) * 32) >> 4), kIdS);
+          issued = true;
           mma_commit(&bars.stg_empty[x]);
         }
         if (!ok) break;
-        mma_commit(&bars.s_full);
-        if (!mbar_wait(&bars.p_full, t & 1, abort_p, kWaitLimit)) { ok = false; break; }
+        mma_commit(&bars.sc_full[sb]);
+      }
+      if (issued) {
+        // nothing may still be writing TMEM when it is freed
+        mma_commit(&bars.fin_s);
+        drain_wait(&bars.fin_s, 0);
+      }
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ P.V-MMA issuer
+    if (lane == 0) {
+      const uint64_t pv_desc0 = sdesc_sw128(smem_addr(pvs), 16384, 1024);
+      const uint64_t p_desc0 = sdesc_sw128(smem_addr(ps), 16, 1024);
+      bool ok = true, issued = false;
+      for (int t = 0; t < n_tiles && ok; ++t) {
+        const int pb = t & 1;
+        if (!mbar_wait(&bars.p_full[pb], (t >> 1) & 1, abort_p, kWaitLimit)) { ok = false; break; }
         tc_fence_after();
+        const uint64_t pd = p_desc0 + (uint64_t)((pb * NP * 256) >> 4);
         for (int u = 0; u < n_units; ++u) {
           const int gp = t * n_units + u, x = u & 1;
           if (!mbar_wait(&bars.pv_full[x], (gp >> 1) & 1, abort_p, kWaitLimit)) { ok = false; break; }
@@ -309,39 +397,36 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t ad = pv_desc0 + (uint64_t)((x * kPvStageBytes) >> 4);
           const uint32_t du = tbase + kColU + u * NP;
           if (t == 0)
-            mma_ss_first(du, ad, p_desc0, kIdP);
+            mma_ss_first(du, ad, pd, kIdP);
           else
-            mma_ss_acc(du, ad, p_desc0, kIdP);
+            mma_ss_acc(du, ad, pd, kIdP);
 #pragma unroll
           for (int k = 1; k < 8; ++k)
             mma_ss_acc(du, ad + (uint64_t)((k * 2048) >> 4),
-                       p_desc0 + (uint64_t)((((k * 16) >> 6) * NP * 128 + ((k * 16) & 63) * 2) >> 4), kIdP);
+                       pd + (uint64_t)((((k * 16) >> 6) * NP * 128 + ((k * 16) & 63) * 2) >> 4), kIdP);
+          issued = true;
           mma_commit(&bars.pv_empty[x]);
         }
         if (!ok) break;
-        mma_commit(&bars.p_empty);
+        mma_commit(&bars.p_empty[pb]);
       }
       if (ok) mma_commit(&bars.u_done);
-      if (issued_any) {
-        // nothing may still be writing TMEM when it is freed
-        mma_commit(&bars.fin);
-        const long long t0 = clock64();
-        while (!mbar_try_wait(&bars.fin, 0) && clock64() - t0 < kWaitLimit) {
-        }
+      if (issued) {
+        mma_commit(&bars.fin_v);
+        drain_wait(&bars.fin_v, 0);
       }
     }
-  } else {
-    // ------------------------------------------------------------ math warps
-    // half 0 (warps 2-5) takes the even units and heads 0-7, half 1 (warps 6-9) the odd
-    // units and heads 8-15; in each half, warp w owns TMEM lanes / tile rows 32*(w%4) ..
+  } else if (warp < kWarpV0) {
+    // ------------------------------------------------------------ score group
+    // warp -> (TMEM lane quarter = row block, half): half 0 takes the even units and
+    // heads 0-7, half 1 the odd units and heads 8-15
     const int quarter = warp & 3;
-    const int half = (warp - 2) >> 2;
+    const int half = (warp - kWarpS0) >> 2;
     const int r = quarter * 32 + lane;
-    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const int h0 = half * 8;  // first head of this half
-    uint32_t* sc_row = scs + (half * 128 + r) * kScaleRowWords;
-    const uint8_t* my_row = ring + r * 128;
     const int xr = r & 7;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const int h0 = half * 8;
+    uint64_t* red_bar = &bars.red[half];
 
     float m_used[8], l_part[8];
 #pragma unroll
@@ -350,178 +435,141 @@ __global__ void __launch_bounds__(kThreads, 1)
       l_part[j] = 0.0f;
     }
     bool ok = true;
-
-    // scales of a tile's rows (INT8: one fp32; INT4: d/64 fp16, up to 16 words), fetched a tile ahead
+    // per-row scales: INT8 one fp32 (fetched a tile ahead); INT4 d/64 fp16 read per unit,
+    // the tile's row brought into L1 a tile ahead
+    auto row_of = [&](int t) { return (size_t)row_base + r_begin + t * 128 + r; };
+    auto row_valid = [&](int t) { return r < (r_end - (r_begin + t * 128)); };
     float scale_next = 0.0f;
-    uint4 scv_next[4];
-    auto fetch_scales = [&](int t_next) {
-      const int row0n = r_begin + t_next * 128;
-      const bool vn = r < (r_end - row0n);
-      const size_t grown = (size_t)row_base + row0n + r;
-      if (FMT == TL_H_INT8_TOKEN) scale_next = vn ? reinterpret_cast<const float*>(p.scales)[grown] : 0.0f;
-      if (FMT == TL_H_INT4_G64) {
-        const uint4* src = reinterpret_cast<const uint4*>(p.scales + grown * (size_t)(D / kInt4Group) * 2);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) scv_next[i] = (vn && i * 8 < D / kInt4Group) ? src[i] : make_uint4(0, 0, 0, 0);
-      }
-    };
-    fetch_scales(0);
+    if (FMT == TL_H_INT8_TOKEN && row_valid(0)) scale_next = __ldg(reinterpret_cast<const float*>(p.scales) + row_of(0));
+    if (FMT == TL_H_INT4_G64 && row_valid(0)) prefetch_l1(p.scales + row_of(0) * (size_t)scale_words * 4);
 
     for (int t = 0; t < n_tiles && ok; ++t) {
-      const int row0 = r_begin + t * 128;
-      const bool valid = r < (r_end - row0);
+      const bool valid = row_valid(t);
       const float scale_row = scale_next;
-      if (FMT == TL_H_INT4_G64) {
-        // into this thread's own padded smem row (read back one word per unit)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          sc_row[4 * i + 0] = scv_next[i].x;
-          sc_row[4 * i + 1] = scv_next[i].y;
-          sc_row[4 * i + 2] = scv_next[i].z;
-          sc_row[4 * i + 3] = scv_next[i].w;
-        }
+      const uint32_t* srow = reinterpret_cast<const uint32_t*>(p.scales + row_of(t) * (size_t)scale_words * 4);
+      if (t + 1 < n_tiles && row_valid(t + 1)) {
+        if (FMT == TL_H_INT8_TOKEN) scale_next = __ldg(reinterpret_cast<const float*>(p.scales) + row_of(t + 1));
+        if (FMT == TL_H_INT4_G64) prefetch_l1(p.scales + row_of(t + 1) * (size_t)scale_words * 4);
       }
 
-      for (int ph = 0; ph < 2 && ok; ++ph) {
-        if (ph == 1) {
-          // ------------------------------------------------ softmax of this tile (this half's heads), then P
-          if (!mbar_wait(&bars.s_full, t & 1, abort_p, kWaitLimit)) { ok = false; break; }
-          tc_fence_after();
-          uint32_t sv[16];
-          tmem_ld8(tbase + lane_off + kColS + h0, sv);
-          if (NS == 32) tmem_ld8(tbase + lane_off + kColS + 16 + h0, sv + 8);
-          tmem_ld_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bars.s_empty);
-          float sc[8];
+      // ------------------------------------------------ this half's units of tile t -> TMEM staging
+      for (int u = half; u < n_units; u += 2) {
+        const uint32_t sw = (FMT == TL_H_INT4_G64 && valid) ? __ldg(srow + u) : 0u;  // groups 2u | 2u+1
+        const int k_use = t * (n_units >> 1) + (u >> 1);
+        const uint32_t ta = tbase + lane_off + kColStg + half * 64;
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            float v = __uint_as_float(sv[j]);
-            if (NS == 32) v += __uint_as_float(sv[8 + j]);
-            if (FMT == TL_H_INT8_TOKEN) v *= scale_row;
-            sc[j] = valid ? v : -CUDART_INF_F;
-          }
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            float v = sc[j];
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-            if (lane == 0) red[half][quarter][j] = v;
-          }
-          named_bar_sync(1 + half, 128);
-          float alpha[8];
-          bool rescale = false;
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float tm = fmaxf(fmaxf(red[half][0][j], red[half][1][j]), fmaxf(red[half][2][j], red[half][3][j]));
-            alpha[j] = 1.0f;
-            if (tm > m_used[j] + 8.0f) {  // lazy rescale: P stays below 2^8 otherwise
-              if (m_used[j] != -CUDART_INF_F) {
-                alpha[j] = exp2f(m_used[j] - tm);
-                rescale = true;
-              }
-              m_used[j] = tm;
-            }
-          }
-          named_bar_sync(1 + half, 128);  // red is rewritten by the next tile
-          float pr[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            pr[j] = valid ? exp2f(sc[j] - m_used[j]) : 0.0f;
-            l_part[j] = l_part[j] * alpha[j] + pr[j];
-          }
-          // the previous tile's P.V must be done before P is rewritten or U rescaled
-          if (t > 0 && !mbar_wait(&bars.p_empty, (t - 1) & 1, abort_p, kWaitLimit)) { ok = false; break; }
-          tc_fence_after();
-          if (rescale) {
-            // rare: the running maximum rose by more than 2^8; rescale this half's columns of U^T
-            for (int u = 0; u < n_units; ++u) {
-              uint32_t uv[16];
-              tmem_ld8(tbase + lane_off + kColU + u * NP + h0, uv);
-              if (NP == 32) tmem_ld8(tbase + lane_off + kColU + u * NP + 16 + h0, uv + 8);
-              tmem_ld_wait();
-#pragma unroll
-              for (int c = 0; c < 16; ++c) uv[c] = __float_as_uint(__uint_as_float(uv[c]) * alpha[c & 7]);
-              tmem_st8(tbase + lane_off + kColU + u * NP + h0, uv);
-              if (NP == 32) tmem_st8(tbase + lane_off + kColU + u * NP + 16 + h0, uv + 8);
-            }
-            tmem_st_wait();
-          }
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float v = FMT == TL_H_INT8_TOKEN ? pr[j] * scale_row : pr[j];
-            const __half hi = __float2half_rn(v);
-            *reinterpret_cast<__half*>(ps + kmajor_offset(h0 + j, r, NP)) = hi;
-            if (NP == 32)
-              *reinterpret_cast<__half*>(ps + kmajor_offset(16 + h0 + j, r, NP)) = __float2half_rn(v - __half2float(hi));
-          }
-          fence_proxy_async_smem();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bars.p_full);
-          if (t + 1 < n_tiles) fetch_scales(t + 1);  // lands while this tile's P.V operands are made
-        }
-
-        // ------------------------------------------------ dequantise this half's units of the tile
-        const int gbase = (t * 2 + ph) * n_chunks;  // producer's load index of chunk 0 of this pass
-        for (int u = half; u < n_units && ok; u += 2) {
-          uint32_t h[64];
-          uint32_t scw = 0;
-          if (FMT == TL_H_INT4_G64) scw = sc_row[u];  // fp16 scales of groups 2u (low) and 2u+1 (high)
-#pragma unroll
-          for (int cc = 0; cc < kChunksPerUnit; ++cc) {
-            const int c = FMT == TL_H_INT4_G64 ? (u >> 1) : FMT == TL_H_INT8_TOKEN ? u : 2 * u + cc;
-            const int g = gbase + c;
-            const int slot = g & (kRing - 1);
-            if (!mbar_wait(&bars.ring_full[slot], (g / kRing) & 1, abort_p, kWaitLimit)) { ok = false; break; }
-            const uint8_t* src = my_row + slot * kSlotBytes;
-            const int v0 = FMT == TL_H_INT4_G64 ? (u & 1) * 4 : 0;
-#pragma unroll
-            for (int v = 0; v < kVecs; ++v) {
-              const uint4 cv = *reinterpret_cast<const uint4*>(src + (((v0 + v) ^ xr) << 4));
-              __half2 s2 = __halves2half2(__float2half_rn(1.0f), __float2half_rn(1.0f));
-              if (FMT == TL_H_INT4_G64) {
-                const uint32_t sbits = (v < 2) ? (scw & 0xFFFFu) : (scw >> 16);
-                s2 = bits_h2(sbits | (sbits << 16));
-              }
-              dequant_vec<FMT>(cv, h + (cc * kVecs + v) * kRegsPerVec, s2);
-            }
+        for (int hh = 0; hh < 2; ++hh) {
+          const int g = t * n_chunks + F::chunk(u, hh);
+          const int slot = g % SR;
+          if (!mbar_wait(&bars.s_full[slot], (g / SR) & 1, abort_p, kWaitLimit)) { ok = false; break; }
+          uint32_t h[32];
+          dequant_half<FMT>(sring + slot * kSlotBytes + r * 128, xr, u, hh, hh ? (sw >> 16) : (sw & 0xFFFFu), h);
+          if (F::score_releases(hh)) {
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars.ring_empty[slot]);
+            if (lane == 0) mbar_arrive(&bars.s_empty[slot]);
           }
-          if (!ok) break;
           if (!valid) {
 #pragma unroll
-            for (int i = 0; i < 64; ++i) h[i] = 0u;
+            for (int i = 0; i < 32; ++i) h[i] = 0u;
           }
-          const int gu = t * n_units + u, x = half;
-          if (ph == 0) {
-            if (gu >= 2 && !mbar_wait(&bars.stg_empty[x], ((gu >> 1) - 1) & 1, abort_p, kWaitLimit)) { ok = false; break; }
+          if (hh == 0) {
+            // the staging buffer is free once the MMAs of this half's previous unit are done
+            if (k_use >= 1 && !mbar_wait(&bars.stg_empty[half], (k_use - 1) & 1, abort_p, kWaitLimit)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t ta = tbase + lane_off + kColStg + x * 64;
-            tmem_st16(ta + 0, h + 0);
-            tmem_st16(ta + 16, h + 16);
-            tmem_st16(ta + 32, h + 32);
-            tmem_st16(ta + 48, h + 48);
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars.stg_full[x]);
-          } else {
-            if (gu >= 2 && !mbar_wait(&bars.pv_empty[x], ((gu >> 1) - 1) & 1, abort_p, kWaitLimit)) { ok = false; break; }
-            uint8_t* st = pvs + x * kPvStageBytes + r * 128;
-#pragma unroll
-            for (int v = 0; v < 16; ++v) {
-              const uint4 val = make_uint4(h[4 * v], h[4 * v + 1], h[4 * v + 2], h[4 * v + 3]);
-              *reinterpret_cast<uint4*>(st + (v >> 3) * 16384 + (((v & 7) ^ xr) << 4)) = val;
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars.pv_full[x]);
           }
+          tmem_st16(ta + hh * 32, h);
+          tmem_st16(ta + hh * 32 + 16, h + 16);
+        }
+        if (!ok) break;
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.stg_full[half]);
+      }
+      if (!ok) break;
+
+      // ------------------------------------------------ online softmax of tile t, this half's heads
+      const int sb = t & 1;
+      if (!mbar_wait(&bars.sc_full[sb], (t >> 1) & 1, abort_p, kWaitLimit)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t sv[16];
+      tmem_ld8(tbase + lane_off + kColS + sb * 32 + h0, sv);
+      if (NS == 32) tmem_ld8(tbase + lane_off + kColS + sb * 32 + 16 + h0, sv + 8);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.sc_empty[sb]);
+      float sc[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float v = __uint_as_float(sv[j]);
+        if (NS == 32) v += __uint_as_float(sv[8 + j]);
+        if (FMT == TL_H_INT8_TOKEN) v *= scale_row;
+        sc[j] = valid ? v : -CUDART_INF_F;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float v = sc[j];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+        if (lane == 0) red[sb][half][quarter][j] = v;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(red_bar);
+      if (!mbar_wait(red_bar, t & 1, abort_p, kWaitLimit)) { ok = false; break; }
+      float alpha[8];
+      bool rescale = false;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float tm = fmaxf(fmaxf(red[sb][half][0][j], red[sb][half][1][j]),
+                               fmaxf(red[sb][half][2][j], red[sb][half][3][j]));
+        alpha[j] = 1.0f;
+        if (tm > m_used[j] + 8.0f) {  // lazy rescale: P stays below 2^8 otherwise
+          if (m_used[j] != -CUDART_INF_F) {
+            alpha[j] = exp2f(m_used[j] - tm);
+            rescale = true;
+          }
+          m_used[j] = tm;
         }
       }
+      float pr[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        pr[j] = valid ? exp2f(sc[j] - m_used[j]) : 0.0f;
+        l_part[j] = l_part[j] * alpha[j] + pr[j];
+      }
+      if (rescale) {
+        // rare: the running maximum rose by more than 2^8; U^T is rescaled once every P.V MMA of
+        // the earlier tiles has landed (those of tile t wait for this half's P)
+        if (t >= 1 && !mbar_wait(&bars.p_empty[(t - 1) & 1], ((t - 1) >> 1) & 1, abort_p, kWaitLimit)) { ok = false; break; }
+        tc_fence_after();
+        for (int u = 0; u < n_units; ++u) {
+          uint32_t uv[16];
+          tmem_ld8(tbase + lane_off + kColU + u * NP + h0, uv);
+          if (NP == 32) tmem_ld8(tbase + lane_off + kColU + u * NP + 16 + h0, uv + 8);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < 16; ++c) uv[c] = __float_as_uint(__uint_as_float(uv[c]) * alpha[c & 7]);
+          tmem_st8(tbase + lane_off + kColU + u * NP + h0, uv);
+          if (NP == 32) tmem_st8(tbase + lane_off + kColU + u * NP + 16 + h0, uv + 8);
+        }
+        tmem_st_wait();
+      }
+      // P buffer sb was last read by the P.V MMAs of tile t-2
+      if (t >= 2 && !mbar_wait(&bars.p_empty[sb], ((t >> 1) - 1) & 1, abort_p, kWaitLimit)) { ok = false; break; }
+      uint8_t* pbuf = ps + sb * NP * 256;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float v = FMT == TL_H_INT8_TOKEN ? pr[j] * scale_row : pr[j];
+        const __half hi = __float2half_rn(v);
+        *reinterpret_cast<__half*>(pbuf + kmajor_offset(h0 + j, r, NP)) = hi;
+        if (NP == 32)
+          *reinterpret_cast<__half*>(pbuf + kmajor_offset(16 + h0 + j, r, NP)) = __float2half_rn(v - __half2float(hi));
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.p_full[sb]);
     }
 
     // ------------------------------------------------ partial (m, l, U) of this split, this half's heads
@@ -541,18 +589,65 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (h0 + j < s.H) p.U[(part * kMaxHeads + h0 + j) * D + d] = v;
         }
       }
+      const int sb = n_tiles & 1;  // last used by tile n_tiles-2, read by every warp since
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         float v = l_part[j];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0) red[half][quarter][j] = v;
+        if (lane == 0) red[sb][half][quarter][j] = v;
       }
-      named_bar_sync(1 + half, 128);
-      if (r < 8) {
-        p.ml[(part * kMaxHeads + h0 + r) * 2 + 0] = m_used[r];
-        p.ml[(part * kMaxHeads + h0 + r) * 2 + 1] =
-            red[half][0][r] + red[half][1][r] + red[half][2][r] + red[half][3][r];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(red_bar);
+      if (mbar_wait(red_bar, n_tiles & 1, abort_p, kWaitLimit) && quarter == 0 && lane < 8) {
+        float m = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (j == lane) m = m_used[j];
+        p.ml[(part * kMaxHeads + h0 + lane) * 2 + 0] = m;
+        p.ml[(part * kMaxHeads + h0 + lane) * 2 + 1] =
+            red[sb][half][0][lane] + red[sb][half][1][lane] + red[sb][half][2][lane] + red[sb][half][3][lane];
+      }
+    }
+    tmem_st_wait();  // no store of this warp may be in flight when TMEM is freed
+  } else {
+    // ------------------------------------------------------------ P.V group
+    // warp -> (row block, part): part 0 dequantises values 0-63 of every unit, part 1 64-127,
+    // into the swizzled shared-memory staging the P.V MMA reads MN-major (d as M, rows as K)
+    const int vw = warp - kWarpV0;
+    const int r = (vw & 3) * 32 + lane;
+    const int part = vw >> 2;
+    const int xr = r & 7;
+    bool ok = true;
+    auto row_of = [&](int t) { return (size_t)row_base + r_begin + t * 128 + r; };
+    auto row_valid = [&](int t) { return r < (r_end - (r_begin + t * 128)); };
+    for (int t = 0; t < n_tiles && ok; ++t) {
+      const bool valid = row_valid(t);
+      const uint32_t* srow = reinterpret_cast<const uint32_t*>(p.scales + row_of(t) * (size_t)scale_words * 4);
+      for (int u = 0; u < n_units; ++u) {
+        const uint32_t sw = (FMT == TL_H_INT4_G64 && valid) ? __ldg(srow + u) : 0u;
+        const int g = t * n_chunks + F::chunk(u, part);
+        const int slot = g % VR;
+        if (!mbar_wait(&bars.v_full[slot], (g / VR) & 1, abort_p, kWaitLimit)) { ok = false; break; }
+        uint32_t h[32];
+        dequant_half<FMT>(vring + slot * kSlotBytes + r * 128, xr, u, part, part ? (sw >> 16) : (sw & 0xFFFFu), h);
+        if (F::pv_releases(u)) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars.v_empty[slot]);
+        }
+        if (!valid) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) h[i] = 0u;
+        }
+        const int gp = t * n_units + u, x = u & 1;
+        if (gp >= 2 && !mbar_wait(&bars.pv_empty[x], ((gp >> 1) - 1) & 1, abort_p, kWaitLimit)) { ok = false; break; }
+        uint8_t* st = pvs + x * kPvStageBytes + part * 16384 + r * 128;
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+          *reinterpret_cast<uint4*>(st + ((v ^ xr) << 4)) = make_uint4(h[4 * v], h[4 * v + 1], h[4 * v + 2], h[4 * v + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.pv_full[x]);
       }
     }
   }
@@ -584,12 +679,23 @@ template <int FMT, bool SPLIT>
 cudaError_t launch_fmt(const DecodeArgs& a, const CUtensorMap& tmap, cudaStream_t st) {
   const Shape& s = a.s;
   constexpr int NP = SPLIT ? 32 : 16;
-  const size_t smem = qimg_bytes(s.d) + 2 * kPvStageBytes + (size_t)NP * 256 + kScaleBytes + 1024 +  // + align
-                      (size_t)kRing * kSlotBytes;
-  if (smem > 225 * 1024) return cudaErrorInvalidConfiguration;
-  cudaError_t e = cudaFuncSetAttribute(stream_tc_kernel<FMT, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  auto kern = stream_tc_kernel<FMT, SPLIT>;
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, kern);
   if (e != cudaSuccess) return e;
+  int dev = 0, optin = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
+  // fixed regions (+ up to 1 KB of alignment), then as many 16 KB ring slots as fit, shared
+  // between the score-side and the P.V-side rings
+  const size_t fixed = 1024 + qimg_bytes(s.d) + 2 * (size_t)kPvStageBytes + 2 * (size_t)NP * 256;
+  const long long room = (long long)optin - (long long)fa.sharedSizeBytes - (long long)fixed;
+  const int slots = room > 0 ? (int)(room / kSlotBytes) : 0;
+  if (slots < 4) return cudaErrorInvalidConfiguration;
+  const int s_ring = std::min(kMaxRing, (slots + 1) / 2);
+  const int v_ring = std::min(kMaxRing, slots - s_ring);
+  const size_t smem = fixed + (size_t)(s_ring + v_ring) * kSlotBytes;
+  if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
   StreamParams p{s,
                  a.iter,
                  a.loops,
@@ -599,9 +705,11 @@ cudaError_t launch_fmt(const DecodeArgs& a, const CUtensorMap& tmap, cudaStream_
                  reinterpret_cast<float*>(a.ws + a.wl.ml_off),
                  reinterpret_cast<float*>(a.ws + a.wl.u_off),
                  reinterpret_cast<uint32_t*>(a.ws + a.wl.status_off),
-                 a.wl.s_max};
+                 a.wl.s_max,
+                 s_ring,
+                 v_ring};
   dim3 grid(a.wl.s_max, a.n_lanes);
-  stream_tc_kernel<FMT, SPLIT><<<grid, kThreads, smem, st>>>(tmap, p);
+  kern<<<grid, kThreads, smem, st>>>(tmap, p);
   count_launch();
   return cudaGetLastError();
 }
