@@ -13,9 +13,10 @@
 // U^T accumulates in TMEM over the whole split; the (m, l, U) partial goes to
 // the workspace and is merged exactly by the epilogue kernel.
 //
-// Warp roles (608 threads): warp 0 = TMA producer; warp 1 = score-MMA issuer
-// (and TMEM owner); warp 2 = P.V-MMA issuer; warps 3-10 = score group; warps
-// 11-18 = P.V group.  The two groups work on different tiles at the same time:
+// Warp roles (640 threads): warp 0 = TMA producer of the score-side ring (and
+// the query image); warp 1 = score-MMA issuer (and TMEM owner); warp 2 = P.V-MMA
+// issuer; warps 3-10 = score group; warps 11-18 = P.V group; warp 19 = TMA
+// producer of the P.V-side ring.  The two groups work on different tiles at the same time:
 // while the score group dequantises tile t+1 into TMEM (the A operand of the
 // score MMAs) and runs its online softmax, the P.V group dequantises tile t into
 // shared memory (the A operand of the P.V MMAs, which take tile t's P).  P is
@@ -67,7 +68,8 @@ constexpr int kSWarps = 8;                      // score group: two warps per TM
 constexpr int kVWarps = 8;                      // P.V group: two warps per 32-row block
 constexpr int kWarpS0 = 3;                      // first score warp
 constexpr int kWarpV0 = kWarpS0 + kSWarps;      // first P.V warp
-constexpr int kThreads = 32 * (kWarpV0 + kVWarps);
+constexpr int kWarpVP = kWarpV0 + kVWarps;     // producer of the P.V-side ring
+constexpr int kThreads = 32 * (kWarpVP + 1);
 constexpr int kSlotBytes = 128 * 128;           // one ring slot: 128 rows x 128 bytes of codes
 constexpr int kPvStageBytes = 128 * 256;        // P.V operand staging: 128 rows x 128 fp16 values
 constexpr int kMaxRing = 4;                     // slots per ring at most
@@ -120,16 +122,6 @@ __device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cas
 __device__ __forceinline__ __half2 bits_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
 __device__ __forceinline__ __half2 splat_h(uint32_t bits16) { return bits_h2(bits16 | (bits16 << 16)); }
 
-// Non-blocking test of a phase (the producer polls two rings).
-__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(smem_addr(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
 __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t* v) {
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
                : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
@@ -146,6 +138,16 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                    smem_addr(dst)),
                "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_addr(bar))
                : "memory");
+}
+// One lane of a converged warp (the same one every time the whole warp asks).
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile("{\n .reg .pred p;\n elect.sync _|p, 0xffffffff;\n selp.u32 %0, 1, 0, p;\n}\n" : "=r"(pred));
+  return pred != 0;
+}
+// Bounded wait of a whole warp; the outcome is made warp-uniform.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, kWaitLimit));
 }
 __device__ __forceinline__ void prefetch_l1(const void* p) {
   asm volatile("prefetch.global.L1 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
@@ -252,6 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ Bars bars;
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
+  __shared__ int s_issued;           // score-side chunk loads issued so far
   __shared__ float red[2][2][4][8];  // [parity][score half][quarter][head]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -280,6 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars.fin_s, 1);
     mbar_init(&bars.fin_v, 1);
     abort_flag = 0;
+    s_issued = 0;
     mbar_fence_init();
     tma_prefetch_desc(&tmap);
   }
@@ -293,8 +297,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tbase = tmem_base;
   volatile int* abort_p = &abort_flag;
 
+  volatile int* s_issued_p = &s_issued;
+  const int total_chunks = n_tiles * n_chunks;
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer (both rings)
+    // ------------------------------------------------------------ TMA producer, score-side ring
     if (lane == 0) {
       // the lane's absorbed-query operand image, straight into place
       mbar_expect_tx(&bars.q_full, qbytes);
@@ -303,63 +309,65 @@ __global__ void __launch_bounds__(kThreads, 1)
         bulk_load(qs + off, qsrc + off, min(16384u, qbytes - off), &bars.q_full);
       // the score pass keeps a tile in L2 for the P.V pass, which is its last use
       const uint64_t pol_keep = l2_policy_evict_normal();
-      const uint64_t pol_last_use = l2_policy_evict_first();
-      const int total = n_tiles * n_chunks;
-      int si = 0, vi = 0;
-      long long t_idle = clock64();
-      while ((si < total || vi < total) && !*abort_p) {
-        bool progress = false;
-        if (si < total) {
-          const int slot = si % SR, use = si / SR;
-          if (use == 0 || mbar_test(&bars.s_empty[slot], (use - 1) & 1)) {
-            mbar_expect_tx(&bars.s_full[slot], kSlotBytes);
-            tma_load_2d(sring + slot * kSlotBytes, &tmap, (si % n_chunks) * 128,
-                        row_base + r_begin + (si / n_chunks) * 128, &bars.s_full[slot], pol_keep);
-            ++si;
-            progress = true;
-          }
-        }
-        if (vi < si) {  // the P.V read of a chunk never overtakes its score read
-          const int slot = vi % VR, use = vi / VR;
-          if (use == 0 || mbar_test(&bars.v_empty[slot], (use - 1) & 1)) {
-            mbar_expect_tx(&bars.v_full[slot], kSlotBytes);
-            tma_load_2d(vring + slot * kSlotBytes, &tmap, (vi % n_chunks) * 128,
-                        row_base + r_begin + (vi / n_chunks) * 128, &bars.v_full[slot], pol_last_use);
-            ++vi;
-            progress = true;
-          }
-        }
-        if (progress) {
-          t_idle = clock64();
-        } else if (clock64() - t_idle > kWaitLimit) {
-          *abort_p = 1;
-        }
+      int g = 0;
+      for (; g < total_chunks; ++g) {
+        const int slot = g % SR, use = g / SR;
+        if (use > 0 && !mbar_wait(&bars.s_empty[slot], (use - 1) & 1, abort_p, kWaitLimit)) break;
+        mbar_expect_tx(&bars.s_full[slot], kSlotBytes);
+        tma_load_2d(sring + slot * kSlotBytes, &tmap, (g % n_chunks) * 128, row_base + r_begin + (g / n_chunks) * 128,
+                    &bars.s_full[slot], pol_keep);
+        *s_issued_p = g + 1;
       }
       // every copy issued lands before the CTA's shared memory goes away
       drain_wait(&bars.q_full, 0);
-      for (int g = si > SR ? si - SR : 0; g < si; ++g) drain_wait(&bars.s_full[g % SR], (g / SR) & 1);
-      for (int g = vi > VR ? vi - VR : 0; g < vi; ++g) drain_wait(&bars.v_full[g % VR], (g / VR) & 1);
+      for (int i = g > SR ? g - SR : 0; i < g; ++i) drain_wait(&bars.s_full[i % SR], (i / SR) & 1);
+    }
+  } else if (warp == kWarpVP) {
+    // ------------------------------------------------------------ TMA producer, P.V-side ring
+    // A chunk's P.V load follows its score load, so it finds the tile in L2.  The score side
+    // never waits for this warp's loads of chunks it has not loaded itself, so no cycle forms.
+    if (lane == 0) {
+      const uint64_t pol_last_use = l2_policy_evict_first();
+      int g = 0;
+      for (; g < total_chunks; ++g) {
+        const int slot = g % VR, use = g / VR;
+        if (use > 0 && !mbar_wait(&bars.v_empty[slot], (use - 1) & 1, abort_p, kWaitLimit)) break;
+        if (*s_issued_p <= g) {
+          const long long t0 = clock64();
+          while (*s_issued_p <= g && !*abort_p) {
+            __nanosleep(128);
+            if (clock64() - t0 > kWaitLimit) *abort_p = 1;
+          }
+          if (*abort_p) break;
+        }
+        mbar_expect_tx(&bars.v_full[slot], kSlotBytes);
+        tma_load_2d(vring + slot * kSlotBytes, &tmap, (g % n_chunks) * 128, row_base + r_begin + (g / n_chunks) * 128,
+                    &bars.v_full[slot], pol_last_use);
+      }
+      for (int i = g > VR ? g - VR : 0; i < g; ++i) drain_wait(&bars.v_full[i % VR], (i / VR) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ score-MMA issuer
-    if (lane == 0) {
-      // the address field of a descriptor is (address >> 4), so adding (byte offset >> 4)
-      // moves it within shared memory
-      const uint64_t q_desc0 = sdesc_sw128(smem_addr(qs), 16, 1024);
-      bool ok = mbar_wait(&bars.q_full, 0, abort_p, kWaitLimit);
-      bool issued = false;
-      for (int t = 0; t < n_tiles && ok; ++t) {
-        const int sb = t & 1;
-        if (t >= 2 && !mbar_wait(&bars.sc_empty[sb], ((t >> 1) - 1) & 1, abort_p, kWaitLimit)) { ok = false; break; }
+    // The whole warp runs the loop, so descriptors and TMEM addresses stay warp-uniform, and one
+    // elected lane issues (a lone divergent lane issues tcgen05.mma at about half the rate).
+    // The address field of a descriptor is (address >> 4), so adding (byte offset >> 4) moves it
+    // within shared memory.
+    const uint64_t q_desc0 = sdesc_sw128(smem_addr(qs), 16, 1024);
+    bool ok = warp_wait(&bars.q_full, 0, abort_p);
+    bool issued = false;
+    for (int t = 0; t < n_tiles && ok; ++t) {
+      const int sb = t & 1;
+      if (t >= 2 && !warp_wait(&bars.sc_empty[sb], ((t >> 1) - 1) & 1, abort_p)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t dS = tbase + kColS + sb * 32;
+      for (int u = 0; u < n_units; ++u) {
+        const int x = u & 1, k_use = t * (n_units >> 1) + (u >> 1);
+        if (!warp_wait(&bars.stg_full[x], k_use & 1, abort_p)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t dS = tbase + kColS + sb * 32;
-        for (int u = 0; u < n_units; ++u) {
-          const int x = u & 1, k_use = t * (n_units >> 1) + (u >> 1);
-          if (!mbar_wait(&bars.stg_full[x], k_use & 1, abort_p, kWaitLimit)) { ok = false; break; }
-          tc_fence_after();
-          // the unit's 8 K-steps: A = 8 TMEM columns each, B = 32 bytes within an atom-column
-          const uint64_t bd = q_desc0 + (uint64_t)((u * 2 * NS * 128) >> 4);
-          const uint32_t ta = tbase + kColStg + x * 64;
+        // the unit's 8 K-steps: A = 8 TMEM columns each, B = 32 bytes within an atom-column
+        const uint64_t bd = q_desc0 + (uint64_t)((u * 2 * NS * 128) >> 4);
+        const uint32_t ta = tbase + kColStg + x * 64;
+        if (elect_one()) {
           if (u == 0)
             mma_ts_first(dS, ta, bd, kIdS);
           else
@@ -367,35 +375,38 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int k = 1; k < 8; ++k)
             mma_ts_acc(dS, ta + k * 8, bd + (uint64_t)(((k >> 2) * NS * 128 + (k & 3) * 32) >> 4), kIdS);
-          issued = true;
           mma_commit(&bars.stg_empty[x]);
         }
-        if (!ok) break;
-        mma_commit(&bars.sc_full[sb]);
+        __syncwarp();
+        issued = true;
       }
-      if (issued) {
-        // nothing may still be writing TMEM when it is freed
-        mma_commit(&bars.fin_s);
-        drain_wait(&bars.fin_s, 0);
-      }
+      if (!ok) break;
+      if (elect_one()) mma_commit(&bars.sc_full[sb]);
+      __syncwarp();
+    }
+    if (issued) {
+      // nothing may still be writing TMEM when it is freed
+      if (elect_one()) mma_commit(&bars.fin_s);
+      __syncwarp();
+      drain_wait(&bars.fin_s, 0);
     }
   } else if (warp == 2) {
-    // ------------------------------------------------------------ P.V-MMA issuer
-    if (lane == 0) {
-      const uint64_t pv_desc0 = sdesc_sw128(smem_addr(pvs), 16384, 1024);
-      const uint64_t p_desc0 = sdesc_sw128(smem_addr(ps), 16, 1024);
-      bool ok = true, issued = false;
-      for (int t = 0; t < n_tiles && ok; ++t) {
-        const int pb = t & 1;
-        if (!mbar_wait(&bars.p_full[pb], (t >> 1) & 1, abort_p, kWaitLimit)) { ok = false; break; }
+    // ------------------------------------------------------------ P.V-MMA issuer (whole warp, one lane issues)
+    const uint64_t pv_desc0 = sdesc_sw128(smem_addr(pvs), 16384, 1024);
+    const uint64_t p_desc0 = sdesc_sw128(smem_addr(ps), 16, 1024);
+    bool ok = true, issued = false;
+    for (int t = 0; t < n_tiles && ok; ++t) {
+      const int pb = t & 1;
+      if (!warp_wait(&bars.p_full[pb], (t >> 1) & 1, abort_p)) { ok = false; break; }
+      tc_fence_after();
+      const uint64_t pd = p_desc0 + (uint64_t)((pb * NP * 256) >> 4);
+      for (int u = 0; u < n_units; ++u) {
+        const int gp = t * n_units + u, x = u & 1;
+        if (!warp_wait(&bars.pv_full[x], (gp >> 1) & 1, abort_p)) { ok = false; break; }
         tc_fence_after();
-        const uint64_t pd = p_desc0 + (uint64_t)((pb * NP * 256) >> 4);
-        for (int u = 0; u < n_units; ++u) {
-          const int gp = t * n_units + u, x = u & 1;
-          if (!mbar_wait(&bars.pv_full[x], (gp >> 1) & 1, abort_p, kWaitLimit)) { ok = false; break; }
-          tc_fence_after();
-          const uint64_t ad = pv_desc0 + (uint64_t)((x * kPvStageBytes) >> 4);
-          const uint32_t du = tbase + kColU + u * NP;
+        const uint64_t ad = pv_desc0 + (uint64_t)((x * kPvStageBytes) >> 4);
+        const uint32_t du = tbase + kColU + u * NP;
+        if (elect_one()) {
           if (t == 0)
             mma_ss_first(du, ad, pd, kIdP);
           else
@@ -404,17 +415,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int k = 1; k < 8; ++k)
             mma_ss_acc(du, ad + (uint64_t)((k * 2048) >> 4),
                        pd + (uint64_t)((((k * 16) >> 6) * NP * 128 + ((k * 16) & 63) * 2) >> 4), kIdP);
-          issued = true;
           mma_commit(&bars.pv_empty[x]);
         }
-        if (!ok) break;
-        mma_commit(&bars.p_empty[pb]);
+        __syncwarp();
+        issued = true;
       }
-      if (ok) mma_commit(&bars.u_done);
-      if (issued) {
-        mma_commit(&bars.fin_v);
-        drain_wait(&bars.fin_v, 0);
-      }
+      if (!ok) break;
+      if (elect_one()) mma_commit(&bars.p_empty[pb]);
+      __syncwarp();
+    }
+    if (ok) {
+      if (elect_one()) mma_commit(&bars.u_done);
+      __syncwarp();
+    }
+    if (issued) {
+      if (elect_one()) mma_commit(&bars.fin_v);
+      __syncwarp();
+      drain_wait(&bars.fin_v, 0);
     }
   } else if (warp < kWarpV0) {
     // ------------------------------------------------------------ score group
