@@ -13,6 +13,10 @@
 //
 // Warps: 0 = TMA producer, 1 = MMA issuer / TMEM owner, 2-5 = epilogue
 // (TMEM -> registers -> global).  Waits are bounded like in the streaming kernel.
+//
+// Epilogues (GemmEpi): the absorbed-query GEMM writes the streaming kernel's operand
+// image straight from TMEM; the split-K GEMMs (q, out) write fp32 partials and the
+// last CTA to finish a 128-row block sums them in split order and writes the result.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -53,10 +57,23 @@ __device__ __forceinline__ void tma_load_2d_plain(void* dst, const void* tmap, i
 
 // A_MN: A given as W^T (MN-major): the tensor map covers W [K rows][M cols]; a stage loads
 // two 64 x 64 boxes (M halves).  Otherwise A = W [M rows][K cols], one 128 x 64 box.
+// The absorbed-query operand image: row j = fp16(qt_j) and, when the operands are split,
+// row 16 + j = fp16(qt_j - fp16(qt_j)); columns in the dequantised position order, 128-byte
+// swizzled atom-columns.
+__device__ __forceinline__ void put_qimg(const GemmEpiParams& e, int b, int j, int c, float v) {
+  const int rows = qimg_rows(e.s.d);
+  uint8_t* img = e.qimg + (size_t)b * qimg_bytes(e.s.d);
+  const int pos = phys_pos(e.s.fmt, c);
+  const __half hi = __float2half_rn(v);
+  *reinterpret_cast<__half*>(img + kmajor_offset(j, pos, rows)) = hi;
+  if (split_operands(e.s.d))
+    *reinterpret_cast<__half*>(img + kmajor_offset(16 + j, pos, rows)) = __float2half_rn(v - __half2float(hi));
+}
+
 template <bool A_MN>
 __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                                                          const __grid_constant__ CUtensorMap tmB,
-                                                         const GemmParams p) {
+                                                         const GemmParams p, const GemmEpiParams e) {
   const int mblk = blockIdx.x, split = blockIdx.y, z = blockIdx.z;
   const int N = p.N;
   const int nk = p.k_per_split / kBK;
@@ -70,6 +87,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
   __shared__ uint64_t full[kStages], empty[kStages], done;
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
+  __shared__ int is_last;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -154,15 +172,44 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
     const int row = quarter * 32 + lane;
     if (mbar_wait(&done, 0, abort_p, kGemmWaitLimit)) {
       tc_fence_after();
-      float* out = p.out + (((size_t)z * gridDim.y + split) * p.M + (size_t)mblk * 128 + row) * N;
-      for (int c = 0; c < N; c += 16) {
-        uint32_t v[16];
-        tmem_ld16(tbase + ((uint32_t)(quarter * 32) << 16) + c, v);
-        tmem_ld_wait();
+      const uint32_t trow = tbase + ((uint32_t)(quarter * 32) << 16);
+      if (e.mode == kEpiQImage) {
+        // qt[c][b] = hi column b + lo column nb + b, scaled by log2(e)/sqrt(hd); batch entry z = head
+        const int c = mblk * 128 + row;
+        const float scale = 1.4426950408889634f / sqrtf((float)e.s.hd);
+        for (int b0 = 0; b0 < e.nb; b0 += 16) {
+          uint32_t vh[16], vl[16];
+          tmem_ld16(trow + b0, vh);
+          tmem_ld16(trow + e.nb + b0, vl);
+          tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 16; i += 4)
-          *reinterpret_cast<float4*>(out + c + i) = make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
-                                                                __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
+          for (int i = 0; i < 16; ++i) {
+            const int b = b0 + i;
+            int nr;
+            if (b < e.n_lanes && lane_active(e.s, e.iter, e.loops, e.ctx_len, b, &nr))
+              put_qimg(e, b, z, c, (__uint_as_float(vh[i]) + __uint_as_float(vl[i])) * scale);
+          }
+        }
+        if (z == 0) {
+          // the rows of heads j >= H stay zero
+          for (int b = 0; b < e.n_lanes; ++b) {
+            int nr;
+            if (!lane_active(e.s, e.iter, e.loops, e.ctx_len, b, &nr)) continue;
+            for (int j = e.s.H; j < kMaxHeads; ++j) put_qimg(e, b, j, c, 0.0f);
+          }
+        }
+      } else {
+        float* out = p.out + (((size_t)z * gridDim.y + split) * p.M + (size_t)mblk * 128 + row) * N;
+        for (int c = 0; c < N; c += 16) {
+          uint32_t v[16];
+          tmem_ld16(trow + c, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; i += 4)
+            *reinterpret_cast<float4*>(out + c + i) = make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
+                                                                  __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
+        }
+        __threadfence();  // the partial is visible device-wide before this CTA is counted
       }
     }
   }
@@ -173,7 +220,97 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
     tc_fence_after();
     tmem_dealloc(tbase, 256);
   }
+  if (e.mode != kEpiQ && e.mode != kEpiOut) return;
+
+  // ---------------------------------------------------------------- split-K reduction by the last CTA
+  // Every CTA is counted exactly once (also after a timeout, so the counters stay consistent);
+  // the last one of the block resets its counter for the next call.
+  if (threadIdx.x == 0) {
+    uint32_t* cnt = e.counters + (size_t)z * gridDim.x + mblk;
+    const uint32_t old = atomicAdd(cnt, 1u);
+    is_last = old == gridDim.y - 1;
+    if (is_last) {
+      atomicExch(cnt, 0u);
+      __threadfence();
+    }
+  }
+  __syncthreads();
+  if (!is_last) return;
+  const int S = gridDim.y;
+  const int nb = e.nb;
+  if (e.mode == kEpiQ && mblk == 0 && warp == 0) {
+    // range check of the per-lane device values, once per decode call
+    for (int b = lane; b < e.n_lanes; b += 32) {
+      const int L = e.loops[b], c = e.ctx_len[b];
+      if (L < 0 || L > e.s.L_max || c < 0 || c >= e.s.max_ctx) atomicOr(e.status, kStatusRange);
+    }
+  }
+  // items (row, 4 lanes), spread over all threads; the split loads of an item are issued
+  // before they are summed (in split order, per component)
+  const int items = 128 * (nb / 4);
+  for (int it = threadIdx.x; it < items; it += blockDim.x) {
+    const int row = it / (nb / 4), b0 = (it % (nb / 4)) * 4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (e.mode == kEpiQ) {
+      const int r = mblk * 128 + row;
+      for (int sp0 = 0; sp0 < S; sp0 += 8) {
+        float4 t[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          if (sp0 + k < S) t[k] = __ldcg(reinterpret_cast<const float4*>(p.out + ((size_t)(sp0 + k) * p.M + r) * N + b0));
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          if (sp0 + k < S) {
+            acc.x += t[k].x;
+            acc.y += t[k].y;
+            acc.z += t[k].z;
+            acc.w += t[k].w;
+          }
+      }
+      const float qv[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int b = b0 + i;
+        int nr;
+        const float q = (b < e.n_lanes && lane_active(e.s, e.iter, e.loops, e.ctx_len, b, &nr)) ? qv[i] : 0.0f;
+        const __half hi = __float2half_rn(q);
+        e.qhl[(size_t)b * e.s.d + r] = hi;
+        e.qhl[(size_t)(nb + b) * e.s.d + r] = __float2half_rn(q - __half2float(hi));
+      }
+    } else {
+      // out feature 128 z + row; with hd = 64 a block holds two heads, whose u columns start at 2 nb
+      if (b0 >= e.n_lanes) continue;
+      const int c0 = e.s.hd == 64 ? (row >> 6) * 2 * nb : 0;
+      for (int sp0 = 0; sp0 < S; sp0 += 8) {
+        float4 th[8], tl[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          if (sp0 + k < S) {
+            const float* pr = p.out + (((size_t)z * S + sp0 + k) * 128 + row) * N + c0 + b0;
+            th[k] = __ldcg(reinterpret_cast<const float4*>(pr));
+            tl[k] = __ldcg(reinterpret_cast<const float4*>(pr + nb));
+          }
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          if (sp0 + k < S) {
+            acc.x += th[k].x + tl[k].x;
+            acc.y += th[k].y + tl[k].y;
+            acc.z += th[k].z + tl[k].z;
+            acc.w += th[k].w + tl[k].w;
+          }
+      }
+      const float ov[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int b = b0 + i;
+        int nr;
+        if (b < e.n_lanes && lane_active(e.s, e.iter, e.loops, e.ctx_len, b, &nr))
+          e.out[(size_t)b * e.s.d + (size_t)z * 128 + row] = ov[i];
+      }
+    }
+  }
 }
+
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -206,7 +343,7 @@ bool make_tmap_f16(void* tmap, const void* base, uint64_t rows, uint64_t cols, u
 
 cudaError_t launch_gemm_tc(bool a_mn, const void* tmA, const void* tmB, int M, int N, int K, int splits, int batch,
                            int a_x_per_z, int a_y_per_z, int b_x_per_z, int b_y_per_z, float* out, uint32_t* status,
-                           cudaStream_t st) {
+                           const GemmEpiParams& epi, cudaStream_t st) {
   if (M % 128 || N % 16 || N < 16 || N > 256 || K % (kBK * splits)) return cudaErrorInvalidValue;
   GemmParams p{M, N, K / splits, a_y_per_z, b_y_per_z, b_x_per_z, a_x_per_z, out, status};
   const size_t smem = (size_t)kStages * (kABytes + N * 128) + 1024;
@@ -216,12 +353,12 @@ cudaError_t launch_gemm_tc(bool a_mn, const void* tmA, const void* tmB, int M, i
     e = cudaFuncSetAttribute(gemm_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     gemm_tc_kernel<true><<<grid, 192, smem, st>>>(*reinterpret_cast<const CUtensorMap*>(tmA),
-                                                  *reinterpret_cast<const CUtensorMap*>(tmB), p);
+                                                  *reinterpret_cast<const CUtensorMap*>(tmB), p, epi);
   } else {
     e = cudaFuncSetAttribute(gemm_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     gemm_tc_kernel<false><<<grid, 192, smem, st>>>(*reinterpret_cast<const CUtensorMap*>(tmA),
-                                                   *reinterpret_cast<const CUtensorMap*>(tmB), p);
+                                                   *reinterpret_cast<const CUtensorMap*>(tmB), p, epi);
   }
   count_launch();
   return cudaGetLastError();

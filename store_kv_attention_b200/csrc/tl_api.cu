@@ -158,8 +158,8 @@ tl_status tl_residual_norm_check(const float* residual, int32_t n_lanes, int32_t
     return fail(TL_ERR_INVALID_ARG, "residual / abort_flags / first_abort_iter is NULL");
   if (n_lanes <= 0 || d <= 0 || iter < 0) return fail(TL_ERR_INVALID_ARG, "n_lanes %d, d %d, iter %d", n_lanes, d, iter);
   if (!(threshold >= 0.0f)) return fail(TL_ERR_INVALID_ARG, "threshold must be a non-negative number");
-  cudaError_t e = tl::launch_norm_check(residual, n_lanes, d, threshold, iter, loops, nullptr, 0, 0, abort_flags,
-                                        first_abort_iter, norms_out, (cudaStream_t)stream);
+  cudaError_t e = tl::launch_norm_check(residual, n_lanes, d, threshold, iter, loops, abort_flags, first_abort_iter,
+                                        norms_out, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "tl_residual_norm_check launch");
   return TL_OK;
 }
@@ -193,7 +193,7 @@ tl_status tl_storeh_attn_decode(const tl_storeh_desc* desc, tl_storeh_cache cach
 
   tl::DecodeArgs a{s, cache.codes, cache.scales, iter, loops, ctx_len, (const __half*)h_new,
                    (const __half*)W_q, (const __half*)W_k, (const __half*)W_v, out, n_lanes,
-                   (uint8_t*)workspace, wl};
+                   (uint8_t*)workspace, wl, residual, threshold, abort_flags, first_abort_iter, norms_out};
   cudaStream_t cs = (cudaStream_t)stream;
   cudaError_t e = tl::launch_prologue(a, cs);
   if (e != cudaSuccess) return cuda_fail(e, "decode prologue launch");
@@ -203,11 +203,6 @@ tl_status tl_storeh_attn_decode(const tl_storeh_desc* desc, tl_storeh_cache cach
   if (e != cudaSuccess) return cuda_fail(e, "decode stream launch");
   e = tl::launch_epilogue(a, cs);
   if (e != cudaSuccess) return cuda_fail(e, "decode epilogue launch");
-  if (residual) {
-    e = tl::launch_norm_check(residual, n_lanes, s.d, threshold, iter, loops, ctx_len, s.max_ctx, s.L_max,
-                              abort_flags, first_abort_iter, norms_out, cs);
-    if (e != cudaSuccess) return cuda_fail(e, "decode norm check launch");
-  }
   return TL_OK;
 }
 
@@ -219,7 +214,7 @@ tl_status tl_storeh_poll_status(void* workspace, size_t workspace_bytes, tl_stre
   if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
   if (e != cudaSuccess) return cuda_fail(e, "reading the status word");
   if (word != 0) {
-    e = cudaMemsetAsync(workspace, 0, sizeof word, cs);
+    e = cudaMemsetAsync(workspace, 0, 256, cs);  // the status word and the reduction counters
     if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
     if (e != cudaSuccess) return cuda_fail(e, "clearing the status word");
   }

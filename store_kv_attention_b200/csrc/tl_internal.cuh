@@ -153,10 +153,9 @@ cudaError_t launch_append(const Shape& s, void* codes, void* scales, int layer, 
                           int n_lanes, int n_rows, const int32_t* start_pos, const int32_t* row_count,
                           const int32_t* loops, cudaStream_t st);
 
-// ctx_len == NULL: standalone check; otherwise lanes with out-of-range loops/ctx_len are skipped.
+// Standalone safety check of tl_residual_norm_check (lanes with iter >= loops[b] skipped when loops is given).
 cudaError_t launch_norm_check(const float* residual, int n_lanes, int d, float threshold, int iter,
-                              const int32_t* loops, const int32_t* ctx_len, int max_ctx, int L_max, uint8_t* flags,
-                              int32_t* first, float* norms, cudaStream_t st);
+                              const int32_t* loops, uint8_t* flags, int32_t* first, float* norms, cudaStream_t st);
 
 struct DecodeArgs {
   Shape s;
@@ -173,6 +172,12 @@ struct DecodeArgs {
   int n_lanes;
   uint8_t* ws;
   Workspace wl;
+  // per-iteration safety check fused into the decode (residual == NULL: none)
+  const float* residual;
+  float threshold;
+  uint8_t* abort_flags;
+  int32_t* first_abort_iter;
+  float* norms;
 };
 
 cudaError_t launch_prologue(const DecodeArgs& a, cudaStream_t st);
@@ -180,9 +185,34 @@ cudaError_t launch_prologue(const DecodeArgs& a, cudaStream_t st);
 // tensor-core skinny GEMM (k_gemm_tc.cu)
 bool make_tmap_f16(void* tmap, const void* base, uint64_t rows, uint64_t cols, uint64_t pitch_elems,
                    uint32_t box_cols, uint32_t box_rows);
+// Epilogues of the decode GEMMs (k_gemm_tc.cu).  The split-K modes write their fp32
+// partials, and the last CTA of each 128-row block (an arrival counter, reset by that CTA)
+// sums them in split order and writes the final values, so the result does not depend on
+// scheduling.
+enum GemmEpi : int {
+  kEpiPartials = 0,  // fp32 partials only
+  kEpiQ = 1,         // q = W_q h_new: reduce the splits, write fp16 hi/lo rows of q (the next GEMM's B)
+  kEpiQImage = 2,    // qt_j = W_k[j]^T q_j: write the streaming kernel's absorbed-query operand image
+  kEpiOut = 3,       // out_j = W_v[j] u_j: reduce the splits, write out
+};
+struct GemmEpiParams {
+  int mode;
+  Shape s;
+  int iter;
+  const int32_t* loops;
+  const int32_t* ctx_len;
+  int n_lanes, nb;
+  uint32_t* counters;  // split-K modes: one per (batch entry, 128-row block), zero between calls
+  uint32_t* status;    // device status word (kEpiQ records out-of-range lanes)
+  __half* qhl;         // kEpiQ: [2 nb][d], hi rows then lo rows
+  uint8_t* qimg;       // kEpiQImage: [n_lanes][qimg_bytes(d)]
+  float* out;          // kEpiOut: [n_lanes][d]
+};
+// Offsets of the arrival counters inside the 256-byte status block of the workspace.
+constexpr size_t kCountersQOff = 64, kCountersOOff = 128;
 cudaError_t launch_gemm_tc(bool a_mn, const void* tmA, const void* tmB, int M, int N, int K, int splits, int batch,
                            int a_x_per_z, int a_y_per_z, int b_x_per_z, int b_y_per_z, float* out, uint32_t* status,
-                           cudaStream_t st);
+                           const GemmEpiParams& epi, cudaStream_t st);
 cudaError_t launch_stream(const DecodeArgs& a, cudaStream_t st);
 cudaError_t launch_epilogue(const DecodeArgs& a, cudaStream_t st);
 
