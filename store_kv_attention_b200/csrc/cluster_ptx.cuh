@@ -1,0 +1,45 @@
+// Thread-block-cluster helpers (sm_100a): cluster barrier, rank, and distributed
+// shared memory (DSMEM) loads and stores into the shared memory of another CTA of the
+// same cluster.  No TMA multicast is used anywhere.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+namespace tl {
+namespace ptx {
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Every thread of every CTA of the cluster must execute both halves, in the same order.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Shared::cluster address of `smem_cta_addr` (a shared::cta address) in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t dsmem_addr(uint32_t smem_cta_addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_cta_addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float4 dsmem_ld_f4(uint32_t cluster_addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(cluster_addr)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ void dsmem_st_b16(uint32_t cluster_addr, __half v) {
+  asm volatile("st.shared::cluster.b16 [%0], %1;" ::"r"(cluster_addr), "h"(__half_as_ushort(v)) : "memory");
+}
+// Orders this thread's generic-proxy shared-memory writes (local or remote) before later
+// async-proxy reads (tensor-core operands) of the cluster.
+__device__ __forceinline__ void fence_proxy_async_cluster() {
+  asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
+}
+
+}  // namespace ptx
+}  // namespace tl

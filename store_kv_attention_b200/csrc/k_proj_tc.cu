@@ -1,0 +1,405 @@
+// Fused projections of one decode iteration on tensor cores, one thread-block cluster per
+// 128-row block of the projection matrix.
+// [Novel Contributions, "Novel Mechanism: Store-h KV Cache": K = W_k h, V = W_v h with the
+//  loop block's shared weights, used here in the absorbed form]
+//
+// qproj (one launch):  q = W_q h_new, then qt_j = W_k[j]^T q_j . log2(e)/sqrt(hd)
+//   Cluster mb owns rows [128 mb, 128 mb + 128) of q, i.e. one head (hd = 128) or two
+//   (hd = 64).  Rank k of the cluster computes the K-split k of those rows into TMEM; the
+//   splits are reduced through distributed shared memory (rank k sums rows of its own
+//   share over all ranks, in rank order, into its own copy of the fp16 hi/lo B operand of
+//   the second GEMM, then every rank pulls the others' rows), whose A operand (W_k^T,
+//   read MN-major) was prefetched by TMA at kernel start.  Each rank then computes its
+//   share of the (head, 128-column block) items of qt and writes the streaming kernel's
+//   absorbed-query operand image directly.
+//
+// Every reduction runs in a fixed order, so a lane's result does not depend on the
+// other lanes of the batch or on scheduling.  All mbarrier waits are bounded; every
+// thread reaches all three cluster barriers whatever happened before them.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <math_constants.h>
+
+#include "cluster_ptx.cuh"
+#include "tc_ptx.cuh"
+#include "tl_internal.cuh"
+
+namespace tl {
+namespace {
+
+using namespace ptx;
+
+constexpr int kProjThreads = 128;                // four warps: TMEM lane quarters 0-3
+constexpr int kTileBytes = 128 * 64 * 2;         // one 128 x 64 fp16 operand tile
+constexpr long long kProjWaitLimit = 4000000000ll;
+
+__device__ __forceinline__ void tma_2d(void* dst, const void* tmap, int32_t x, int32_t y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_addr(bar))
+      : "memory");
+}
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile("{\n .reg .pred p;\n elect.sync _|p, 0xffffffff;\n selp.u32 %0, 1, 0, p;\n}\n" : "=r"(pred));
+  return pred != 0;
+}
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return p + ((1024 - (smem_addr(p) & 1023)) & 1023);
+}
+
+// The absorbed-query operand image of a lane: row j = fp16(qt_j) and, when the operands
+// are split, row 16 + j = fp16(qt_j - fp16(qt_j)); columns in the dequantised position
+// order, 128-byte swizzled atom-columns of 64 positions (kmajor_offset).
+
+struct QProjParams {
+  Shape s;
+  int iter;
+  const int32_t* loops;
+  const int32_t* ctx_len;
+  int n_lanes, nb;
+  int cl;            // cluster size = K splits of q
+  uint32_t* status;
+  uint8_t* qimg;     // [n_lanes][qimg_bytes(d)]
+};
+
+// Shared memory: region 0 holds the phase-1 operands; once the phase-1 MMAs are done it
+// holds the fp32 partial (read by the other ranks) followed by the phase-2 W_k^T tiles,
+// loaded then, and finally the image staging.  Small enough for two CTAs per SM when
+// nb <= 32, so all clusters of a launch are resident at once.
+struct QProjLayout {
+  int KS, nk1, heads_in_block, mblocks, items, ipr, kst2;
+  uint32_t part_bytes, region0, a2_bytes, b2_bytes, total;
+  uint32_t tmem_cols;  // 128 per phase-2 item (phase 1 uses columns 0..nb-1 first)
+  __host__ __device__ QProjLayout(const Shape& s, int nb, int cl) {
+    KS = s.d / cl;
+    nk1 = KS / 64;
+    heads_in_block = 128 / s.hd;
+    mblocks = s.d / 128;
+    items = heads_in_block * mblocks;
+    ipr = (items + cl - 1) / cl;
+    kst2 = s.hd / 64;
+    const uint32_t ld1 = (uint32_t)nk1 * (kTileBytes + nb * 128);
+    const uint32_t stage = 2u * nb * 128u * 2u;             // image staging [hl][nb][128] fp16
+    const uint32_t part = 128u * (uint32_t)(nb + 4) * 4u;  // fp32 partial, rows padded by 4 floats
+    part_bytes = ((part > stage ? part : stage) + 1023u) & ~1023u;
+    a2_bytes = (uint32_t)ipr * kst2 * kTileBytes;
+    region0 = ((ld1 > part_bytes + a2_bytes ? ld1 : part_bytes + a2_bytes) + 1023u) & ~1023u;
+    b2_bytes = 2u * 2u * nb * 128u;  // two atom-columns of 2 nb rows
+    total = 1024u + region0 + b2_bytes;
+    tmem_cols = ipr <= 1 ? 128u : ipr <= 2 ? 256u : 512u;
+  }
+};
+
+__global__ void __launch_bounds__(kProjThreads, 1)
+    qproj_kernel(const __grid_constant__ CUtensorMap tmWq, const __grid_constant__ CUtensorMap tmH,
+                 const __grid_constant__ CUtensorMap tmWk, const QProjParams p) {
+  const Shape& s = p.s;
+  const int nb = p.nb, CL = p.cl;
+  const QProjLayout lay(s, nb, CL);
+  const int k = (int)cluster_rank();  // K split of q; also selects this rank's phase-2 items
+  const int mb = blockIdx.y;          // 128-row block of q
+  const int it0 = k * lay.ipr, it1 = min(lay.items, it0 + lay.ipr);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = (warp & 3) * 32 + lane;  // TMEM lane of this thread
+  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = align1024(smem_raw);
+  uint8_t* a1 = base;                                // nk1 tiles of W_q
+  uint8_t* b1 = a1 + lay.nk1 * kTileBytes;           // nk1 tiles of h_new (nb rows)
+  float* part = reinterpret_cast<float*>(base);      // after phase-1 MMAs: fp32 partial [128][nb + 4]
+  uint8_t* a2 = base + lay.part_bytes;               // phase-2 W_k^T tiles, two 64 x 64 boxes per stage
+  uint8_t* b2 = base + lay.region0;                  // q hi/lo operand [2 nb][128], K-major swizzled
+  __shared__ uint64_t bar_ld1, bar_ld2, bar_m1, bar_m2;
+  __shared__ uint32_t tmem_base;
+  __shared__ int abort_flag;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bar_ld1, 1);
+    mbar_init(&bar_ld2, 1);
+    mbar_init(&bar_m1, 1);
+    mbar_init(&bar_m2, 1);
+    abort_flag = 0;
+    mbar_fence_init();
+    tma_prefetch_desc(&tmWq);
+    tma_prefetch_desc(&tmH);
+    tma_prefetch_desc(&tmWk);
+  }
+  if (warp == 0) {
+    tmem_alloc(&tmem_base, lay.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = tmem_base;
+  volatile int* abort_p = &abort_flag;
+
+  // ---------------------------------------------------------------- phase-1 loads (phase 2 loads once they are dead)
+  if (threadIdx.x == 0) {
+    mbar_expect_tx(&bar_ld1, (uint32_t)lay.nk1 * (kTileBytes + nb * 128));
+    for (int i = 0; i < lay.nk1; ++i) {
+      const int x = k * lay.KS + 64 * i;
+      tma_2d(a1 + i * kTileBytes, &tmWq, x, mb * 128, &bar_ld1);
+      tma_2d(b1 + i * nb * 128, &tmH, x, 0, &bar_ld1);  // rows past n_lanes read as zero
+    }
+  }
+
+  // ---------------------------------------------------------------- phase 1: K split k of q
+  if (warp == 1) {
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_ld1, 0, abort_p, kProjWaitLimit));
+    if (ok) {
+      tc_fence_after();
+      if (elect_one()) {
+        const uint32_t id1 = idesc_f16_f32(128, nb, false, false);
+        for (int i = 0; i < lay.nk1; ++i) {
+          const uint64_t ad = sdesc_sw128(smem_addr(a1 + i * kTileBytes), 16, 1024);
+          const uint64_t bd = sdesc_sw128(smem_addr(b1 + i * nb * 128), 16, 1024);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(tbase, ad + (uint64_t)((kk * 32) >> 4), bd + (uint64_t)((kk * 32) >> 4), id1, (i | kk) != 0);
+        }
+        mma_commit(&bar_m1);
+      }
+      __syncwarp();
+    }
+  }
+  // partial -> own shared memory (the phase-1 operands are dead once the MMAs are done)
+  const int pstride = nb + 4;
+  if (mbar_wait(&bar_m1, 0, abort_p, kProjWaitLimit)) {
+    tc_fence_after();
+    if (threadIdx.x == 0) {
+      // the phase-1 operands are dead: load the phase-2 W_k^T tiles behind the partial
+      if (it1 > it0) {
+        mbar_expect_tx(&bar_ld2, (uint32_t)(it1 - it0) * lay.kst2 * kTileBytes);
+        for (int it = it0; it < it1; ++it) {
+          const int h2 = it / lay.mblocks, mc = it % lay.mblocks;
+          const int j = mb * lay.heads_in_block + h2;
+          for (int st = 0; st < lay.kst2; ++st) {
+            uint8_t* dst = a2 + ((it - it0) * lay.kst2 + st) * kTileBytes;
+            tma_2d(dst, &tmWk, mc * 128, j * s.hd + 64 * st, &bar_ld2);
+            tma_2d(dst + kTileBytes / 2, &tmWk, mc * 128 + 64, j * s.hd + 64 * st, &bar_ld2);
+          }
+        }
+      }
+    }
+    for (int c0 = 0; c0 < nb; c0 += 16) {
+      uint32_t v[16];
+      tmem_ld16(tbase + lane_off + c0, v);
+      tmem_ld_wait();
+      float* dst = part + row * pstride + c0;
+#pragma unroll
+      for (int i = 0; i < 16; i += 4)
+        *reinterpret_cast<float4*>(dst + i) = make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
+                                                          __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
+    }
+  }
+  tc_fence_before();
+  cluster_sync();  // 1: every rank's partial is in place
+
+  // ---------------------------------------------------------------- reduce the K splits through DSMEM
+  // Rank k owns rows [k * 128/CL, (k+1) * 128/CL): it sums them over all ranks in rank order
+  // and writes fp16 hi (operand row b) and lo (row nb + b) into every rank's B operand.
+  if (mb == 0 && k == 0 && warp == 0) {
+    // range check of the per-lane device values, once per decode call
+    for (int b = lane; b < p.n_lanes; b += 32) {
+      const int L = p.loops[b], c = p.ctx_len[b];
+      if (L < 0 || L > s.L_max || c < 0 || c >= s.max_ctx) atomicOr(p.status, kStatusRange);
+    }
+  }
+  // lanes active in this iteration (n_lanes <= 64)
+  uint64_t act = 0;
+  for (int b = 0; b < p.n_lanes; ++b) {
+    int nr;
+    if (lane_active(s, p.iter, p.loops, p.ctx_len, b, &nr)) act |= 1ull << b;
+  }
+  const int rpr = 128 / CL;
+  {
+    const int nq = nb / 4;
+    const uint32_t part_s = smem_addr(part);
+    for (int it = threadIdx.x; it < rpr * nq; it += kProjThreads) {
+      const int r = k * rpr + it / nq, b0 = (it % nq) * 4;
+      float4 v[8];
+#pragma unroll
+      for (int rk = 0; rk < 8; ++rk)
+        if (rk < CL) v[rk] = dsmem_ld_f4(dsmem_addr(part_s + (uint32_t)((r * pstride + b0) * 4), (uint32_t)rk));
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int rk = 0; rk < 8; ++rk)
+        if (rk < CL) {
+          acc.x += v[rk].x;
+          acc.y += v[rk].y;
+          acc.z += v[rk].z;
+          acc.w += v[rk].w;
+        }
+      const float qv[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int b = b0 + i;
+        const float q = ((act >> b) & 1) ? qv[i] : 0.0f;
+        const __half hi = __float2half_rn(q);
+        *reinterpret_cast<__half*>(b2 + kmajor_offset(b, r, 2 * nb)) = hi;
+        *reinterpret_cast<__half*>(b2 + kmajor_offset(nb + b, r, 2 * nb)) = __float2half_rn(q - __half2float(hi));
+      }
+    }
+  }
+  cluster_sync();  // 2: every rank's reduced rows are in its own B operand
+  {
+    // pull the other ranks' rows: rows [r0, r0 + rpr) of operand row n are 2 rpr bytes
+    // (rpr/8 16-byte chunks) at the same swizzled offsets in every rank's copy
+    const uint32_t b2_s = smem_addr(b2);
+    const int chunks = rpr / 8;
+    const int per_rank = 2 * nb * chunks;
+    const int total = CL * per_rank;
+    for (int it0p = threadIdx.x; it0p < total; it0p += 4 * kProjThreads) {
+      float4 v[4];
+      uint32_t off[4];
+      bool use[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int it = it0p + u * kProjThreads;
+        const int rk = it / per_rank;
+        use[u] = it < total && rk != k;
+        const int n = (it % per_rank) / chunks, ch = it % chunks;
+        off[u] = kmajor_offset(n, rk * rpr + ch * 8, 2 * nb);  // 16-byte aligned chunk
+        if (use[u]) v[u] = dsmem_ld_f4(dsmem_addr(b2_s + off[u], (uint32_t)rk));
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (use[u]) *reinterpret_cast<float4*>(b2 + off[u]) = v[u];
+    }
+  }
+  fence_proxy_async_smem();
+  cluster_sync();  // 3: no DSMEM access after this point
+
+  // ---------------------------------------------------------------- phase 2: qt = W_k^T q
+  // item (h2, mc): head mb * heads_in_block + h2, output columns [128 mc, 128 mc + 128);
+  // D of item i at TMEM column 128 i (D of phase 1 is dead by now).
+  const bool has_items = it1 > it0;
+  if (warp == 1 && has_items) {
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_ld2, 0, abort_p, kProjWaitLimit));
+    if (ok) {
+      fence_proxy_async_smem();
+      tc_fence_after();
+      if (elect_one()) {
+        const uint32_t id2 = idesc_f16_f32(128, 2 * nb, true, false);
+        for (int it = it0; it < it1; ++it) {
+          const int i = it - it0, h2 = it / lay.mblocks;
+          for (int st = 0; st < lay.kst2; ++st) {
+            const uint64_t ad = sdesc_sw128(smem_addr(a2 + (i * lay.kst2 + st) * kTileBytes), kTileBytes / 2, 1024);
+            // K rows [h2 hd + 64 st, +64) of the q block = atom-column h2 kst2 + st of the B operand
+            const uint64_t bd = sdesc_sw128(smem_addr(b2 + (h2 * lay.kst2 + st) * 2 * nb * 128), 16, 1024);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ss(tbase + 128 * i, ad + (uint64_t)((kk * 2048) >> 4), bd + (uint64_t)((kk * 32) >> 4), id2,
+                     (st | kk) != 0);
+          }
+        }
+        mma_commit(&bar_m2);
+      }
+      __syncwarp();
+    }
+  }
+  // Image epilogue, one item at a time: fp16 hi/lo values are staged in shared memory in the
+  // image's physical position order (the dead phase-1 region), then copied out as 16-byte
+  // chunks at their swizzled image offsets.  The item loop count is the same for all threads.
+  const bool split = split_operands(s.d);
+  const int nhl = split ? 2 : 1;
+  const int rows_img = qimg_rows(s.d);
+  __half* stg = reinterpret_cast<__half*>(base);  // [hl][nb][128]
+  const bool ok2 = has_items && mbar_wait(&bar_m2, 0, abort_p, kProjWaitLimit);
+  const float scale = 1.4426950408889634f / sqrtf((float)s.hd);
+  for (int it = it0; it < it1; ++it) {
+    const int i = it - it0, h2 = it / lay.mblocks, mc = it % lay.mblocks;
+    const int j = mb * lay.heads_in_block + h2;
+    if (ok2) {
+      tc_fence_after();
+      const int pp = phys_pos(s.fmt, row);  // blocks are 128-aligned, so the permutation is local
+      for (int b0 = 0; b0 < nb; b0 += 16) {
+        uint32_t vh[16], vl[16];
+        tmem_ld16(tbase + lane_off + 128 * i + b0, vh);
+        tmem_ld16(tbase + lane_off + 128 * i + nb + b0, vl);
+        tmem_ld_wait();
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          const float v = (__uint_as_float(vh[q]) + __uint_as_float(vl[q])) * scale;
+          const __half hi = __float2half_rn(v);
+          stg[(b0 + q) * 128 + pp] = hi;
+          if (split) stg[(nb + b0 + q) * 128 + pp] = __float2half_rn(v - __half2float(hi));
+        }
+      }
+    }
+    __syncthreads();
+    if (ok2) {
+      for (int x = threadIdx.x; x < nhl * nb * 16; x += kProjThreads) {
+        const int hl = x / (nb * 16), b = (x / 16) % nb, g = x % 16;
+        if (!((act >> b) & 1)) continue;
+        const uint4 v = *reinterpret_cast<const uint4*>(stg + (hl * nb + b) * 128 + 8 * g);
+        uint8_t* img = p.qimg + (size_t)b * qimg_bytes(s.d);
+        *reinterpret_cast<uint4*>(img + kmajor_offset(16 * hl + j, mc * 128 + 8 * g, rows_img)) = v;
+      }
+    }
+    __syncthreads();
+  }
+  if (mb == 0 && s.H < kMaxHeads) {
+    // the rows of heads j >= H stay zero; rank k covers columns [k d/CL, (k+1) d/CL)
+    const int cs = s.d / CL, groups = cs / 8;
+    const int per_lane = (kMaxHeads - s.H) * nhl * groups;
+    for (int x = threadIdx.x; x < p.n_lanes * per_lane; x += kProjThreads) {
+      const int b = x / per_lane;
+      if (!((act >> b) & 1)) continue;
+      const int y = x % per_lane;
+      const int j = s.H + y / (nhl * groups), hl = (y / groups) % nhl, g = y % groups;
+      uint8_t* img = p.qimg + (size_t)b * qimg_bytes(s.d);
+      *reinterpret_cast<uint4*>(img + kmajor_offset(16 * hl + j, k * cs + 8 * g, rows_img)) = make_uint4(0, 0, 0, 0);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && abort_flag) atomicOr(p.status, kStatusTimeout);
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tbase, lay.tmem_cols);
+  }
+}
+
+}  // namespace
+
+// Cluster size of the projection kernels: K splits of d, each a multiple of 64 wide.
+int proj_cluster(int d) { return d / 64 < 8 ? d / 64 : 8; }
+
+cudaError_t launch_qproj(const DecodeArgs& a, cudaStream_t st) {
+  const Shape& s = a.s;
+  const Workspace& w = a.wl;
+  const int CL = proj_cluster(s.d);
+  const QProjLayout lay(s, w.nb, CL);
+  alignas(64) CUtensorMap tmWq, tmH, tmWk;
+  if (!make_tmap_f16(&tmWq, a.Wq, s.d, s.d, s.d, 64, 128) || !make_tmap_f16(&tmH, a.h_new, a.n_lanes, s.d, s.d, 64, w.nb) ||
+      !make_tmap_f16(&tmWk, a.Wk, s.d, s.d, s.d, 64, 64))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(qproj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lay.total);
+  if (e != cudaSuccess) return e;
+  QProjParams p{s, a.iter, a.loops, a.ctx_len, a.n_lanes, w.nb, CL,
+                reinterpret_cast<uint32_t*>(a.ws + w.status_off), a.ws + w.qt_off};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(CL, s.d / 128, 1);
+  cfg.blockDim = dim3(kProjThreads, 1, 1);
+  cfg.dynamicSmemBytes = lay.total;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, qproj_kernel, tmWq, tmH, tmWk, p);
+  count_launch();
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace tl

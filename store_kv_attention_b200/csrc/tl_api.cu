@@ -195,7 +195,7 @@ tl_status tl_storeh_attn_decode(const tl_storeh_desc* desc, tl_storeh_cache cach
                    (const __half*)W_q, (const __half*)W_k, (const __half*)W_v, out, n_lanes,
                    (uint8_t*)workspace, wl, residual, threshold, abort_flags, first_abort_iter, norms_out};
   cudaStream_t cs = (cudaStream_t)stream;
-  cudaError_t e = tl::launch_prologue(a, cs);
+  cudaError_t e = tl::launch_qproj(a, cs);
   if (e != cudaSuccess) return cuda_fail(e, "decode prologue launch");
   tl::profile_stream_begin(cs);
   e = tl::launch_stream(a, cs);

@@ -181,6 +181,9 @@ struct DecodeArgs {
 };
 
 cudaError_t launch_prologue(const DecodeArgs& a, cudaStream_t st);
+// Fused q and absorbed-query projections, one thread-block cluster per 128 rows of W_q (k_proj_tc.cu).
+cudaError_t launch_qproj(const DecodeArgs& a, cudaStream_t st);
+int proj_cluster(int d);
 
 // tensor-core skinny GEMM (k_gemm_tc.cu)
 bool make_tmap_f16(void* tmap, const void* base, uint64_t rows, uint64_t cols, uint64_t pitch_elems,
