@@ -21,6 +21,7 @@
 #include <math_constants.h>
 
 #include "cluster_ptx.cuh"
+#include "norm_block.cuh"
 #include "tc_ptx.cuh"
 #include "tl_internal.cuh"
 
@@ -366,6 +367,241 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   }
 }
 
+// ================================================================ oproj
+// oproj (one launch): merge the splits of u, out_j = W_v[j] u_j, and the safety check.
+//   Cluster mb owns output features [128 mb, 128 mb + 128), i.e. rows of W_v of one head
+//   (hd = 128) or two (hd = 64).  Rank k owns the K slice [k KS, (k+1) KS) of u: it merges
+//   the streaming kernel's split partials exactly for that slice,
+//     u_j = sum_s 2^(m_s - M) U_s / sum_s 2^(m_s - M) l_s   (the same order and operations
+//   as a separate merge), writes it as the fp16 hi/lo B operand in shared memory, and
+//   multiplies it with its W_v tile (prefetched at kernel start).  The K slices are reduced
+//   through DSMEM in rank order, as in qproj.  CTA (k, mb) also runs the per-iteration
+//   safety check of lane mb * CL + k.
+struct OProjParams {
+  Shape s;
+  int iter;
+  const int32_t* loops;
+  const int32_t* ctx_len;
+  int n_lanes, nb, cl, s_max;
+  const float* ml;  // [n_lanes][s_max][16][2]
+  const float* U;   // [n_lanes][s_max][16][d]
+  float* out;       // [n_lanes][d]
+  uint32_t* status;
+  const float* residual;
+  float threshold;
+  uint8_t* flags;
+  int32_t* first;
+  float* norms;
+};
+
+struct OProjLayout {
+  int KS, nk, hib, N;
+  uint32_t a_bytes, b_bytes, part_bytes, w_bytes, region0, total, tmem_cols;
+  __host__ __device__ OProjLayout(const Shape& s, int nb, int cl, int n_lanes, int s_max) {
+    KS = s.d / cl;
+    nk = KS / 64;
+    hib = 128 / s.hd;  // heads in the block
+    N = hib * 2 * nb;  // operand rows: per head, nb hi rows then nb lo rows
+    a_bytes = (uint32_t)nk * kTileBytes;
+    part_bytes = 128u * (uint32_t)(N + 4) * 4u;
+    region0 = ((a_bytes > part_bytes ? a_bytes : part_bytes) + 1023u) & ~1023u;
+    b_bytes = (uint32_t)N * KS * 2u;
+    w_bytes = (((uint32_t)n_lanes * hib * s_max * 4u) + 1023u) & ~1023u;
+    total = 1024u + region0 + b_bytes + w_bytes;
+    tmem_cols = N <= 32 ? 32u : N <= 64 ? 64u : N <= 128 ? 128u : 256u;
+  }
+};
+
+__global__ void __launch_bounds__(kProjThreads, 1)
+    oproj_kernel(const __grid_constant__ CUtensorMap tmWv, const OProjParams p) {
+  const Shape& s = p.s;
+  const int nb = p.nb, CL = p.cl;
+  const OProjLayout lay(s, nb, CL, p.n_lanes, p.s_max);
+  const int k = (int)cluster_rank();
+  const int mb = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = (warp & 3) * 32 + lane;
+  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+  const int N = lay.N;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = align1024(smem_raw);
+  uint8_t* a = base;                                   // nk W_v tiles (128 x 64)
+  float* part = reinterpret_cast<float*>(base);        // after the MMAs: fp32 partial [128][N + 4]
+  uint8_t* bop = base + lay.region0;                   // u hi/lo operand [N][KS], K-major swizzled
+  float* wgt = reinterpret_cast<float*>(bop + lay.b_bytes);  // [n_lanes][hib][s_max] merge weights
+  __shared__ uint64_t bar_ld, bar_m;
+  __shared__ uint32_t tmem_base;
+  __shared__ int abort_flag;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bar_ld, 1);
+    mbar_init(&bar_m, 1);
+    abort_flag = 0;
+    mbar_fence_init();
+    tma_prefetch_desc(&tmWv);
+  }
+  if (warp == 0) {
+    tmem_alloc(&tmem_base, lay.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = tmem_base;
+  volatile int* abort_p = &abort_flag;
+
+  if (threadIdx.x == 0) {
+    mbar_expect_tx(&bar_ld, (uint32_t)lay.nk * kTileBytes);
+    for (int i = 0; i < lay.nk; ++i) tma_2d(a + i * kTileBytes, &tmWv, k * lay.KS + 64 * i, mb * 128, &bar_ld);
+  }
+
+  // lanes active in this iteration (n_lanes <= 64) and their split counts
+  uint64_t act = 0;
+  for (int b = 0; b < p.n_lanes; ++b) {
+    int nr;
+    if (lane_active(s, p.iter, p.loops, p.ctx_len, b, &nr)) act |= 1ull << b;
+  }
+  // the safety check of one lane per CTA (it depends only on the residual)
+  const int nl = mb * CL + k;
+  if (p.residual && nl < p.n_lanes && ((act >> nl) & 1))
+    norm_check_lane<kProjThreads>(p.residual, nl, s.d, p.threshold, p.iter, p.flags, p.first, p.norms);
+
+  // ---------------------------------------------------------------- merge weights
+  for (int x = threadIdx.x; x < p.n_lanes * lay.hib; x += kProjThreads) {
+    const int b = x / lay.hib, h2 = x % lay.hib, j = mb * lay.hib + h2;
+    if (!((act >> b) & 1)) continue;
+    const int S = splits_for_rows(p.ctx_len[b] + 1);
+    const float* ml = p.ml + (((size_t)b * p.s_max) * kMaxHeads + j) * 2;
+    float M = -CUDART_INF_F;
+    for (int sp = 0; sp < S; ++sp) M = fmaxf(M, ml[(size_t)sp * kMaxHeads * 2]);
+    float L = 0.0f;
+    for (int sp = 0; sp < S; ++sp) L += ml[(size_t)sp * kMaxHeads * 2 + 1] * exp2f(ml[(size_t)sp * kMaxHeads * 2] - M);
+    for (int sp = 0; sp < S; ++sp) wgt[x * p.s_max + sp] = exp2f(ml[(size_t)sp * kMaxHeads * 2] - M) / L;
+  }
+  __syncthreads();
+
+  // ---------------------------------------------------------------- u slice -> B operand
+  // item (operand lane b, head h2, 8 consecutive K positions): the hi and lo rows
+  {
+    const int chunks = lay.KS / 8;
+    for (int x = threadIdx.x; x < nb * lay.hib * chunks; x += kProjThreads) {
+      const int b = x / (lay.hib * chunks), h2 = (x / chunks) % lay.hib, ch = x % chunks;
+      const int j = mb * lay.hib + h2;
+      const int kk = k * lay.KS + 8 * ch;  // position in d
+      float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      if (b < p.n_lanes && ((act >> b) & 1)) {
+        const int S = splits_for_rows(p.ctx_len[b] + 1);
+        const float* w = wgt + (b * lay.hib + h2) * p.s_max;
+        const float* U0 = p.U + ((size_t)b * p.s_max * kMaxHeads + j) * s.d + kk;
+        for (int sp = 0; sp < S; ++sp) {
+          const float4* src = reinterpret_cast<const float4*>(U0 + (size_t)sp * kMaxHeads * s.d);
+          const float4 x0 = __ldcs(src), x1 = __ldcs(src + 1);
+          const float ws = w[sp];
+          v[0] = fmaf(ws, x0.x, v[0]);
+          v[1] = fmaf(ws, x0.y, v[1]);
+          v[2] = fmaf(ws, x0.z, v[2]);
+          v[3] = fmaf(ws, x0.w, v[3]);
+          v[4] = fmaf(ws, x1.x, v[4]);
+          v[5] = fmaf(ws, x1.y, v[5]);
+          v[6] = fmaf(ws, x1.z, v[6]);
+          v[7] = fmaf(ws, x1.w, v[7]);
+        }
+      }
+      __align__(16) __half hi[8], lo[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        hi[i] = __float2half_rn(v[i]);
+        lo[i] = __float2half_rn(v[i] - __half2float(hi[i]));
+      }
+      const int nh = h2 * 2 * nb + b, nlo = h2 * 2 * nb + nb + b;
+      *reinterpret_cast<uint4*>(bop + kmajor_offset(nh, 8 * ch, N)) = *reinterpret_cast<const uint4*>(hi);
+      *reinterpret_cast<uint4*>(bop + kmajor_offset(nlo, 8 * ch, N)) = *reinterpret_cast<const uint4*>(lo);
+    }
+  }
+  fence_proxy_async_smem();
+  __syncthreads();
+
+  // ---------------------------------------------------------------- out partial of K slice k
+  if (warp == 1) {
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_ld, 0, abort_p, kProjWaitLimit));
+    if (ok) {
+      tc_fence_after();
+      if (elect_one()) {
+        const uint32_t id = idesc_f16_f32(128, N, false, false);
+        for (int i = 0; i < lay.nk; ++i) {
+          const uint64_t ad = sdesc_sw128(smem_addr(a + i * kTileBytes), 16, 1024);
+          const uint64_t bd = sdesc_sw128(smem_addr(bop + i * N * 128), 16, 1024);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(tbase, ad + (uint64_t)((kk * 32) >> 4), bd + (uint64_t)((kk * 32) >> 4), id, (i | kk) != 0);
+        }
+        mma_commit(&bar_m);
+      }
+      __syncwarp();
+    }
+  }
+  const int pstride = N + 4;
+  if (mbar_wait(&bar_m, 0, abort_p, kProjWaitLimit)) {
+    tc_fence_after();
+    for (int c0 = 0; c0 < N; c0 += 16) {
+      uint32_t v[16];
+      tmem_ld16(tbase + lane_off + c0, v);
+      tmem_ld_wait();
+      float* dst = part + row * pstride + c0;
+#pragma unroll
+      for (int i = 0; i < 16; i += 4)
+        *reinterpret_cast<float4*>(dst + i) = make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
+                                                          __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
+    }
+  }
+  tc_fence_before();
+  cluster_sync();  // 1: every rank's partial is in place
+
+  // ---------------------------------------------------------------- reduce the K slices, write out
+  // rank k: rows [k * 128/CL, (k+1) * 128/CL) of the block, 4 lanes per item; per rank the hi
+  // and lo columns of a lane are added, then the ranks are summed in rank order
+  {
+    const int rpr = 128 / CL, nq = nb / 4;
+    const uint32_t part_s = smem_addr(part);
+    for (int x = threadIdx.x; x < rpr * nq; x += kProjThreads) {
+      const int r = k * rpr + x / nq, b0 = (x % nq) * 4;
+      if (b0 >= p.n_lanes) continue;
+      const int c0 = (r / s.hd) * 2 * nb;  // the head's columns in the operand
+      float4 vh[8], vl[8];
+#pragma unroll
+      for (int rk = 0; rk < 8; ++rk)
+        if (rk < CL) {
+          vh[rk] = dsmem_ld_f4(dsmem_addr(part_s + (uint32_t)((r * pstride + c0 + b0) * 4), (uint32_t)rk));
+          vl[rk] = dsmem_ld_f4(dsmem_addr(part_s + (uint32_t)((r * pstride + c0 + nb + b0) * 4), (uint32_t)rk));
+        }
+      float o[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int rk = 0; rk < 8; ++rk)
+        if (rk < CL) {
+          o[0] += vh[rk].x + vl[rk].x;
+          o[1] += vh[rk].y + vl[rk].y;
+          o[2] += vh[rk].z + vl[rk].z;
+          o[3] += vh[rk].w + vl[rk].w;
+        }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int b = b0 + i;
+        if (b < p.n_lanes && ((act >> b) & 1)) p.out[(size_t)b * s.d + (size_t)mb * 128 + r] = o[i];
+      }
+    }
+  }
+  cluster_sync();  // 2: no rank leaves while its partial may still be read
+
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && abort_flag) atomicOr(p.status, kStatusTimeout);
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tbase, lay.tmem_cols);
+  }
+}
+
 }  // namespace
 
 // Cluster size of the projection kernels: K splits of d, each a multiple of 64 wide.
@@ -397,6 +633,50 @@ cudaError_t launch_qproj(const DecodeArgs& a, cudaStream_t st) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   e = cudaLaunchKernelEx(&cfg, qproj_kernel, tmWq, tmH, tmWk, p);
+  count_launch();
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_oproj(const DecodeArgs& a, cudaStream_t st) {
+  const Shape& s = a.s;
+  const Workspace& w = a.wl;
+  const int CL = proj_cluster(s.d);
+  const OProjLayout lay(s, w.nb, CL, a.n_lanes, w.s_max);
+  alignas(64) CUtensorMap tmWv;
+  if (!make_tmap_f16(&tmWv, a.Wv, s.d, s.d, s.d, 64, 128)) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(oproj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lay.total);
+  if (e != cudaSuccess) return e;
+  OProjParams p{s,
+                a.iter,
+                a.loops,
+                a.ctx_len,
+                a.n_lanes,
+                w.nb,
+                CL,
+                w.s_max,
+                reinterpret_cast<const float*>(a.ws + w.ml_off),
+                reinterpret_cast<const float*>(a.ws + w.u_off),
+                a.out,
+                reinterpret_cast<uint32_t*>(a.ws + w.status_off),
+                a.residual,
+                a.threshold,
+                a.abort_flags,
+                a.first_abort_iter,
+                a.norms};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(CL, s.d / 128, 1);
+  cfg.blockDim = dim3(kProjThreads, 1, 1);
+  cfg.dynamicSmemBytes = lay.total;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, oproj_kernel, tmWv, p);
   count_launch();
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

@@ -201,7 +201,7 @@ tl_status tl_storeh_attn_decode(const tl_storeh_desc* desc, tl_storeh_cache cach
   e = tl::launch_stream(a, cs);
   tl::profile_stream_end(cs);
   if (e != cudaSuccess) return cuda_fail(e, "decode stream launch");
-  e = tl::launch_epilogue(a, cs);
+  e = tl::launch_oproj(a, cs);
   if (e != cudaSuccess) return cuda_fail(e, "decode epilogue launch");
   return TL_OK;
 }

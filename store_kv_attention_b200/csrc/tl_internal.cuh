@@ -183,6 +183,8 @@ struct DecodeArgs {
 cudaError_t launch_prologue(const DecodeArgs& a, cudaStream_t st);
 // Fused q and absorbed-query projections, one thread-block cluster per 128 rows of W_q (k_proj_tc.cu).
 cudaError_t launch_qproj(const DecodeArgs& a, cudaStream_t st);
+// Fused split merge, value projection and safety check on thread-block clusters (k_proj_tc.cu).
+cudaError_t launch_oproj(const DecodeArgs& a, cudaStream_t st);
 int proj_cluster(int d);
 
 // tensor-core skinny GEMM (k_gemm_tc.cu)
