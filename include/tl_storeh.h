@@ -228,10 +228,10 @@ TL_API tl_status tl_storeh_attn_decode_static_ws(const tl_storeh_desc* desc, tl_
  * TL_ERR_DEVICE_TIMEOUT (a bounded device wait gave up), TL_ERR_DEVICE_RANGE
  * (a lane's loops/ctx_len was out of range and the lane was skipped) or
  * TL_ERR_CUDA.  The status word starts at the beginning of the workspace,
- * whose first 256 bytes also hold arrival counters of the decode kernels
- * (each kernel leaves them at zero); a freshly allocated workspace must have
- * those 256 bytes zero-filled once before its first use.  When the word is
- * not zero this call clears all 256 bytes.
+ * whose first 256 bytes are reserved for it; a freshly allocated workspace
+ * must have those 256 bytes zero-filled once (or be cleared with this call)
+ * before its first use.  When the word is not zero this call clears all 256
+ * bytes.
  */
 TL_API tl_status tl_storeh_poll_status(void* workspace, size_t workspace_bytes, tl_stream_t stream);
 

@@ -214,7 +214,7 @@ tl_status tl_storeh_poll_status(void* workspace, size_t workspace_bytes, tl_stre
   if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
   if (e != cudaSuccess) return cuda_fail(e, "reading the status word");
   if (word != 0) {
-    e = cudaMemsetAsync(workspace, 0, 256, cs);  // the status word and the reduction counters
+    e = cudaMemsetAsync(workspace, 0, 256, cs);  // the status block
     if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
     if (e != cudaSuccess) return cuda_fail(e, "clearing the status word");
   }

@@ -66,20 +66,12 @@ __host__ __device__ inline uint32_t kmajor_offset(int row, int pos, int rows) {
 __host__ __device__ inline int splits_for_rows(int n_rows) { return (n_rows + kSplitRows - 1) / kSplitRows; }
 
 // ---------------------------------------------------------------- decode-step geometry
-constexpr int kMaxGemmLanes = 64;  // lanes per decode call on the tensor-core GEMMs (N <= 256)
+constexpr int kMaxGemmLanes = 64;  // lanes per decode call (projection MMAs with N <= 256, 64-bit lane masks)
 
 __host__ __device__ inline int lanes_padded(int n_lanes) { return (n_lanes + 15) & ~15; }
-// K splits of a skinny GEMM over d so that (d/128) M-blocks x splits ~ 128 CTAs, K per split >= 64
-__host__ __device__ inline int gemm_splits(int d) {
-  int s = 128 / (d / 128);
-  if (s < 1) s = 1;
-  if (s > d / 64) s = d / 64;
-  while ((d / 64) % s) --s;
-  return s;
-}
-// columns of the value-projection GEMM: hi/lo x lanes, for two heads per 128-row block when hd = 64
-__host__ __device__ inline int o_cols(const Shape& s, int nb) { return s.hd == 64 ? 4 * nb : 2 * nb; }
 
+// Whether lane b takes part in iteration `iter` (loops / ctx_len in range and iter < loops[b]);
+// n_rows = the lane's cached positions plus the new one.
 __device__ __forceinline__ bool lane_active(const Shape& s, int iter, const int32_t* loops, const int32_t* ctx_len,
                                             int b, int* n_rows) {
   const int L = loops[b];
@@ -93,17 +85,12 @@ __device__ __forceinline__ bool lane_active(const Shape& s, int iter, const int3
 // ---------------------------------------------------------------- workspace layout
 // All offsets are 256-byte aligned.
 struct Workspace {
-  size_t status_off;   // uint32 status word (+ padding)
-  size_t qpart_off;    // fp32 [Sq][d][NB]         split-K partials of q = W_q h_new
-  size_t qhl_off;      // fp16 [2 NB][d]           q as hi (rows 0..NB-1) + lo (rows NB..2NB-1)
-  size_t qtpart_off;   // fp32 [H][d][2 NB]        W_k[j]^T q_j for q hi and q lo
+  size_t status_off;   // uint32 status word (+ padding to 256 bytes)
   size_t qt_off;       // fp16 [n_lanes][qimg_rows(d) x d] absorbed query operand images (stream kernel)
   size_t ml_off;       // fp32 [n_lanes][S_max][16][2]   per-split running max and sum
   size_t u_off;        // fp32 [n_lanes][S_max][16][d]   per-split unnormalised sum_c p_c h_c
-  size_t uhl_off;      // fp16 [H][2 NB][d]        merged u_j as hi + lo
-  size_t opart_off;    // fp32 [d/128][So][128][o_cols]  split-K partials of W_v[j] u_j
   size_t total;
-  int s_max, nb, sq, so;
+  int s_max, nb;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -112,27 +99,15 @@ inline Workspace workspace_layout(const Shape& s, int n_lanes) {
   Workspace w;
   w.s_max = splits_for_rows(s.max_ctx);
   w.nb = lanes_padded(n_lanes);
-  w.sq = gemm_splits(s.d);
-  w.so = gemm_splits(s.d);
   size_t off = 0;
   w.status_off = off;
   off += 256;
-  w.qpart_off = off;
-  off = align256(off + (size_t)w.sq * s.d * w.nb * 4);
-  w.qhl_off = off;
-  off = align256(off + (size_t)2 * w.nb * s.d * 2);
-  w.qtpart_off = off;
-  off = align256(off + (size_t)s.H * s.d * 2 * w.nb * 4);
   w.qt_off = off;
   off = align256(off + (size_t)n_lanes * qimg_bytes(s.d));
   w.ml_off = off;
   off = align256(off + (size_t)n_lanes * w.s_max * kMaxHeads * 2 * 4);
   w.u_off = off;
   off = align256(off + (size_t)n_lanes * w.s_max * kMaxHeads * (size_t)s.d * 4);
-  w.uhl_off = off;
-  off = align256(off + (size_t)s.H * 2 * w.nb * s.d * 2);
-  w.opart_off = off;
-  off = align256(off + (size_t)(s.d / 128) * w.so * 128 * o_cols(s, w.nb) * 4);
   w.total = off;
   return w;
 }
@@ -180,45 +155,16 @@ struct DecodeArgs {
   float* norms;
 };
 
-cudaError_t launch_prologue(const DecodeArgs& a, cudaStream_t st);
 // Fused q and absorbed-query projections, one thread-block cluster per 128 rows of W_q (k_proj_tc.cu).
 cudaError_t launch_qproj(const DecodeArgs& a, cudaStream_t st);
 // Fused split merge, value projection and safety check on thread-block clusters (k_proj_tc.cu).
 cudaError_t launch_oproj(const DecodeArgs& a, cudaStream_t st);
 int proj_cluster(int d);
 
-// tensor-core skinny GEMM (k_gemm_tc.cu)
+// fp16 2D tensor map [rows][cols] (row pitch `pitch_elems`), box [box_cols x box_rows], 128-byte swizzle
+// (k_proj_tc.cu).
 bool make_tmap_f16(void* tmap, const void* base, uint64_t rows, uint64_t cols, uint64_t pitch_elems,
                    uint32_t box_cols, uint32_t box_rows);
-// Epilogues of the decode GEMMs (k_gemm_tc.cu).  The split-K modes write their fp32
-// partials, and the last CTA of each 128-row block (an arrival counter, reset by that CTA)
-// sums them in split order and writes the final values, so the result does not depend on
-// scheduling.
-enum GemmEpi : int {
-  kEpiPartials = 0,  // fp32 partials only
-  kEpiQ = 1,         // q = W_q h_new: reduce the splits, write fp16 hi/lo rows of q (the next GEMM's B)
-  kEpiQImage = 2,    // qt_j = W_k[j]^T q_j: write the streaming kernel's absorbed-query operand image
-  kEpiOut = 3,       // out_j = W_v[j] u_j: reduce the splits, write out
-};
-struct GemmEpiParams {
-  int mode;
-  Shape s;
-  int iter;
-  const int32_t* loops;
-  const int32_t* ctx_len;
-  int n_lanes, nb;
-  uint32_t* counters;  // split-K modes: one per (batch entry, 128-row block), zero between calls
-  uint32_t* status;    // device status word (kEpiQ records out-of-range lanes)
-  __half* qhl;         // kEpiQ: [2 nb][d], hi rows then lo rows
-  uint8_t* qimg;       // kEpiQImage: [n_lanes][qimg_bytes(d)]
-  float* out;          // kEpiOut: [n_lanes][d]
-};
-// Offsets of the arrival counters inside the 256-byte status block of the workspace.
-constexpr size_t kCountersQOff = 64, kCountersOOff = 128;
-cudaError_t launch_gemm_tc(bool a_mn, const void* tmA, const void* tmB, int M, int N, int K, int splits, int batch,
-                           int a_x_per_z, int a_y_per_z, int b_x_per_z, int b_y_per_z, float* out, uint32_t* status,
-                           const GemmEpiParams& epi, cudaStream_t st);
 cudaError_t launch_stream(const DecodeArgs& a, cudaStream_t st);
-cudaError_t launch_epilogue(const DecodeArgs& a, cudaStream_t st);
 
 }  // namespace tl
