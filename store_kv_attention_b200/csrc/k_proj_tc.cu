@@ -32,7 +32,8 @@ namespace {
 
 using namespace ptx;
 
-constexpr int kProjThreads = 128;                // four warps: TMEM lane quarters 0-3
+constexpr int kProjThreads = 128;                // qproj: four warps, TMEM lane quarters 0-3
+constexpr int kOProjThreads = 256;               // oproj: eight warps (two per lane quarter)
 constexpr int kTileBytes = 128 * 64 * 2;         // one 128 x 64 fp16 operand tile
 constexpr long long kProjWaitLimit = 4000000000ll;
 
@@ -55,6 +56,22 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 // The absorbed-query operand image of a lane: row j = fp16(qt_j) and, when the operands
 // are split, row 16 + j = fp16(qt_j - fp16(qt_j)); columns in the dequantised position
 // order, 128-byte swizzled atom-columns of 64 positions (kmajor_offset).
+
+// Lanes active in this iteration as a 64-bit mask (n_lanes <= 64), computed by warp 0 in
+// parallel and broadcast through shared memory; every thread of the block must call it.
+__device__ __forceinline__ uint64_t active_mask(const Shape& s, int iter, const int32_t* loops, const int32_t* ctx_len,
+                                               int n_lanes, uint64_t* slot) {
+  if (threadIdx.x < 32) {
+    int nr;
+    const int b0 = threadIdx.x, b1 = threadIdx.x + 32;
+    const bool a0 = b0 < n_lanes && lane_active(s, iter, loops, ctx_len, b0, &nr);
+    const bool a1 = b1 < n_lanes && lane_active(s, iter, loops, ctx_len, b1, &nr);
+    const uint32_t lo = __ballot_sync(0xffffffffu, a0), hi = __ballot_sync(0xffffffffu, a1);
+    if (threadIdx.x == 0) *slot = (uint64_t)lo | ((uint64_t)hi << 32);
+  }
+  __syncthreads();
+  return *slot;
+}
 
 struct QProjParams {
   Shape s;
@@ -212,12 +229,8 @@ __global__ void __launch_bounds__(kProjThreads, 1)
       if (L < 0 || L > s.L_max || c < 0 || c >= s.max_ctx) atomicOr(p.status, kStatusRange);
     }
   }
-  // lanes active in this iteration (n_lanes <= 64)
-  uint64_t act = 0;
-  for (int b = 0; b < p.n_lanes; ++b) {
-    int nr;
-    if (lane_active(s, p.iter, p.loops, p.ctx_len, b, &nr)) act |= 1ull << b;
-  }
+  __shared__ uint64_t act_slot;
+  const uint64_t act = active_mask(s, p.iter, p.loops, p.ctx_len, p.n_lanes, &act_slot);
   const int rpr = 128 / CL;
   {
     const int nq = nb / 4;
@@ -414,7 +427,7 @@ struct OProjLayout {
   }
 };
 
-__global__ void __launch_bounds__(kProjThreads, 1)
+__global__ void __launch_bounds__(kOProjThreads, 1)
     oproj_kernel(const __grid_constant__ CUtensorMap tmWv, const OProjParams p) {
   const Shape& s = p.s;
   const int nb = p.nb, CL = p.cl;
@@ -458,67 +471,113 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     for (int i = 0; i < lay.nk; ++i) tma_2d(a + i * kTileBytes, &tmWv, k * lay.KS + 64 * i, mb * 128, &bar_ld);
   }
 
-  // lanes active in this iteration (n_lanes <= 64) and their split counts
-  uint64_t act = 0;
-  for (int b = 0; b < p.n_lanes; ++b) {
-    int nr;
-    if (lane_active(s, p.iter, p.loops, p.ctx_len, b, &nr)) act |= 1ull << b;
-  }
+  __shared__ uint64_t act_slot;
+  const uint64_t act = active_mask(s, p.iter, p.loops, p.ctx_len, p.n_lanes, &act_slot);
   // the safety check of one lane per CTA (it depends only on the residual)
   const int nl = mb * CL + k;
   if (p.residual && nl < p.n_lanes && ((act >> nl) & 1))
-    norm_check_lane<kProjThreads>(p.residual, nl, s.d, p.threshold, p.iter, p.flags, p.first, p.norms);
+    norm_check_lane<kOProjThreads>(p.residual, nl, s.d, p.threshold, p.iter, p.flags, p.first, p.norms);
 
   // ---------------------------------------------------------------- merge weights
-  for (int x = threadIdx.x; x < p.n_lanes * lay.hib; x += kProjThreads) {
+  for (int x = threadIdx.x; x < p.n_lanes * lay.hib; x += kOProjThreads) {
     const int b = x / lay.hib, h2 = x % lay.hib, j = mb * lay.hib + h2;
     if (!((act >> b) & 1)) continue;
     const int S = splits_for_rows(p.ctx_len[b] + 1);
-    const float* ml = p.ml + (((size_t)b * p.s_max) * kMaxHeads + j) * 2;
+    const float2* ml = reinterpret_cast<const float2*>(p.ml + (((size_t)b * p.s_max) * kMaxHeads + j) * 2);
+    float* wl = wgt + x * p.s_max;
+    // (m, l) of the splits, staged in this thread's weight slots before the reductions
+    for (int sp = 0; sp < S; ++sp) wl[sp] = 0.0f;
     float M = -CUDART_INF_F;
-    for (int sp = 0; sp < S; ++sp) M = fmaxf(M, ml[(size_t)sp * kMaxHeads * 2]);
+    for (int sp0 = 0; sp0 < S; sp0 += 8) {
+      float2 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (sp0 + u < S) v[u] = ml[(size_t)(sp0 + u) * kMaxHeads];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (sp0 + u < S) {
+          M = fmaxf(M, v[u].x);
+          wl[sp0 + u] = v[u].x;  // m_s for now
+        }
+    }
     float L = 0.0f;
-    for (int sp = 0; sp < S; ++sp) L += ml[(size_t)sp * kMaxHeads * 2 + 1] * exp2f(ml[(size_t)sp * kMaxHeads * 2] - M);
-    for (int sp = 0; sp < S; ++sp) wgt[x * p.s_max + sp] = exp2f(ml[(size_t)sp * kMaxHeads * 2] - M) / L;
+    for (int sp = 0; sp < S; ++sp) L += ml[(size_t)sp * kMaxHeads].y * exp2f(wl[sp] - M);
+    for (int sp = 0; sp < S; ++sp) wl[sp] = exp2f(wl[sp] - M) / L;
   }
   __syncthreads();
 
   // ---------------------------------------------------------------- u slice -> B operand
-  // item (operand lane b, head h2, 8 consecutive K positions): the hi and lo rows
+  // item (operand lane b, head h2, 8 consecutive K positions): the hi and lo rows.  Two items
+  // per thread at a time, the loads of four splits issued before their multiply-adds, which
+  // run in split order.
   {
     const int chunks = lay.KS / 8;
-    for (int x = threadIdx.x; x < nb * lay.hib * chunks; x += kProjThreads) {
-      const int b = x / (lay.hib * chunks), h2 = (x / chunks) % lay.hib, ch = x % chunks;
-      const int j = mb * lay.hib + h2;
-      const int kk = k * lay.KS + 8 * ch;  // position in d
-      float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      if (b < p.n_lanes && ((act >> b) & 1)) {
-        const int S = splits_for_rows(p.ctx_len[b] + 1);
-        const float* w = wgt + (b * lay.hib + h2) * p.s_max;
-        const float* U0 = p.U + ((size_t)b * p.s_max * kMaxHeads + j) * s.d + kk;
-        for (int sp = 0; sp < S; ++sp) {
-          const float4* src = reinterpret_cast<const float4*>(U0 + (size_t)sp * kMaxHeads * s.d);
-          const float4 x0 = __ldcs(src), x1 = __ldcs(src + 1);
-          const float ws = w[sp];
-          v[0] = fmaf(ws, x0.x, v[0]);
-          v[1] = fmaf(ws, x0.y, v[1]);
-          v[2] = fmaf(ws, x0.z, v[2]);
-          v[3] = fmaf(ws, x0.w, v[3]);
-          v[4] = fmaf(ws, x1.x, v[4]);
-          v[5] = fmaf(ws, x1.y, v[5]);
-          v[6] = fmaf(ws, x1.z, v[6]);
-          v[7] = fmaf(ws, x1.w, v[7]);
+    const int n_items = nb * lay.hib * chunks;
+    for (int x0 = threadIdx.x; x0 < n_items; x0 += 2 * kOProjThreads) {
+      float v[2][8];
+      int S2[2];
+      const float* U0[2];
+      const float* w2[2];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int x = x0 + q * kOProjThreads;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[q][i] = 0.0f;
+        S2[q] = 0;
+        U0[q] = nullptr;
+        w2[q] = nullptr;
+        if (x < n_items) {
+          const int b = x / (lay.hib * chunks), h2 = (x / chunks) % lay.hib, ch = x % chunks;
+          if (b < p.n_lanes && ((act >> b) & 1)) {
+            S2[q] = splits_for_rows(p.ctx_len[b] + 1);
+            U0[q] = p.U + ((size_t)b * p.s_max * kMaxHeads + mb * lay.hib + h2) * s.d + k * lay.KS + 8 * ch;
+            w2[q] = wgt + (b * lay.hib + h2) * p.s_max;
+          }
         }
       }
-      __align__(16) __half hi[8], lo[8];
+      const int Smax = S2[0] > S2[1] ? S2[0] : S2[1];
+      for (int sp0 = 0; sp0 < Smax; sp0 += 4) {
+        float4 xs[2][8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        hi[i] = __float2half_rn(v[i]);
-        lo[i] = __float2half_rn(v[i] - __half2float(hi[i]));
+        for (int q = 0; q < 2; ++q)
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (sp0 + u < S2[q]) {
+              const float4* src = reinterpret_cast<const float4*>(U0[q] + (size_t)(sp0 + u) * kMaxHeads * s.d);
+              xs[q][2 * u] = __ldcs(src);
+              xs[q][2 * u + 1] = __ldcs(src + 1);
+            }
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (sp0 + u < S2[q]) {
+              const float ws = w2[q][sp0 + u];
+              v[q][0] = fmaf(ws, xs[q][2 * u].x, v[q][0]);
+              v[q][1] = fmaf(ws, xs[q][2 * u].y, v[q][1]);
+              v[q][2] = fmaf(ws, xs[q][2 * u].z, v[q][2]);
+              v[q][3] = fmaf(ws, xs[q][2 * u].w, v[q][3]);
+              v[q][4] = fmaf(ws, xs[q][2 * u + 1].x, v[q][4]);
+              v[q][5] = fmaf(ws, xs[q][2 * u + 1].y, v[q][5]);
+              v[q][6] = fmaf(ws, xs[q][2 * u + 1].z, v[q][6]);
+              v[q][7] = fmaf(ws, xs[q][2 * u + 1].w, v[q][7]);
+            }
       }
-      const int nh = h2 * 2 * nb + b, nlo = h2 * 2 * nb + nb + b;
-      *reinterpret_cast<uint4*>(bop + kmajor_offset(nh, 8 * ch, N)) = *reinterpret_cast<const uint4*>(hi);
-      *reinterpret_cast<uint4*>(bop + kmajor_offset(nlo, 8 * ch, N)) = *reinterpret_cast<const uint4*>(lo);
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int x = x0 + q * kOProjThreads;
+        if (x >= n_items) continue;
+        const int b = x / (lay.hib * chunks), h2 = (x / chunks) % lay.hib, ch = x % chunks;
+        __align__(16) __half hi[8], lo[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          hi[i] = __float2half_rn(v[q][i]);
+          lo[i] = __float2half_rn(v[q][i] - __half2float(hi[i]));
+        }
+        const int nh = h2 * 2 * nb + b, nlo = h2 * 2 * nb + nb + b;
+        *reinterpret_cast<uint4*>(bop + kmajor_offset(nh, 8 * ch, N)) = *reinterpret_cast<const uint4*>(hi);
+        *reinterpret_cast<uint4*>(bop + kmajor_offset(nlo, 8 * ch, N)) = *reinterpret_cast<const uint4*>(lo);
+      }
     }
   }
   fence_proxy_async_smem();
@@ -546,7 +605,8 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   const int pstride = N + 4;
   if (mbar_wait(&bar_m, 0, abort_p, kProjWaitLimit)) {
     tc_fence_after();
-    for (int c0 = 0; c0 < N; c0 += 16) {
+    // warps w and w + 4 share lane quarter w % 4 and take alternate 16-column groups
+    for (int c0 = (warp >> 2) * 16; c0 < N; c0 += 32) {
       uint32_t v[16];
       tmem_ld16(tbase + lane_off + c0, v);
       tmem_ld_wait();
@@ -566,7 +626,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   {
     const int rpr = 128 / CL, nq = nb / 4;
     const uint32_t part_s = smem_addr(part);
-    for (int x = threadIdx.x; x < rpr * nq; x += kProjThreads) {
+    for (int x = threadIdx.x; x < rpr * nq; x += kOProjThreads) {
       const int r = k * rpr + x / nq, b0 = (x % nq) * 4;
       if (b0 >= p.n_lanes) continue;
       const int c0 = (r / s.hd) * 2 * nb;  // the head's columns in the operand
@@ -695,7 +755,7 @@ cudaError_t launch_oproj(const DecodeArgs& a, cudaStream_t st) {
                 a.norms};
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(CL, s.d / 128, 1);
-  cfg.blockDim = dim3(kProjThreads, 1, 1);
+  cfg.blockDim = dim3(kOProjThreads, 1, 1);
   cfg.dynamicSmemBytes = lay.total;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
