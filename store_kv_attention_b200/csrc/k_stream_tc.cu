@@ -73,6 +73,7 @@ constexpr int kThreads = 32 * (kWarpVP + 1);
 constexpr int kSlotBytes = 128 * 128;           // one ring slot: 128 rows x 128 bytes of codes
 constexpr int kPvStageBytes = 128 * 256;        // P.V operand staging: 128 rows x 128 fp16 values
 constexpr int kMaxRing = 4;                     // slots per ring at most
+constexpr int kL2AheadTiles = 2;                // L2 prefetch distance of the codes stream, in tiles
 constexpr long long kWaitLimit = 4000000000ll;  // ~2 s of SM clocks, far beyond any legitimate wait
 
 template <int FMT>
@@ -91,6 +92,38 @@ struct Fmt {
   __device__ static bool score_releases(int hh) { return FMT == TL_H_FP16 || hh == 1; }
   // A P.V warp reads one half of every unit: INT4 chunks hold two units.
   __device__ static bool pv_releases(int u) { return FMT != TL_H_INT4_G64 || (u & 1); }
+
+  // Ring slots.  A consumer waits on a slot's full barrier by phase parity, which is only
+  // sound if it sees every use of that slot in order.  So each ring is split into one
+  // sub-ring per set of consumers that read the same chunks: score side, INT4 chunks are
+  // read by both halves (one owner), INT8 chunk g by half g & 1, FP16 chunk g by half
+  // (g >> 1) & 1; P.V side, FP16 chunk g by the warps of part g & 1, otherwise by all.
+  // Chunk g is the k-th chunk of its owner o and lives in slot o * R + k % R, use k / R,
+  // with R the sub-ring size.
+  static constexpr int kOwnersS = FMT == TL_H_INT4_G64 ? 1 : 2;
+  static constexpr int kOwnersV = FMT == TL_H_FP16 ? 2 : 1;
+  __host__ __device__ static void s_slot(int g, int ring, int& slot, int& use) {
+    const int R = ring / kOwnersS;
+    int o, k;
+    if (FMT == TL_H_INT4_G64) {
+      o = 0;
+      k = g;
+    } else if (FMT == TL_H_INT8_TOKEN) {
+      o = g & 1;
+      k = g >> 1;
+    } else {
+      o = (g >> 1) & 1;
+      k = ((g >> 2) << 1) | (g & 1);
+    }
+    slot = o * R + k % R;
+    use = k / R;
+  }
+  __host__ __device__ static void v_slot(int g, int ring, int& slot, int& use) {
+    const int R = ring / kOwnersV;
+    const int o = kOwnersV == 2 ? (g & 1) : 0, k = kOwnersV == 2 ? (g >> 1) : g;
+    slot = o * R + k % R;
+    use = k / R;
+  }
 };
 
 struct StreamParams {
@@ -309,10 +342,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         bulk_load(qs + off, qsrc + off, min(16384u, qbytes - off), &bars.q_full);
       // the score pass keeps a tile in L2 for the P.V pass, which is its last use
       const uint64_t pol_keep = l2_policy_evict_normal();
+      // L2 prefetch kL2Ahead chunks ahead of the ring (no shared memory): more of the codes
+      // stream is in flight than the ring slots alone allow
+      const int ahead = kL2AheadTiles * n_chunks;
+      auto prefetch = [&](int c) {
+        if (c < total_chunks) tma_prefetch_l2_2d(&tmap, (c % n_chunks) * 128, row_base + r_begin + (c / n_chunks) * 128);
+      };
+      for (int c = 0; c < ahead; ++c) prefetch(c);
       int g = 0;
       for (; g < total_chunks; ++g) {
-        const int slot = g % SR, use = g / SR;
+        int slot, use;
+        F::s_slot(g, SR, slot, use);
         if (use > 0 && !mbar_wait(&bars.s_empty[slot], (use - 1) & 1, abort_p, kWaitLimit)) break;
+        prefetch(g + ahead);
         mbar_expect_tx(&bars.s_full[slot], kSlotBytes);
         tma_load_2d(sring + slot * kSlotBytes, &tmap, (g % n_chunks) * 128, row_base + r_begin + (g / n_chunks) * 128,
                     &bars.s_full[slot], pol_keep);
@@ -320,7 +362,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // every copy issued lands before the CTA's shared memory goes away
       drain_wait(&bars.q_full, 0);
-      for (int i = g > SR ? g - SR : 0; i < g; ++i) drain_wait(&bars.s_full[i % SR], (i / SR) & 1);
+      for (int i = g > SR ? g - SR : 0; i < g; ++i) {
+        int slot, use;
+        F::s_slot(i, SR, slot, use);
+        drain_wait(&bars.s_full[slot], use & 1);
+      }
     }
   } else if (warp == kWarpVP) {
     // ------------------------------------------------------------ TMA producer, P.V-side ring
@@ -330,7 +376,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t pol_last_use = l2_policy_evict_first();
       int g = 0;
       for (; g < total_chunks; ++g) {
-        const int slot = g % VR, use = g / VR;
+        int slot, use;
+        F::v_slot(g, VR, slot, use);
         if (use > 0 && !mbar_wait(&bars.v_empty[slot], (use - 1) & 1, abort_p, kWaitLimit)) break;
         if (*s_issued_p <= g) {
           const long long t0 = clock64();
@@ -344,7 +391,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_2d(vring + slot * kSlotBytes, &tmap, (g % n_chunks) * 128, row_base + r_begin + (g / n_chunks) * 128,
                     &bars.v_full[slot], pol_last_use);
       }
-      for (int i = g > VR ? g - VR : 0; i < g; ++i) drain_wait(&bars.v_full[i % VR], (i / VR) & 1);
+      for (int i = g > VR ? g - VR : 0; i < g; ++i) {
+        int slot, use;
+        F::v_slot(i, VR, slot, use);
+        drain_wait(&bars.v_full[slot], use & 1);
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ score-MMA issuer
@@ -477,8 +528,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           const int g = t * n_chunks + F::chunk(u, hh);
-          const int slot = g % SR;
-          if (!mbar_wait(&bars.s_full[slot], (g / SR) & 1, abort_p, kWaitLimit)) { ok = false; break; }
+          int slot, use;
+          F::s_slot(g, SR, slot, use);
+          if (!mbar_wait(&bars.s_full[slot], use & 1, abort_p, kWaitLimit)) { ok = false; break; }
           uint32_t h[32];
           dequant_half<FMT>(sring + slot * kSlotBytes + r * 128, xr, u, hh, hh ? (sw >> 16) : (sw & 0xFFFFu), h);
           if (F::score_releases(hh)) {
@@ -644,8 +696,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int u = 0; u < n_units; ++u) {
         const uint32_t sw = (FMT == TL_H_INT4_G64 && valid) ? __ldg(srow + u) : 0u;
         const int g = t * n_chunks + F::chunk(u, part);
-        const int slot = g % VR;
-        if (!mbar_wait(&bars.v_full[slot], (g / VR) & 1, abort_p, kWaitLimit)) { ok = false; break; }
+        int slot, use;
+        F::v_slot(g, VR, slot, use);
+        if (!mbar_wait(&bars.v_full[slot], use & 1, abort_p, kWaitLimit)) { ok = false; break; }
         uint32_t h[32];
         dequant_half<FMT>(vring + slot * kSlotBytes + r * 128, xr, u, part, part ? (sw >> 16) : (sw & 0xFFFFu), h);
         if (F::pv_releases(u)) {
@@ -708,9 +761,11 @@ cudaError_t launch_fmt(const DecodeArgs& a, const CUtensorMap& tmap, cudaStream_
   const size_t fixed = 1024 + qimg_bytes(s.d) + 2 * (size_t)kPvStageBytes + 2 * (size_t)NP * 256;
   const long long room = (long long)optin - (long long)fa.sharedSizeBytes - (long long)fixed;
   const int slots = room > 0 ? (int)(room / kSlotBytes) : 0;
-  if (slots < 4) return cudaErrorInvalidConfiguration;
-  const int s_ring = std::min(kMaxRing, (slots + 1) / 2);
-  const int v_ring = std::min(kMaxRing, slots - s_ring);
+  using F = Fmt<FMT>;
+  // ring sizes: about half the slots each, multiples of the sub-ring counts
+  const int s_ring = std::min(kMaxRing, std::max(F::kOwnersS, (slots + 1) / 2 / F::kOwnersS * F::kOwnersS));
+  const int v_ring = std::min(kMaxRing, (slots - s_ring) / F::kOwnersV * F::kOwnersV);
+  if (v_ring < F::kOwnersV || v_ring < 2 || s_ring < 2) return cudaErrorInvalidConfiguration;
   const size_t smem = fixed + (size_t)(s_ring + v_ring) * kSlotBytes;
   if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
   StreamParams p{s,
