@@ -73,7 +73,6 @@ constexpr int kThreads = 32 * (kWarpVP + 1);
 constexpr int kSlotBytes = 128 * 128;           // one ring slot: 128 rows x 128 bytes of codes
 constexpr int kPvStageBytes = 128 * 256;        // P.V operand staging: 128 rows x 128 fp16 values
 constexpr int kMaxRing = 4;                     // slots per ring at most
-constexpr int kL2AheadTiles = 2;                // L2 prefetch distance of the codes stream, in tiles
 constexpr long long kWaitLimit = 4000000000ll;  // ~2 s of SM clocks, far beyond any legitimate wait
 
 template <int FMT>
@@ -342,19 +341,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         bulk_load(qs + off, qsrc + off, min(16384u, qbytes - off), &bars.q_full);
       // the score pass keeps a tile in L2 for the P.V pass, which is its last use
       const uint64_t pol_keep = l2_policy_evict_normal();
-      // L2 prefetch kL2Ahead chunks ahead of the ring (no shared memory): more of the codes
-      // stream is in flight than the ring slots alone allow
-      const int ahead = kL2AheadTiles * n_chunks;
-      auto prefetch = [&](int c) {
-        if (c < total_chunks) tma_prefetch_l2_2d(&tmap, (c % n_chunks) * 128, row_base + r_begin + (c / n_chunks) * 128);
-      };
-      for (int c = 0; c < ahead; ++c) prefetch(c);
       int g = 0;
       for (; g < total_chunks; ++g) {
         int slot, use;
         F::s_slot(g, SR, slot, use);
         if (use > 0 && !mbar_wait(&bars.s_empty[slot], (use - 1) & 1, abort_p, kWaitLimit)) break;
-        prefetch(g + ahead);
         mbar_expect_tx(&bars.s_full[slot], kSlotBytes);
         tma_load_2d(sring + slot * kSlotBytes, &tmap, (g % n_chunks) * 128, row_base + r_begin + (g / n_chunks) * 128,
                     &bars.s_full[slot], pol_keep);
