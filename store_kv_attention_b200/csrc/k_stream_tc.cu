@@ -23,7 +23,7 @@
 // double-buffered across tiles; the scores S are double-buffered in TMEM.
 // Score group: two warps per TMEM lane quarter, one for the even and one for the
 // odd 128-value units of each row, and for heads 0-7 / 8-15 in the softmax.
-// P.V group: two warps per 32-row block, one per 64-value half of every unit.
+// P.V group: two warps per 32-row block, one for the even and one for the odd units.
 // Each group reads the codes of a tile through its own TMA ring; the second
 // read of a tile (P.V) finds it in L2.  The online softmax runs in base 2 and
 // each split writes its partial (m, l, U) at the end.
@@ -89,18 +89,16 @@ struct Fmt {
   // A score warp reads both halves of its own units: its last read of a chunk is half 1
   // (FP16: every half is a chunk of its own).
   __device__ static bool score_releases(int hh) { return FMT == TL_H_FP16 || hh == 1; }
-  // A P.V warp reads one half of every unit: INT4 chunks hold two units.
-  __device__ static bool pv_releases(int u) { return FMT != TL_H_INT4_G64 || (u & 1); }
 
   // Ring slots.  A consumer waits on a slot's full barrier by phase parity, which is only
   // sound if it sees every use of that slot in order.  So each ring is split into one
-  // sub-ring per set of consumers that read the same chunks: score side, INT4 chunks are
-  // read by both halves (one owner), INT8 chunk g by half g & 1, FP16 chunk g by half
-  // (g >> 1) & 1; P.V side, FP16 chunk g by the warps of part g & 1, otherwise by all.
+  // sub-ring per set of consumers that read the same chunks: INT4 chunks are read by both
+  // score halves (and both P.V sets), INT8 chunk g by half / set g & 1, FP16 chunk g by
+  // half / set (g >> 1) & 1.
   // Chunk g is the k-th chunk of its owner o and lives in slot o * R + k % R, use k / R,
   // with R the sub-ring size.
   static constexpr int kOwnersS = FMT == TL_H_INT4_G64 ? 1 : 2;
-  static constexpr int kOwnersV = FMT == TL_H_FP16 ? 2 : 1;
+  static constexpr int kOwnersV = kOwnersS;  // the P.V sets read units like the score halves
   __host__ __device__ static void s_slot(int g, int ring, int& slot, int& use) {
     const int R = ring / kOwnersS;
     int o, k;
@@ -117,12 +115,7 @@ struct Fmt {
     slot = o * R + k % R;
     use = k / R;
   }
-  __host__ __device__ static void v_slot(int g, int ring, int& slot, int& use) {
-    const int R = ring / kOwnersV;
-    const int o = kOwnersV == 2 ? (g & 1) : 0, k = kOwnersV == 2 ? (g >> 1) : g;
-    slot = o * R + k % R;
-    use = k / R;
-  }
+  __host__ __device__ static void v_slot(int g, int ring, int& slot, int& use) { s_slot(g, ring, slot, use); }
 };
 
 struct StreamParams {
@@ -251,7 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int NS = SPLIT ? 32 : 16;  // score columns (heads, or hi/lo x heads)
   constexpr int NP = SPLIT ? 32 : 16;  // P.V columns
   constexpr int kSReaders = FMT == TL_H_INT4_G64 ? kSWarps : kSWarps / 2;  // score warps reading a slot
-  constexpr int kVReaders = FMT == TL_H_FP16 ? kVWarps / 2 : kVWarps;      // P.V warps reading a slot
+  constexpr int kVReaders = FMT == TL_H_INT4_G64 ? kVWarps : kVWarps / 2;  // P.V warps reading a slot
   constexpr uint32_t kIdS = idesc_f16_f32(128, NS, false, false);
   constexpr uint32_t kIdP = idesc_f16_f32(128, NP, true, false);
   constexpr uint32_t kColS = 0, kColStg = 64, kColU = 256;  // TMEM columns: S[2] x 32, staging[2] x 64, U^T
@@ -302,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.stg_full[i], 4);
       mbar_init(&bars.stg_empty[i], 1);
-      mbar_init(&bars.pv_full[i], kVWarps);
+      mbar_init(&bars.pv_full[i], kVWarps / 2);
       mbar_init(&bars.pv_empty[i], 1);
       mbar_init(&bars.sc_full[i], 1);
       mbar_init(&bars.sc_empty[i], kSWarps);
@@ -443,8 +436,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint64_t pd = p_desc0 + (uint64_t)((pb * NP * 256) >> 4);
       for (int u = 0; u < n_units; ++u) {
-        const int gp = t * n_units + u, x = u & 1;
-        if (!warp_wait(&bars.pv_full[x], (gp >> 1) & 1, abort_p)) { ok = false; break; }
+        const int x = u & 1, k_use = t * (n_units >> 1) + (u >> 1);
+        if (!warp_wait(&bars.pv_full[x], k_use & 1, abort_p)) { ok = false; break; }
         tc_fence_after();
         const uint64_t ad = pv_desc0 + (uint64_t)((x * kPvStageBytes) >> 4);
         const uint32_t du = tbase + kColU + u * NP;
@@ -672,11 +665,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_st_wait();  // no store of this warp may be in flight when TMEM is freed
   } else {
     // ------------------------------------------------------------ P.V group
-    // warp -> (row block, part): part 0 dequantises values 0-63 of every unit, part 1 64-127,
-    // into the swizzled shared-memory staging the P.V MMA reads MN-major (d as M, rows as K)
+    // warp -> (row block, set): set 0 dequantises the even units, set 1 the odd units, each
+    // whole unit into its own shared-memory staging buffer that the P.V MMA reads MN-major
+    // (d as M, rows as K); a unit's MMAs wait for the four warps of its set only.
     const int vw = warp - kWarpV0;
     const int r = (vw & 3) * 32 + lane;
-    const int part = vw >> 2;
+    const int set = vw >> 2;
     const int xr = r & 7;
     bool ok = true;
     auto row_of = [&](int t) { return (size_t)row_base + r_begin + t * 128 + r; };
@@ -684,31 +678,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = 0; t < n_tiles && ok; ++t) {
       const bool valid = row_valid(t);
       const uint32_t* srow = reinterpret_cast<const uint32_t*>(p.scales + row_of(t) * (size_t)scale_words * 4);
-      for (int u = 0; u < n_units; ++u) {
-        const uint32_t sw = (FMT == TL_H_INT4_G64 && valid) ? __ldg(srow + u) : 0u;
-        const int g = t * n_chunks + F::chunk(u, part);
-        int slot, use;
-        F::v_slot(g, VR, slot, use);
-        if (!mbar_wait(&bars.v_full[slot], use & 1, abort_p, kWaitLimit)) { ok = false; break; }
-        uint32_t h[32];
-        dequant_half<FMT>(vring + slot * kSlotBytes + r * 128, xr, u, part, part ? (sw >> 16) : (sw & 0xFFFFu), h);
-        if (F::pv_releases(u)) {
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bars.v_empty[slot]);
-        }
-        if (!valid) {
+      for (int u = set; u < n_units && ok; u += 2) {
+        const uint32_t sw = (FMT == TL_H_INT4_G64 && valid) ? __ldg(srow + u) : 0u;  // groups 2u | 2u+1
+        const int k_use = t * (n_units >> 1) + (u >> 1);  // this set's units so far
+        uint8_t* st = pvs + set * kPvStageBytes + r * 128;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) h[i] = 0u;
-        }
-        const int gp = t * n_units + u, x = u & 1;
-        if (gp >= 2 && !mbar_wait(&bars.pv_empty[x], ((gp >> 1) - 1) & 1, abort_p, kWaitLimit)) { ok = false; break; }
-        uint8_t* st = pvs + x * kPvStageBytes + part * 16384 + r * 128;
+        for (int hh = 0; hh < 2; ++hh) {
+          const int g = t * n_chunks + F::chunk(u, hh);
+          int slot, use;
+          F::v_slot(g, VR, slot, use);
+          if (!mbar_wait(&bars.v_full[slot], use & 1, abort_p, kWaitLimit)) { ok = false; break; }
+          uint32_t h[32];
+          dequant_half<FMT>(vring + slot * kSlotBytes + r * 128, xr, u, hh, hh ? (sw >> 16) : (sw & 0xFFFFu), h);
+          if (F::score_releases(hh)) {  // same reading pattern as a score half
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars.v_empty[slot]);
+          }
+          if (!valid) {
 #pragma unroll
-        for (int v = 0; v < 8; ++v)
-          *reinterpret_cast<uint4*>(st + ((v ^ xr) << 4)) = make_uint4(h[4 * v], h[4 * v + 1], h[4 * v + 2], h[4 * v + 3]);
+            for (int i = 0; i < 32; ++i) h[i] = 0u;
+          }
+          // the staging buffer is free once the MMAs of this set's previous unit are done
+          if (hh == 0 && k_use >= 1 && !mbar_wait(&bars.pv_empty[set], (k_use - 1) & 1, abort_p, kWaitLimit)) {
+            ok = false;
+            break;
+          }
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            *reinterpret_cast<uint4*>(st + hh * 16384 + ((v ^ xr) << 4)) =
+                make_uint4(h[4 * v], h[4 * v + 1], h[4 * v + 2], h[4 * v + 3]);
+        }
+        if (!ok) break;
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.pv_full[x]);
+        if (lane == 0) mbar_arrive(&bars.pv_full[set]);
       }
     }
   }
