@@ -517,10 +517,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(&bars.s_full[slot], use & 1, abort_p, kWaitLimit)) { ok = false; break; }
           uint32_t h[32];
           dequant_half<FMT>(sring + slot * kSlotBytes + r * 128, xr, u, hh, hh ? (sw >> 16) : (sw & 0xFFFFu), h);
-          if (F::score_releases(hh)) {
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars.s_empty[slot]);
-          }
           if (!valid) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) h[i] = 0u;
@@ -532,6 +528,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tmem_st16(ta + hh * 32, h);
           tmem_st16(ta + hh * 32 + 16, h + 16);
+          // The slot is released only after the stores above have taken the values read from it:
+          // an arrive issued while this warp's shared-memory loads of the slot are still in flight
+          // lets the next TMA load into the slot overwrite them before they are read.
+          if (F::score_releases(hh)) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars.s_empty[slot]);
+          }
         }
         if (!ok) break;
         tmem_st_wait();
@@ -690,10 +693,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(&bars.v_full[slot], use & 1, abort_p, kWaitLimit)) { ok = false; break; }
           uint32_t h[32];
           dequant_half<FMT>(vring + slot * kSlotBytes + r * 128, xr, u, hh, hh ? (sw >> 16) : (sw & 0xFFFFu), h);
-          if (F::score_releases(hh)) {  // same reading pattern as a score half
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars.v_empty[slot]);
-          }
           if (!valid) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) h[i] = 0u;
@@ -707,6 +706,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int v = 0; v < 8; ++v)
             *reinterpret_cast<uint4*>(st + hh * 16384 + ((v ^ xr) << 4)) =
                 make_uint4(h[4 * v], h[4 * v + 1], h[4 * v + 2], h[4 * v + 3]);
+          // released once the stores above have taken the values read from the slot, as on the
+          // score side (and with the same reading pattern as a score half)
+          if (F::score_releases(hh)) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars.v_empty[slot]);
+          }
         }
         if (!ok) break;
         fence_proxy_async_smem();
