@@ -183,6 +183,22 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   while (!mbar_try_wait(bar, parity) && clock64() - t0 < kWaitLimit) {
   }
 }
+// Exit path of a ring producer that issued chunks [0, issued): waits for the latest load into
+// each slot.  Only a slot's latest use is waited for: with sub-rings two of the last chunks can
+// share a slot, and a barrier that has completed both uses reads as not complete for the older.
+// Each owner's latest uses lie within the last 4 x ring chunks.
+template <int FMT>
+__device__ void drain_ring(uint64_t* full, int ring, int issued) {
+  for (int sl = 0; sl < ring; ++sl)
+    for (int i = issued - 1; i >= 0 && i >= issued - 4 * ring; --i) {
+      int slot, use;
+      Fmt<FMT>::s_slot(i, ring, slot, use);
+      if (slot == sl) {
+        drain_wait(&full[slot], use & 1);
+        break;
+      }
+    }
+}
 
 // Dequantise one 16-byte vector of codes into fp16 pairs.
 // FP16: 8 values -> 4 regs; INT8: 16 values -> 8 regs; INT4: 32 values -> 16 regs.
@@ -251,7 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const Shape& s = p.s;
   const int D = s.d;
-  const int split = blockIdx.x, b = blockIdx.y;
+  const int b = blockIdx.x, split = blockIdx.y;
   {
     const int L = p.loops[b], c = p.ctx_len[b];
     if (L < 0 || L > s.L_max || c < 0 || c >= s.max_ctx || p.iter >= L) return;
@@ -346,11 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // every copy issued lands before the CTA's shared memory goes away
       drain_wait(&bars.q_full, 0);
-      for (int i = g > SR ? g - SR : 0; i < g; ++i) {
-        int slot, use;
-        F::s_slot(i, SR, slot, use);
-        drain_wait(&bars.s_full[slot], use & 1);
-      }
+      drain_ring<FMT>(bars.s_full, SR, g);
     }
   } else if (warp == kWarpVP) {
     // ------------------------------------------------------------ TMA producer, P.V-side ring
@@ -375,11 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_2d(vring + slot * kSlotBytes, &tmap, (g % n_chunks) * 128, row_base + r_begin + (g / n_chunks) * 128,
                     &bars.v_full[slot], pol_last_use);
       }
-      for (int i = g > VR ? g - VR : 0; i < g; ++i) {
-        int slot, use;
-        F::v_slot(i, VR, slot, use);
-        drain_wait(&bars.v_full[slot], use & 1);
-      }
+      drain_ring<FMT>(bars.v_full, VR, g);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ score-MMA issuer
@@ -779,7 +787,9 @@ cudaError_t launch_fmt(const DecodeArgs& a, const CUtensorMap& tmap, cudaStream_
                  a.wl.s_max,
                  s_ring,
                  v_ring};
-  dim3 grid(a.wl.s_max, a.n_lanes);
+  // lanes vary fastest, so every lane's first splits are scheduled before any lane's last
+  // (often short) split, and the full-length CTAs fill the first wave
+  dim3 grid(a.n_lanes, a.wl.s_max);
   kern<<<grid, kThreads, smem, st>>>(tmap, p);
   count_launch();
   return cudaGetLastError();

@@ -271,3 +271,26 @@ def test_decode_bitwise_reproducible(name):
         dw.decode(0)
         torch.cuda.synchronize()
         assert np.array_equal(dw.out[0].cpu().numpy(), ref, equal_nan=True)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name", ["fp16_407m", "int8_b16", "int4_2b"])
+def test_decode_has_no_stalled_waits(name):
+    """No decode of a full-size lane takes anywhere near the kernels' bounded-wait limit
+    (about 2 s).  A wait that can never succeed (an exit-path wait on a ring slot whose barrier
+    has moved two phases on, say) ends only at that limit and leaves the results intact, so
+    neither the status word nor the outputs would show it; the time does."""
+    import time
+    w = get_workload(name)
+    w = select_lanes(w, [0])
+    dw = _dw(w)
+    worst = 0.0
+    for rep in range(3):
+        for it in range(w.L_max):
+            dw.append_new(it)
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            dw.decode(it)
+            torch.cuda.synchronize()
+            worst = max(worst, time.perf_counter() - t0)
+    assert worst < 0.25, f"{name}: slowest decode took {worst:.3f} s"
