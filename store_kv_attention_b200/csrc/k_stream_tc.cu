@@ -116,6 +116,22 @@ struct Fmt {
     use = k / R;
   }
   __host__ __device__ static void v_slot(int g, int ring, int& slot, int& use) { s_slot(g, ring, slot, use); }
+
+  // A consumer warp's place in its sub-ring.  Each consumer warp reads every chunk of its owner
+  // (INT4: the one owner; INT8 / FP16: its score half or P.V set) in order, so its k-th chunk
+  // is in slot o * R + k % R, use k / R (as s_slot maps it), and the place moves on once per
+  // chunk the warp releases -- no division in the consumers' loops.
+  struct Cursor {
+    int base, R, idx, use;
+    __device__ Cursor(int owner, int ring) : base(owner * (ring / kOwnersS)), R(ring / kOwnersS), idx(0), use(0) {}
+    __device__ int slot() const { return base + idx; }
+    __device__ void next() {
+      if (++idx == R) {
+        idx = 0;
+        ++use;
+      }
+    }
+  };
 };
 
 struct StreamParams {
@@ -503,6 +519,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (FMT == TL_H_INT8_TOKEN && row_valid(0)) scale_next = __ldg(reinterpret_cast<const float*>(p.scales) + row_of(0));
     if (FMT == TL_H_INT4_G64 && row_valid(0)) prefetch_l1(p.scales + row_of(0) * (size_t)scale_words * 4);
 
+    typename F::Cursor cur(FMT == TL_H_INT4_G64 ? 0 : half, SR);
     for (int t = 0; t < n_tiles && ok; ++t) {
       const bool valid = row_valid(t);
       const float scale_row = scale_next;
@@ -513,22 +530,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
 
       // ------------------------------------------------ this half's units of tile t -> TMEM staging
+      // Rows past the lane's end are not zeroed: a score row depends on its own operand row
+      // only, and its score is masked to -inf below.
       for (int u = half; u < n_units; u += 2) {
         const uint32_t sw = (FMT == TL_H_INT4_G64 && valid) ? __ldg(srow + u) : 0u;  // groups 2u | 2u+1
         const int k_use = t * (n_units >> 1) + (u >> 1);
         const uint32_t ta = tbase + lane_off + kColStg + half * 64;
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
-          const int g = t * n_chunks + F::chunk(u, hh);
-          int slot, use;
-          F::s_slot(g, SR, slot, use);
-          if (!mbar_wait(&bars.s_full[slot], use & 1, abort_p, kWaitLimit)) { ok = false; break; }
+          const int slot = cur.slot();
+          if (!mbar_wait(&bars.s_full[slot], cur.use & 1, abort_p, kWaitLimit)) { ok = false; break; }
           uint32_t h[32];
           dequant_half<FMT>(sring + slot * kSlotBytes + r * 128, xr, u, hh, hh ? (sw >> 16) : (sw & 0xFFFFu), h);
-          if (!valid) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) h[i] = 0u;
-          }
           if (hh == 0) {
             // the staging buffer is free once the MMAs of this half's previous unit are done
             if (k_use >= 1 && !mbar_wait(&bars.stg_empty[half], (k_use - 1) & 1, abort_p, kWaitLimit)) { ok = false; break; }
@@ -542,6 +555,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (F::score_releases(hh)) {
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars.s_empty[slot]);
+            cur.next();
           }
         }
         if (!ok) break;
@@ -686,8 +700,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     auto row_of = [&](int t) { return (size_t)row_base + r_begin + t * 128 + r; };
     auto row_valid = [&](int t) { return r < (r_end - (r_begin + t * 128)); };
+    typename F::Cursor cur(FMT == TL_H_INT4_G64 ? 0 : set, VR);
     for (int t = 0; t < n_tiles && ok; ++t) {
       const bool valid = row_valid(t);
+      // Rows past the lane's end meet P = 0.  INT4 rows there get scale 0 and INT8 codes are
+      // finite, so only FP16 rows (whose bytes may hold Inf or NaN) are zeroed, and only in a
+      // tile that has such rows.
+      const bool zero_rows = FMT == TL_H_FP16 && __any_sync(0xffffffffu, !valid);
       const uint32_t* srow = reinterpret_cast<const uint32_t*>(p.scales + row_of(t) * (size_t)scale_words * 4);
       for (int u = set; u < n_units && ok; u += 2) {
         const uint32_t sw = (FMT == TL_H_INT4_G64 && valid) ? __ldg(srow + u) : 0u;  // groups 2u | 2u+1
@@ -695,13 +714,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* st = pvs + set * kPvStageBytes + r * 128;
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
-          const int g = t * n_chunks + F::chunk(u, hh);
-          int slot, use;
-          F::v_slot(g, VR, slot, use);
-          if (!mbar_wait(&bars.v_full[slot], use & 1, abort_p, kWaitLimit)) { ok = false; break; }
+          const int slot = cur.slot();
+          if (!mbar_wait(&bars.v_full[slot], cur.use & 1, abort_p, kWaitLimit)) { ok = false; break; }
           uint32_t h[32];
           dequant_half<FMT>(vring + slot * kSlotBytes + r * 128, xr, u, hh, hh ? (sw >> 16) : (sw & 0xFFFFu), h);
-          if (!valid) {
+          if (zero_rows && !valid) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) h[i] = 0u;
           }
@@ -719,6 +736,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (F::score_releases(hh)) {
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars.v_empty[slot]);
+            cur.next();
           }
         }
         if (!ok) break;
