@@ -254,6 +254,20 @@ __device__ __forceinline__ void dequant_vec(const uint4 v, uint32_t* out, __half
   }
 }
 
+// INT4: the unit's four 16-byte code vectors of this row (both half-units of unit u lie in one
+// slot row), loaded together so that their latencies overlap.
+__device__ __forceinline__ void load_unit_int4(const uint8_t* row, int xr, int u, uint4* c) {
+  const int v0 = (u & 1) * 4;
+#pragma unroll
+  for (int v = 0; v < 4; ++v) c[v] = *reinterpret_cast<const uint4*>(row + (((v0 + v) ^ xr) << 4));
+}
+// INT4: half-unit hh of loaded code vectors c into h[32], scale bits from the unit's scale word.
+__device__ __forceinline__ void dequant_int4_half(const uint4* c, int hh, uint32_t sw, uint32_t* h) {
+  const __half2 s2 = splat_h(hh ? (sw >> 16) : (sw & 0xFFFFu));
+  dequant_vec<TL_H_INT4_G64>(c[2 * hh], h, s2);
+  dequant_vec<TL_H_INT4_G64>(c[2 * hh + 1], h + 16, s2);
+}
+
 // Dequantise half-unit hh (64 values) of unit u from a codes slot row into h[32].
 // INT4: the scale of group 2u + hh comes in `sbits` (fp16 bits).
 template <int FMT>
@@ -536,6 +550,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t sw = (FMT == TL_H_INT4_G64 && valid) ? __ldg(srow + u) : 0u;  // groups 2u | 2u+1
         const int k_use = t * (n_units >> 1) + (u >> 1);
         const uint32_t ta = tbase + lane_off + kColStg + half * 64;
+        if constexpr (FMT == TL_H_INT4_G64) {
+          // one slot wait per unit; the whole unit's codes loaded at once
+          const int slot = cur.slot();
+          if (!mbar_wait(&bars.s_full[slot], cur.use & 1, abort_p, kWaitLimit)) { ok = false; break; }
+          uint4 c[4];
+          load_unit_int4(sring + slot * kSlotBytes + r * 128, xr, u, c);
+          uint32_t h[32];
+          dequant_int4_half(c, 0, sw, h);
+          if (k_use >= 1 && !mbar_wait(&bars.stg_empty[half], (k_use - 1) & 1, abort_p, kWaitLimit)) { ok = false; break; }
+          tc_fence_after();
+          tmem_st16(ta, h);
+          tmem_st16(ta + 16, h + 16);
+          dequant_int4_half(c, 1, sw, h);
+          tmem_st16(ta + 32, h);
+          tmem_st16(ta + 48, h + 16);
+          // released only after the stores above have taken the values read from the slot
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars.s_empty[slot]);
+          cur.next();
+        } else {
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           const int slot = cur.slot();
@@ -557,6 +591,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) mbar_arrive(&bars.s_empty[slot]);
             cur.next();
           }
+        }
         }
         if (!ok) break;
         tmem_st_wait();
@@ -712,6 +747,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t sw = (FMT == TL_H_INT4_G64 && valid) ? __ldg(srow + u) : 0u;  // groups 2u | 2u+1
         const int k_use = t * (n_units >> 1) + (u >> 1);  // this set's units so far
         uint8_t* st = pvs + set * kPvStageBytes + r * 128;
+        if constexpr (FMT == TL_H_INT4_G64) {
+          const int slot = cur.slot();
+          if (!mbar_wait(&bars.v_full[slot], cur.use & 1, abort_p, kWaitLimit)) { ok = false; break; }
+          uint4 c[4];
+          load_unit_int4(vring + slot * kSlotBytes + r * 128, xr, u, c);
+          uint32_t h[32];
+          dequant_int4_half(c, 0, sw, h);
+          if (k_use >= 1 && !mbar_wait(&bars.pv_empty[set], (k_use - 1) & 1, abort_p, kWaitLimit)) { ok = false; break; }
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            *reinterpret_cast<uint4*>(st + ((v ^ xr) << 4)) = make_uint4(h[4 * v], h[4 * v + 1], h[4 * v + 2], h[4 * v + 3]);
+          dequant_int4_half(c, 1, sw, h);
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            *reinterpret_cast<uint4*>(st + 16384 + ((v ^ xr) << 4)) =
+                make_uint4(h[4 * v], h[4 * v + 1], h[4 * v + 2], h[4 * v + 3]);
+          // released only after the stores above have taken the values read from the slot
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars.v_empty[slot]);
+          cur.next();
+        } else {
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           const int slot = cur.slot();
@@ -738,6 +794,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) mbar_arrive(&bars.v_empty[slot]);
             cur.next();
           }
+        }
         }
         if (!ok) break;
         fence_proxy_async_smem();
