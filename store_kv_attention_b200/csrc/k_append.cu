@@ -5,6 +5,7 @@
 // One CTA of 128 threads per (row, lane).  Codes are bit-exact with the format
 // definitions in tl_storeh.h: the scale is an IEEE fp32 division of the absolute
 // maximum, every code an IEEE fp32 division rounded half to even, then clamped.
+#include "tc_ptx.cuh"
 #include "tl_internal.cuh"
 
 namespace tl {
@@ -29,6 +30,8 @@ __global__ void __launch_bounds__(kThreads) append_kernel(Shape s, uint8_t* code
                                                           const int32_t* __restrict__ start_pos,
                                                           const int32_t* __restrict__ row_count,
                                                           const int32_t* __restrict__ loops) {
+  ptx::pdl_wait();  // the rows may come from the previous kernel in the stream
+  ptx::pdl_trigger();
   const int r = blockIdx.x;
   const int b = blockIdx.y;
   if (loops && layer >= s.n_pre + loops[b]) return;
@@ -86,10 +89,17 @@ cudaError_t launch_append(const Shape& s, void* codes, void* scales, int layer, 
                           int n_rows, const int32_t* start_pos, const int32_t* row_count, const int32_t* loops,
                           cudaStream_t st) {
   if (n_lanes > 65535) return cudaErrorInvalidValue;
-  dim3 grid(n_rows, n_lanes);
-  append_kernel<<<grid, kThreads, 0, st>>>(s, (uint8_t*)codes, (uint8_t*)scales, layer, h_rows, n_rows, start_pos,
-                                           row_count, loops);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(n_rows, n_lanes, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1] = {pdl_attribute()};
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, append_kernel, s, (uint8_t*)codes, (uint8_t*)scales, layer, h_rows, n_rows,
+                                     start_pos, row_count, loops);
   count_launch();
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

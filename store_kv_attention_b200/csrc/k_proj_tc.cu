@@ -136,6 +136,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
 
+  pdl_wait();  // h_new and the workspace may come from the previous kernel in the stream
   if (threadIdx.x == 0) {
     mbar_init(&bar_ld1, 1);
     mbar_init(&bar_ld2, 1);
@@ -156,6 +157,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   tc_fence_after();
   const uint32_t tbase = tmem_base;
   volatile int* abort_p = &abort_flag;
+  pdl_trigger();  // TMEM is held
 
   // ---------------------------------------------------------------- phase-1 loads (phase 2 loads once they are dead)
   if (threadIdx.x == 0) {
@@ -449,6 +451,7 @@ __global__ void __launch_bounds__(kOProjThreads, 1)
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
 
+  pdl_wait();  // the split partials come from the streaming kernel just before
   if (threadIdx.x == 0) {
     mbar_init(&bar_ld, 1);
     mbar_init(&bar_m, 1);
@@ -465,6 +468,7 @@ __global__ void __launch_bounds__(kOProjThreads, 1)
   tc_fence_after();
   const uint32_t tbase = tmem_base;
   volatile int* abort_p = &abort_flag;
+  pdl_trigger();  // TMEM is held
 
   if (threadIdx.x == 0) {
     mbar_expect_tx(&bar_ld, (uint32_t)lay.nk * kTileBytes);
@@ -714,13 +718,14 @@ cudaError_t launch_qproj(const DecodeArgs& a, cudaStream_t st) {
   cfg.blockDim = dim3(kProjThreads, 1, 1);
   cfg.dynamicSmemBytes = lay.total;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = CL;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1] = pdl_attribute();
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   e = cudaLaunchKernelEx(&cfg, qproj_kernel, tmWq, tmH, tmWk, p);
   count_launch();
   if (e != cudaSuccess) return e;
@@ -758,13 +763,14 @@ cudaError_t launch_oproj(const DecodeArgs& a, cudaStream_t st) {
   cfg.blockDim = dim3(kOProjThreads, 1, 1);
   cfg.dynamicSmemBytes = lay.total;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = CL;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1] = pdl_attribute();
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   e = cudaLaunchKernelEx(&cfg, oproj_kernel, tmWv, p);
   count_launch();
   if (e != cudaSuccess) return e;

@@ -297,6 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const Shape& s = p.s;
   const int D = s.d;
+  pdl_wait();  // the absorbed-query images (and the cache rows) come from the kernels just before
   const int b = blockIdx.x, split = blockIdx.y;
   {
     const int L = p.loops[b], c = p.ctx_len[b];
@@ -367,6 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tbase = tmem_base;
   volatile int* abort_p = &abort_flag;
+  pdl_trigger();  // TMEM is held
 
   volatile int* s_issued_p = &s_issued;
   const int total_chunks = n_tiles * n_chunks;
@@ -864,9 +866,17 @@ cudaError_t launch_fmt(const DecodeArgs& a, const CUtensorMap& tmap, cudaStream_
                  v_ring};
   // lanes vary fastest, so every lane's first splits are scheduled before any lane's last
   // (often short) split, and the full-length CTAs fill the first wave
-  dim3 grid(a.n_lanes, a.wl.s_max);
-  kern<<<grid, kThreads, smem, st>>>(tmap, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.n_lanes, a.wl.s_max, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1] = {pdl_attribute()};
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, tmap, p);
   count_launch();
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -48,6 +48,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialization may be scheduled before the previous
+// kernel in its stream has finished.  pdl_wait() returns once that kernel has completed and its
+// memory is visible (at once when the launch was an ordinary one), so every kernel calls it before
+// its first access to global memory.  pdl_trigger() lets the next kernel be scheduled once every
+// CTA of this grid has issued it or exited; each kernel issues it only after it holds its TMEM, so
+// an early CTA of the next kernel can never take TMEM that a CTA of this one still waits for.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- proxies / fences
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t threads) {

@@ -112,6 +112,15 @@ inline Workspace workspace_layout(const Shape& s, int n_lanes) {
   return w;
 }
 
+// Launch attribute for programmatic dependent launch: the kernel may be scheduled while the previous
+// kernel in the stream drains, and waits for it (griddepcontrol.wait) before touching global memory.
+inline cudaLaunchAttribute pdl_attribute() {
+  cudaLaunchAttribute a;
+  a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  a.val.programmaticStreamSerializationAllowed = 1;
+  return a;
+}
+
 // Records a message for tl_last_error_message() and returns `st`.
 tl_status set_error(tl_status st, const char* fmt, ...);
 
