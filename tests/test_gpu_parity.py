@@ -294,3 +294,25 @@ def test_decode_has_no_stalled_waits(name):
             torch.cuda.synchronize()
             worst = max(worst, time.perf_counter() - t0)
     assert worst < 0.25, f"{name}: slowest decode took {worst:.3f} s"
+
+
+def test_decode_at_maximum_sizes():
+    """The largest decode call the kernels take: 64 lanes, one of them with 65535 cached
+    positions (64 splits of 1024 rows, the most a lane can have), the others ragged down to no
+    cached position at all; sampled lanes against the oracle."""
+    import dataclasses
+    import store_kv_attention_b200 as tl
+    ctx = [65535] + [(37 * b * b + 11 * b) % 3000 for b in range(1, 64)]
+    ctx[1], ctx[2], ctx[63] = 0, 1, 4097
+    loops = [2 if b % 2 == 0 else 1 for b in range(64)]
+    w = dataclasses.replace(get_workload("int4_2b"), ctx=ctx, loops=loops, n_pre=1, L_max=2, name="int4_2b_max")
+    dw = _dw(w)
+    dw.step()
+    torch.cuda.synchronize()
+    assert tl.poll_status(dw.cache) == tl.TL_OK
+    out = dw.out.cpu().numpy()
+    for it, b in [(0, 0), (1, 0), (0, 1), (0, 2), (1, 40), (0, 63)]:
+        assert it < w.loops[b]
+        _assert_close(out[it, b], _oracle_lane(w, it, b, form="absorbed"), f"max sizes lane {b} it {it}")
+    act = np.array([[it < w.loops[b] for b in range(w.B)] for it in range(w.L_max)])
+    assert np.all(np.isfinite(out[act])) and np.all(np.isnan(out[~act]))
