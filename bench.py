@@ -54,6 +54,22 @@ def workload_for_rank(name, rank):
     return w
 
 
+def max_over_ranks(value, world, device):
+    """The largest of every rank's `value` (each rank gets it); `value` itself on one rank."""
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank_step, steps, ms_max, world):
+    """Units all ranks processed per second, timed by the slowest rank (weak scaling: every rank
+    has its own batch of the same shape)."""
+    return world * steps * units_per_rank_step / (ms_max / 1000.0)
+
+
 def row_bytes(w):
     return {0: 2 * w.d, 1: w.d + 4, 2: w.d // 2 + 2 * (w.d // 64)}[w.fmt]
 
@@ -278,13 +294,9 @@ def run_ours(args, rank, world, local_rank):
             for _ in range(K):
                 dw.step()
             torch.cuda.synchronize()
-    ms = start.elapsed_time(end)
-    t = torch.tensor([ms], dtype=torch.float64, device=f"cuda:{local_rank}")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(start.elapsed_time(end), world, f"cuda:{local_rank}")
     pos_step = w.cached_positions_per_step()
-    value = world * K * pos_step / (ms_max / 1000.0)
+    value = whole_job_rate(pos_step, K, ms_max, world)
 
     # dominant kernel (context streaming): algorithmic bytes per launch / CUDA-event duration
     kms = prof.stream_kernel_ms()
@@ -360,10 +372,7 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     for n in names:
         setattr(dw, n, sets[0][n])
-    t2 = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=f"cuda:{local_rank}")
-    if world > 1:
-        dist.all_reduce(t2, op=dist.ReduceOp.MAX)
-    e2e_value = world * K * pos_step / (float(t2.item()) / 1000.0)
+    e2e_value = whole_job_rate(pos_step, K, max_over_ranks(e0.elapsed_time(e1), world, f"cuda:{local_rank}"), world)
 
     if rank != 0:
         return
