@@ -257,6 +257,7 @@ __device__ __forceinline__ void dequant_vec(const uint4 v, uint32_t* out, __half
 // INT4: the unit's four 16-byte code vectors of this row (both half-units of unit u lie in one
 // slot row), loaded together so that their latencies overlap.
 __device__ __forceinline__ void load_unit_int4(const uint8_t* row, int xr, int u, uint4* c) {
+  static_assert(2 * Fmt<TL_H_INT4_G64>::kVecs == 4, "an INT4 unit row is four 16-byte vectors");
   const int v0 = (u & 1) * 4;
 #pragma unroll
   for (int v = 0; v < 4; ++v) c[v] = *reinterpret_cast<const uint4*>(row + (((v0 + v) ^ xr) << 4));

@@ -109,7 +109,7 @@ const char* tl_status_string(tl_status st) {
 }
 
 tl_status tl_storeh_cache_bytes(const tl_storeh_desc* desc, size_t* codes_bytes, size_t* scales_bytes) {
-  tl::Shape s;
+  tl::Shape s{};
   tl_status st = check_desc(desc, &s);
   if (st != TL_OK) return st;
   if (!codes_bytes || !scales_bytes) return fail(TL_ERR_INVALID_ARG, "output pointer is NULL");
@@ -119,7 +119,7 @@ tl_status tl_storeh_cache_bytes(const tl_storeh_desc* desc, size_t* codes_bytes,
 }
 
 tl_status tl_storeh_workspace_bytes(const tl_storeh_desc* desc, int32_t n_lanes, size_t* bytes) {
-  tl::Shape s;
+  tl::Shape s{};
   tl_status st = check_desc(desc, &s);
   if (st != TL_OK) return st;
   if (!bytes) return fail(TL_ERR_INVALID_ARG, "bytes is NULL");
@@ -135,7 +135,7 @@ tl_status tl_storeh_append(const tl_storeh_desc* desc, tl_storeh_cache cache, in
                            const void* h_rows, int32_t n_lanes, int32_t n_rows,
                            const int32_t* start_pos, const int32_t* row_count,
                            const int32_t* loops, tl_stream_t stream) {
-  tl::Shape s;
+  tl::Shape s{};
   tl_status st = check_desc(desc, &s);
   if (st != TL_OK) return st;
   if ((st = check_cache(s, cache)) != TL_OK) return st;
@@ -170,7 +170,7 @@ tl_status tl_storeh_attn_decode(const tl_storeh_desc* desc, tl_storeh_cache cach
                                 const float* residual, float threshold, uint8_t* abort_flags,
                                 int32_t* first_abort_iter, float* norms_out, void* workspace,
                                 size_t workspace_bytes, int32_t n_lanes, tl_stream_t stream) {
-  tl::Shape s;
+  tl::Shape s{};
   tl_status st = check_desc(desc, &s);
   if (st != TL_OK) return st;
   if ((st = check_cache(s, cache)) != TL_OK) return st;
