@@ -22,6 +22,11 @@
  *     no state between calls.
  *   - Work is enqueued asynchronously on `stream` (NULL = legacy default stream);
  *     a return of TL_OK means "validated and launched", not "finished".
+ *   - Kernels are launched with programmatic dependent launch: one may be
+ *     scheduled while the kernel before it on the stream is still finishing, but
+ *     it touches no memory until that kernel has completed, so stream order holds
+ *     exactly as for ordinary launches (inputs written by the preceding kernel are
+ *     seen, outputs are not written before it is done).
  *   - Arguments are validated on the host before anything is launched; a
  *     non-TL_OK return means nothing was enqueued, except TL_ERR_CUDA, which
  *     reports a failed launch.  tl_last_error_message() gives details.
@@ -242,7 +247,10 @@ TL_API tl_status tl_storeh_poll_status(void* workspace, size_t workspace_bytes, 
  * (cudaEvent_t handles created by the caller) on the call's stream right before
  * and right after each launch of the context-streaming kernel of
  * tl_storeh_attn_decode, for k = recorded++ while recorded < capacity.
- * Pass NULL to uninstall.  The struct must outlive its installation.
+ * Pass NULL to uninstall.  The struct must outlive its installation.  The events
+ * sit between kernels, which stops a kernel from being scheduled during the tail
+ * of the one before it, so a step timed with the hook installed runs a little
+ * slower than one without.
  */
 typedef struct {
   void** begin_events;
