@@ -271,7 +271,7 @@ def run_ours(args, rank, world, local_rank):
             dist.barrier()
 
     for _ in range(args.warmup):
-        dw.step()
+        dw.step(fused_append=True)
     torch.cuda.synchronize()
     if tl.poll_status(dw.cache) != tl.TL_OK:
         raise RuntimeError("device status after warm-up: " + tl.lib.tl_last_error_message().decode())
@@ -285,14 +285,14 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         start.record(stream)
         for _ in range(K):
-            dw.step()
+            dw.step(fused_append=True)
         end.record(stream)
         torch.cuda.synchronize()
         barrier()
         # kernel pass: the same K steps again, with events around every streaming-kernel launch
         with tl.ProfileHook(K * w.L_max) as prof:
             for _ in range(K):
-                dw.step()
+                dw.step(fused_append=True)
             torch.cuda.synchronize()
     ms_max = max_over_ranks(start.elapsed_time(end), world, f"cuda:{local_rank}")
     pos_step = w.cached_positions_per_step()
@@ -358,7 +358,7 @@ def run_ours(args, rank, world, local_rank):
         for n in names:
             setattr(dw, n, sets[i][n])
         dw.reset_flags()
-        dw.step()
+        dw.step(fused_append=True)
         inputs_free[i].record(stream)
         with torch.cuda.stream(down):
             down.wait_event(inputs_free[i])
@@ -384,7 +384,8 @@ def run_ours(args, rank, world, local_rank):
             "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": DTYPE_OF_FMT[w.fmt] + "-h codes, fp16 tensor operands, fp32 accumulate",
             "data": "synthetic (seeded generator: SplitMix64 + Box-Muller)",
-            "config": workload_config(w, world, {"cached_positions_per_step_per_gpu": pos_step,
+            "config": workload_config(w, world, {"entry_point": "tl_storeh_append_attn_decode per loop iteration",
+                                                 "cached_positions_per_step_per_gpu": pos_step,
                                                  "step_roofline_ms_hbm": step_roofline_ms,
                                                  "step_frac_of_hbm_roofline": step_roofline_ms / (ms_max / K)}),
             "roofline": roofline,

@@ -178,6 +178,24 @@ TL_API tl_status tl_storeh_attn_decode(const tl_storeh_desc* desc, tl_storeh_cac
                                 size_t workspace_bytes, int32_t n_lanes, tl_stream_t stream);
 
 /*
+ * tl_storeh_append followed by tl_storeh_attn_decode in one enqueue: for every lane b
+ * with iter < loops[b] (and loops[b], ctx_len[b] in range), h_new[b] is first
+ * quantised into cache layer n_pre + iter at position ctx_len[b] -- exactly what
+ * tl_storeh_append(desc, cache, n_pre + iter, h_new, n_lanes, 1, ctx_len, NULL,
+ * loops, stream) writes -- and then the decode of tl_storeh_attn_decode runs on it.
+ * The append is done inside the decode's first kernel while its weight tiles load,
+ * which saves a launch and its latency per iteration.  Arguments, results and
+ * errors as for tl_storeh_attn_decode; h_new is both the row appended and the query
+ * input.
+ */
+TL_API tl_status tl_storeh_append_attn_decode(const tl_storeh_desc* desc, tl_storeh_cache cache, int32_t iter,
+                                const int32_t* loops, const int32_t* ctx_len, const void* h_new,
+                                const void* W_q, const void* W_k, const void* W_v, float* out,
+                                const float* residual, float threshold, uint8_t* abort_flags,
+                                int32_t* first_abort_iter, float* norms_out, void* workspace,
+                                size_t workspace_bytes, int32_t n_lanes, tl_stream_t stream);
+
+/*
  * Per-iteration safety check [Novel Contributions, "Novel: Per-Iteration
  * Safety Check"; Architecture-Exclusive Features, "Per-iteration safety check"].
  * For every lane b with iter < loops[b] (all lanes when loops is NULL):

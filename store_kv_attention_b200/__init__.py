@@ -34,7 +34,8 @@ TL_H_INT4_G64 = 2
 # every symbol include/tl_storeh.h declares
 EXPORTS = ["tl_storeh_cache_bytes", "tl_storeh_workspace_bytes", "tl_storeh_append", "tl_storeh_attn_decode",
            "tl_residual_norm_check", "tl_storeh_poll_status", "tl_status_string", "tl_last_error_message",
-           "tl_storeh_abi_version", "tl_set_profile", "tl_storeh_attn_decode_static_ws"]
+           "tl_storeh_abi_version", "tl_set_profile", "tl_storeh_attn_decode_static_ws",
+           "tl_storeh_append_attn_decode"]
 
 
 class TLError(RuntimeError):
@@ -77,10 +78,11 @@ def _load():
     L.tl_storeh_append.argtypes = [P(Desc), Cache, i32, vp, i32, i32, vp, vp, vp, vp]
     L.tl_storeh_attn_decode.argtypes = [P(Desc), Cache, i32, vp, vp, vp, vp, vp, vp, vp, vp, f32, vp, vp, vp, vp,
                                         sz, i32, vp]
+    L.tl_storeh_append_attn_decode.argtypes = L.tl_storeh_attn_decode.argtypes
     L.tl_residual_norm_check.argtypes = [vp, i32, i32, f32, i32, vp, vp, vp, vp, vp]
     L.tl_storeh_poll_status.argtypes = [vp, sz, vp]
     for f in ("tl_storeh_cache_bytes", "tl_storeh_workspace_bytes", "tl_storeh_append", "tl_storeh_attn_decode",
-              "tl_residual_norm_check", "tl_storeh_poll_status"):
+              "tl_storeh_append_attn_decode", "tl_residual_norm_check", "tl_storeh_poll_status"):
         getattr(L, f).restype = ctypes.c_int
     L.tl_status_string.argtypes = [ctypes.c_int]
     L.tl_status_string.restype = ctypes.c_char_p
@@ -181,13 +183,15 @@ def append(cache: StoreHCache, layer: int, h_rows, start_pos, row_count=None, lo
 
 def attn_decode(cache: StoreHCache, it: int, loops, ctx_len, h_new, W_q, W_k, W_v, out,
                 residual=None, threshold: float = 0.0, abort_flags=None, first_abort_iter=None,
-                norms_out=None, stream=None) -> None:
+                norms_out=None, stream=None, append: bool = False) -> None:
+    """tl_storeh_attn_decode, or with append=True tl_storeh_append_attn_decode (h_new is first
+    written as the new token's row of every active lane, in the same enqueue)."""
     n_lanes = int(h_new.shape[0])
-    _check(_load().tl_storeh_attn_decode(ctypes.byref(cache.desc.c()), cache.c(), it, _ptr(loops), _ptr(ctx_len),
-                                     _ptr(h_new), _ptr(W_q), _ptr(W_k), _ptr(W_v), _ptr(out), _ptr(residual),
-                                     float(threshold), _ptr(abort_flags), _ptr(first_abort_iter), _ptr(norms_out),
-                                     cache.workspace.data_ptr(), cache.ws_bytes, n_lanes, _stream(stream)),
-           "tl_storeh_attn_decode")
+    name = "tl_storeh_append_attn_decode" if append else "tl_storeh_attn_decode"
+    _check(getattr(_load(), name)(ctypes.byref(cache.desc.c()), cache.c(), it, _ptr(loops), _ptr(ctx_len),
+                                  _ptr(h_new), _ptr(W_q), _ptr(W_k), _ptr(W_v), _ptr(out), _ptr(residual),
+                                  float(threshold), _ptr(abort_flags), _ptr(first_abort_iter), _ptr(norms_out),
+                                  cache.workspace.data_ptr(), cache.ws_bytes, n_lanes, _stream(stream)), name)
 
 
 def attn_decode_static_ws(cache: StoreHCache, it: int, loops, ctx_len, h_new, W_q, W_k, W_v, out,

@@ -22,6 +22,7 @@
 
 #include <mutex>
 
+#include "append_row.cuh"
 #include "cluster_ptx.cuh"
 #include "norm_block.cuh"
 #include "tc_ptx.cuh"
@@ -82,6 +83,10 @@ struct QProjParams {
   int cl;            // cluster size = K splits of q
   uint32_t* status;
   uint8_t* qimg;     // [n_lanes][qimg_bytes(d)]
+  // fused append (codes == NULL: none): h_new of every active lane becomes its new token's row
+  const __half* h_new;
+  uint8_t* codes;
+  uint8_t* scales;
 };
 
 // Shared memory: region 0 holds the phase-1 operands; once the phase-1 MMAs are done it
@@ -166,6 +171,20 @@ __global__ void __launch_bounds__(kProjThreads, 1)
       const int x = k * lay.KS + 64 * i;
       tma_2d(a1 + i * kTileBytes, &tmWq, x, mb * 128, &bar_ld1);
       tma_2d(b1 + i * nb * 128, &tmH, x, 0, &bar_ld1);  // rows past n_lanes read as zero
+    }
+  }
+
+  // ---------------------------------------------------------------- fused append (optional)
+  // Each CTA quantises the new token's row of some active lanes into the cache while its weight
+  // tiles load.  Nothing in this kernel reads the cache; the streaming kernel that does runs
+  // only once this kernel has completed.
+  if (p.codes) {
+    const int n_ctas = (int)(gridDim.x * gridDim.y);
+    for (int b = (int)(blockIdx.y * gridDim.x + blockIdx.x); b < p.n_lanes; b += n_ctas) {
+      int nr;
+      if (!lane_active(s, p.iter, p.loops, p.ctx_len, b, &nr)) continue;  // the same for the whole CTA
+      const size_t row = ((size_t)(s.n_pre + p.iter) * s.max_lanes + b) * s.max_ctx + (size_t)(nr - 1);
+      append_row_block<kProjThreads>(s, p.codes, p.scales, row, p.h_new + (size_t)b * s.d);
     }
   }
 
@@ -711,8 +730,18 @@ cudaError_t launch_qproj(const DecodeArgs& a, cudaStream_t st) {
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(qproj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lay.total);
   if (e != cudaSuccess) return e;
-  QProjParams p{s, a.iter, a.loops, a.ctx_len, a.n_lanes, w.nb, CL,
-                reinterpret_cast<uint32_t*>(a.ws + w.status_off), a.ws + w.qt_off};
+  QProjParams p{s,
+                a.iter,
+                a.loops,
+                a.ctx_len,
+                a.n_lanes,
+                w.nb,
+                CL,
+                reinterpret_cast<uint32_t*>(a.ws + w.status_off),
+                a.ws + w.qt_off,
+                a.h_new,
+                a.append ? (uint8_t*)a.codes : nullptr,
+                a.append ? (uint8_t*)a.scales : nullptr};
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(CL, s.d / 128, 1);
   cfg.blockDim = dim3(kProjThreads, 1, 1);

@@ -164,12 +164,14 @@ tl_status tl_residual_norm_check(const float* residual, int32_t n_lanes, int32_t
   return TL_OK;
 }
 
-tl_status tl_storeh_attn_decode(const tl_storeh_desc* desc, tl_storeh_cache cache, int32_t iter,
-                                const int32_t* loops, const int32_t* ctx_len, const void* h_new,
-                                const void* W_q, const void* W_k, const void* W_v, float* out,
-                                const float* residual, float threshold, uint8_t* abort_flags,
-                                int32_t* first_abort_iter, float* norms_out, void* workspace,
-                                size_t workspace_bytes, int32_t n_lanes, tl_stream_t stream) {
+namespace {
+// The decode, optionally preceded (inside its first kernel) by the append of h_new as the new
+// token's row of every active lane.
+tl_status decode_impl(const tl_storeh_desc* desc, tl_storeh_cache cache, int32_t iter, const int32_t* loops,
+                      const int32_t* ctx_len, const void* h_new, const void* W_q, const void* W_k, const void* W_v,
+                      float* out, const float* residual, float threshold, uint8_t* abort_flags,
+                      int32_t* first_abort_iter, float* norms_out, void* workspace, size_t workspace_bytes,
+                      int32_t n_lanes, tl_stream_t stream, bool append) {
   tl::Shape s{};
   tl_status st = check_desc(desc, &s);
   if (st != TL_OK) return st;
@@ -194,6 +196,7 @@ tl_status tl_storeh_attn_decode(const tl_storeh_desc* desc, tl_storeh_cache cach
   tl::DecodeArgs a{s, cache.codes, cache.scales, iter, loops, ctx_len, (const __half*)h_new,
                    (const __half*)W_q, (const __half*)W_k, (const __half*)W_v, out, n_lanes,
                    (uint8_t*)workspace, wl, residual, threshold, abort_flags, first_abort_iter, norms_out};
+  a.append = append;
   cudaStream_t cs = (cudaStream_t)stream;
   cudaError_t e = tl::launch_qproj(a, cs);
   if (e != cudaSuccess) return cuda_fail(e, "decode prologue launch");
@@ -204,6 +207,25 @@ tl_status tl_storeh_attn_decode(const tl_storeh_desc* desc, tl_storeh_cache cach
   e = tl::launch_oproj(a, cs);
   if (e != cudaSuccess) return cuda_fail(e, "decode epilogue launch");
   return TL_OK;
+}
+}  // namespace
+
+tl_status tl_storeh_attn_decode(const tl_storeh_desc* desc, tl_storeh_cache cache, int32_t iter,
+                                const int32_t* loops, const int32_t* ctx_len, const void* h_new,
+                                const void* W_q, const void* W_k, const void* W_v, float* out,
+                                const float* residual, float threshold, uint8_t* abort_flags,
+                                int32_t* first_abort_iter, float* norms_out, void* workspace,
+                                size_t workspace_bytes, int32_t n_lanes, tl_stream_t stream) {
+  return decode_impl(desc, cache, iter, loops, ctx_len, h_new, W_q, W_k, W_v, out, residual, threshold, abort_flags, first_abort_iter, norms_out, workspace, workspace_bytes, n_lanes, stream, false);
+}
+
+tl_status tl_storeh_append_attn_decode(const tl_storeh_desc* desc, tl_storeh_cache cache, int32_t iter,
+                                const int32_t* loops, const int32_t* ctx_len, const void* h_new,
+                                const void* W_q, const void* W_k, const void* W_v, float* out,
+                                const float* residual, float threshold, uint8_t* abort_flags,
+                                int32_t* first_abort_iter, float* norms_out, void* workspace,
+                                size_t workspace_bytes, int32_t n_lanes, tl_stream_t stream) {
+  return decode_impl(desc, cache, iter, loops, ctx_len, h_new, W_q, W_k, W_v, out, residual, threshold, abort_flags, first_abort_iter, norms_out, workspace, workspace_bytes, n_lanes, stream, true);
 }
 
 tl_status tl_storeh_poll_status(void* workspace, size_t workspace_bytes, tl_stream_t stream) {

@@ -162,6 +162,8 @@ struct DecodeArgs {
   uint8_t* abort_flags;
   int32_t* first_abort_iter;
   float* norms;
+  // append h_new as the new token's row of every active lane first (fused into qproj_kernel)
+  bool append = false;
 };
 
 // Fused q and absorbed-query projections, one thread-block cluster per 128 rows of W_q (k_proj_tc.cu).

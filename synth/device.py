@@ -77,15 +77,21 @@ class DeviceWorkload:
         tl.append(self.cache, self.w.n_pre + it, self.h_new[it].unsqueeze(1), self.ctx, loops=self.loops,
                   stream=stream)
 
-    def decode(self, it: int, fused_check: bool = True, stream=None) -> None:
+    def decode(self, it: int, fused_check: bool = True, stream=None, append: bool = False) -> None:
+        """Iteration `it` of the decode; with append=True the new token's row is written by the
+        same call (tl_storeh_append_attn_decode) instead of a separate append_new."""
         w = self.w
         tl.attn_decode(self.cache, it, self.loops, self.ctx, self.h_new[it], self.W["q"], self.W["k"], self.W["v"],
                        self.out[it], residual=self.residual[it] if fused_check else None, threshold=w.threshold,
                        abort_flags=self.flags, first_abort_iter=self.first, norms_out=self.norms[it],
-                       stream=stream)
+                       stream=stream, append=append)
 
-    def step(self, stream=None) -> None:
-        """One decode step: every loop iteration, append then attend (with the safety check)."""
+    def step(self, stream=None, fused_append: bool = False) -> None:
+        """One decode step: every loop iteration, append then attend (with the safety check),
+        as two calls or (fused_append) as one."""
         for it in range(self.w.L_max):
-            self.append_new(it, stream)
-            self.decode(it, stream=stream)
+            if fused_append:
+                self.decode(it, stream=stream, append=True)
+            else:
+                self.append_new(it, stream)
+                self.decode(it, stream=stream)

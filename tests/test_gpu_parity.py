@@ -316,3 +316,34 @@ def test_decode_at_maximum_sizes():
         _assert_close(out[it, b], _oracle_lane(w, it, b, form="absorbed"), f"max sizes lane {b} it {it}")
     act = np.array([[it < w.loops[b] for b in range(w.B)] for it in range(w.L_max)])
     assert np.all(np.isfinite(out[act])) and np.all(np.isnan(out[~act]))
+
+
+@pytest.mark.parametrize("name,ctx,loops", [
+    ("fp16_407m", [0, 5, 130, 1030], [3, 1, 3, 2]),
+    ("int8_b16", [1, 255, 1024, 2049], [2, 3, 1, 3]),
+    ("int4_2b", [0, 3, 1000, 2048], [3, 1, 2, 3]),
+], ids=["fp16", "int8", "int4"])
+def test_fused_append_equals_separate_calls(name, ctx, loops):
+    """tl_storeh_append_attn_decode writes exactly the rows tl_storeh_append writes (cache bytes
+    identical) and gives bit-identical outputs, flags and first-abort iterations."""
+    w = _small(name, ctx, loops)
+    sep, fus = _dw(w, flag_mix=True, fill=False), _dw(w, flag_mix=True, fill=False)
+    for dw in (sep, fus):  # the same bytes everywhere, so that the whole caches can be compared
+        dw.cache.codes.fill_(0x5A)
+        if dw.cache.scales is not None:
+            dw.cache.scales.fill_(0x5A)
+        dw.fill_context()
+    sep.step()
+    fus.step(fused_append=True)
+    torch.cuda.synchronize()
+    assert torch.equal(sep.cache.codes, fus.cache.codes)
+    if sep.cache.scales is not None:
+        assert torch.equal(sep.cache.scales, fus.cache.scales)
+    a, b = sep.out.cpu().numpy(), fus.out.cpu().numpy()
+    assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+    assert torch.equal(sep.flags, fus.flags) and torch.equal(sep.first, fus.first)
+    # and against the oracle, for one active lane per iteration
+    for it in range(w.L_max):
+        bs = [bb for bb in range(w.B) if it < w.loops[bb]]
+        if bs:
+            _assert_close(b[it, bs[-1]], _oracle_lane(w, it, bs[-1]), f"{name} fused lane {bs[-1]} it {it}")
