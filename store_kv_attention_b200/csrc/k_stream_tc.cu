@@ -11,7 +11,7 @@
 //   scores  S[128 x N_S]   = H . QT^T   M=128 rows, K=d       A = H from TMEM, B = QT (smem)
 //   P.V     U^T[d x N_P]  += H^T . P    M=128 d-values, K=rows A = H (smem, MN-major), B = P (smem)
 // U^T accumulates in TMEM over the whole split; the (m, l, U) partial goes to
-// the workspace and is merged exactly by the epilogue kernel.
+// the workspace and is merged exactly by oproj_kernel (k_proj_tc.cu).
 //
 // Warp roles (640 threads): warp 0 = TMA producer of the score-side ring (and
 // the query image); warp 1 = score-MMA issuer (and TMEM owner); warp 2 = P.V-MMA
@@ -27,12 +27,19 @@
 // Each group reads the codes of a tile through its own TMA ring; the second
 // read of a tile (P.V) finds it in L2.  The online softmax runs in base 2 and
 // each split writes its partial (m, l, U) at the end.
-// The absorbed query arrives as a ready-made fp16 operand image (written by the
-// prologue) through bulk copies.
+// The absorbed query arrives as a ready-made fp16 operand image (written by
+// qproj_kernel) through bulk copies.
 //
 // Codes tiles arrive in 16 KB slots (128 rows x 128 bytes, 128-byte swizzle)
 // loaded by TMA; every row of a slot is read by its own thread, conflict-free
-// thanks to the swizzle.
+// thanks to the swizzle.  Each ring is split into one sub-ring per set of consumers
+// reading the same chunks (so every consumer sees every phase of its slots in order),
+// and a slot is released only once the values read from it have been consumed.
+//
+// The grid is (lane, split) with lanes fastest, so every lane's full-length splits are
+// scheduled before any lane's short last split.  The kernel is launched with
+// programmatic dependent launch: it waits for qproj_kernel before its first global
+// access and lets oproj_kernel be scheduled once it holds its TMEM.
 //
 // Precision: dequantised h is fp16 (INT8 keeps the exact integer codes and
 // applies the per-row scale to the scores and to P instead).  When the
