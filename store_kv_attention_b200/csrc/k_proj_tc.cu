@@ -8,10 +8,18 @@
 //   (hd = 64).  Rank k of the cluster computes the K-split k of those rows into TMEM; the
 //   splits are reduced through distributed shared memory (rank k sums rows of its own
 //   share over all ranks, in rank order, into its own copy of the fp16 hi/lo B operand of
-//   the second GEMM, then every rank pulls the others' rows), whose A operand (W_k^T,
-//   read MN-major) was prefetched by TMA at kernel start.  Each rank then computes its
-//   share of the (head, 128-column block) items of qt and writes the streaming kernel's
-//   absorbed-query operand image directly.
+//   the second GEMM, then every rank pulls the others' rows).  The A operand of that GEMM
+//   (W_k^T, read MN-major) is loaded by TMA as soon as the first GEMM's operands are dead.
+//   Each rank then computes its share of the (head, 128-column block) items of qt and
+//   writes the streaming kernel's absorbed-query operand image directly.  With the fused
+//   append, each CTA also quantises the new token's row of some lanes into the cache
+//   (append_row.cuh) while its first weight tiles load.
+//
+// oproj (one launch):  u_j = sum_s w_s U_sj (the exact merge of the splits), out_j = W_v[j] u_j
+//   Rank k of cluster mb merges the K-slice k of u for the block's heads and every lane into
+//   an fp16 hi/lo B operand, multiplies it by its W_v tiles, and the ranks' partial outputs
+//   are summed in rank order through distributed shared memory.  Each CTA also runs the
+//   FP64 safety check of one lane.
 //
 // Every reduction runs in a fixed order, so a lane's result does not depend on the
 // other lanes of the batch or on scheduling.  All mbarrier waits are bounded; every
