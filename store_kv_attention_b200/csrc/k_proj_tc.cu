@@ -46,18 +46,6 @@ constexpr int kOProjThreads = 256;               // oproj: eight warps (two per 
 constexpr int kTileBytes = 128 * 64 * 2;         // one 128 x 64 fp16 operand tile
 constexpr long long kProjWaitLimit = 4000000000ll;
 
-__device__ __forceinline__ void tma_2d(void* dst, const void* tmap, int32_t x, int32_t y, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
-          smem_addr(dst)),
-      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_addr(bar))
-      : "memory");
-}
-__device__ __forceinline__ bool elect_one() {
-  uint32_t pred;
-  asm volatile("{\n .reg .pred p;\n elect.sync _|p, 0xffffffff;\n selp.u32 %0, 1, 0, p;\n}\n" : "=r"(pred));
-  return pred != 0;
-}
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return p + ((1024 - (smem_addr(p) & 1023)) & 1023);
 }
@@ -177,8 +165,8 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     mbar_expect_tx(&bar_ld1, (uint32_t)lay.nk1 * (kTileBytes + nb * 128));
     for (int i = 0; i < lay.nk1; ++i) {
       const int x = k * lay.KS + 64 * i;
-      tma_2d(a1 + i * kTileBytes, &tmWq, x, mb * 128, &bar_ld1);
-      tma_2d(b1 + i * nb * 128, &tmH, x, 0, &bar_ld1);  // rows past n_lanes read as zero
+      tma_load_2d(a1 + i * kTileBytes, &tmWq, x, mb * 128, &bar_ld1);
+      tma_load_2d(b1 + i * nb * 128, &tmH, x, 0, &bar_ld1);  // rows past n_lanes read as zero
     }
   }
 
@@ -228,8 +216,8 @@ __global__ void __launch_bounds__(kProjThreads, 1)
           const int j = mb * lay.heads_in_block + h2;
           for (int st = 0; st < lay.kst2; ++st) {
             uint8_t* dst = a2 + ((it - it0) * lay.kst2 + st) * kTileBytes;
-            tma_2d(dst, &tmWk, mc * 128, j * s.hd + 64 * st, &bar_ld2);
-            tma_2d(dst + kTileBytes / 2, &tmWk, mc * 128 + 64, j * s.hd + 64 * st, &bar_ld2);
+            tma_load_2d(dst, &tmWk, mc * 128, j * s.hd + 64 * st, &bar_ld2);
+            tma_load_2d(dst + kTileBytes / 2, &tmWk, mc * 128 + 64, j * s.hd + 64 * st, &bar_ld2);
           }
         }
       }
@@ -499,7 +487,7 @@ __global__ void __launch_bounds__(kOProjThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_expect_tx(&bar_ld, (uint32_t)lay.nk * kTileBytes);
-    for (int i = 0; i < lay.nk; ++i) tma_2d(a + i * kTileBytes, &tmWv, k * lay.KS + 64 * i, mb * 128, &bar_ld);
+    for (int i = 0; i < lay.nk; ++i) tma_load_2d(a + i * kTileBytes, &tmWv, k * lay.KS + 64 * i, mb * 128, &bar_ld);
   }
 
   __shared__ uint64_t act_slot;
