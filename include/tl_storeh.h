@@ -259,6 +259,20 @@ TL_API tl_status tl_storeh_attn_decode_static_ws(const tl_storeh_desc* desc, tl_
 TL_API tl_status tl_storeh_poll_status(void* workspace, size_t workspace_bytes, tl_stream_t stream);
 
 /*
+ * Self-test of the device failure-detection path: enqueues one kernel whose only wait
+ * can never complete (an mbarrier nothing arrives at), bounded by the helper every
+ * kernel of the library uses.  After `limit_cycles` SM clocks it gives up and records
+ * TL_ERR_DEVICE_TIMEOUT in the workspace status word, as a kernel that timed out in
+ * earnest would; tl_storeh_poll_status then returns it and clears the word.  No GPU
+ * fault, trap or hang is involved, and the context stays usable.
+ *   workspace     a decode workspace (only its status word is touched)
+ *   limit_cycles  in (0, 4e9] SM clocks
+ * Errors: TL_ERR_INVALID_ARG, TL_ERR_CUDA.
+ */
+TL_API tl_status tl_storeh_selftest_wait_timeout(void* workspace, size_t workspace_bytes, int64_t limit_cycles,
+                                                 tl_stream_t stream);
+
+/*
  * Measurement hook (optional).  While a tl_profile is installed on the calling
  * thread, every tl_storeh_* call made from that thread counts the kernels it
  * launches in `launches`, and records begin_events[k] / end_events[k]

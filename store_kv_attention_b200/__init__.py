@@ -35,7 +35,7 @@ TL_H_INT4_G64 = 2
 EXPORTS = ["tl_storeh_cache_bytes", "tl_storeh_workspace_bytes", "tl_storeh_append", "tl_storeh_attn_decode",
            "tl_residual_norm_check", "tl_storeh_poll_status", "tl_status_string", "tl_last_error_message",
            "tl_storeh_abi_version", "tl_set_profile", "tl_storeh_attn_decode_static_ws",
-           "tl_storeh_append_attn_decode"]
+           "tl_storeh_append_attn_decode", "tl_storeh_selftest_wait_timeout"]
 
 
 class TLError(RuntimeError):
@@ -81,6 +81,8 @@ def _load():
     L.tl_storeh_append_attn_decode.argtypes = L.tl_storeh_attn_decode.argtypes
     L.tl_residual_norm_check.argtypes = [vp, i32, i32, f32, i32, vp, vp, vp, vp, vp]
     L.tl_storeh_poll_status.argtypes = [vp, sz, vp]
+    L.tl_storeh_selftest_wait_timeout.argtypes = [vp, sz, ctypes.c_int64, vp]
+    L.tl_storeh_selftest_wait_timeout.restype = ctypes.c_int
     for f in ("tl_storeh_cache_bytes", "tl_storeh_workspace_bytes", "tl_storeh_append", "tl_storeh_attn_decode",
               "tl_storeh_append_attn_decode", "tl_residual_norm_check", "tl_storeh_poll_status"):
         getattr(L, f).restype = ctypes.c_int
@@ -218,6 +220,13 @@ def residual_norm_check(residual, threshold: float, it: int, loops, abort_flags,
 def poll_status(cache: StoreHCache, stream=None) -> int:
     """Synchronise and return (and clear) the device status of the cache's workspace."""
     return _load().tl_storeh_poll_status(cache.workspace.data_ptr(), cache.ws_bytes, _stream(stream))
+
+
+def selftest_wait_timeout(cache: StoreHCache, limit_cycles: int, stream=None) -> None:
+    """Enqueue the self-test of the timeout path: a kernel whose only wait cannot complete gives
+    up after limit_cycles SM clocks and records TL_ERR_DEVICE_TIMEOUT in the workspace."""
+    _check(_load().tl_storeh_selftest_wait_timeout(cache.workspace.data_ptr(), cache.ws_bytes, int(limit_cycles),
+                                                   _stream(stream)), "tl_storeh_selftest_wait_timeout")
 
 
 class ProfileHook:

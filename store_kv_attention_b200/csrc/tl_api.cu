@@ -228,6 +228,17 @@ tl_status tl_storeh_append_attn_decode(const tl_storeh_desc* desc, tl_storeh_cac
   return decode_impl(desc, cache, iter, loops, ctx_len, h_new, W_q, W_k, W_v, out, residual, threshold, abort_flags, first_abort_iter, norms_out, workspace, workspace_bytes, n_lanes, stream, true);
 }
 
+tl_status tl_storeh_selftest_wait_timeout(void* workspace, size_t workspace_bytes, int64_t limit_cycles,
+                                          tl_stream_t stream) {
+  if (!workspace || workspace_bytes < 256) return fail(TL_ERR_INVALID_ARG, "workspace is NULL or too small");
+  if (!aligned(workspace, 256)) return fail(TL_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (limit_cycles <= 0 || limit_cycles > (int64_t)4000000000ll)
+    return fail(TL_ERR_INVALID_ARG, "limit_cycles %lld outside (0, 4e9]", (long long)limit_cycles);
+  cudaError_t e = tl::launch_wait_selftest((uint32_t*)workspace, (long long)limit_cycles, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "tl_storeh_selftest_wait_timeout launch");
+  return TL_OK;
+}
+
 tl_status tl_storeh_poll_status(void* workspace, size_t workspace_bytes, tl_stream_t stream) {
   if (!workspace || workspace_bytes < 256) return fail(TL_ERR_INVALID_ARG, "workspace is NULL or too small");
   cudaStream_t cs = (cudaStream_t)stream;

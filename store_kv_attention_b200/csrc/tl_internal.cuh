@@ -177,5 +177,7 @@ int proj_cluster(int d);
 bool make_tmap_f16(void* tmap, const void* base, uint64_t rows, uint64_t cols, uint64_t pitch_elems,
                    uint32_t box_cols, uint32_t box_rows);
 cudaError_t launch_stream(const DecodeArgs& a, cudaStream_t st);
+// Self-test of the timeout path: one wait that cannot complete, bounded by limit_cycles (k_selftest.cu).
+cudaError_t launch_wait_selftest(uint32_t* status, long long limit_cycles, cudaStream_t st);
 
 }  // namespace tl

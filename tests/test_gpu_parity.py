@@ -347,3 +347,20 @@ def test_fused_append_equals_separate_calls(name, ctx, loops):
         bs = [bb for bb in range(w.B) if it < w.loops[bb]]
         if bs:
             _assert_close(b[it, bs[-1]], _oracle_lane(w, it, bs[-1]), f"{name} fused lane {bs[-1]} it {it}")
+
+
+def test_device_timeout_is_reported_and_cleared():
+    """The failure-detection path, without a GPU fault: a kernel's wait that cannot complete
+    gives up after its bound, the status word reports TL_ERR_DEVICE_TIMEOUT once (then it is
+    cleared), and the library keeps working afterwards."""
+    import store_kv_attention_b200 as tl
+    w = get_workload("tiny_fp16")
+    dw = _dw(w)
+    tl.selftest_wait_timeout(dw.cache, 2_000_000)  # about 1 ms of SM clocks
+    assert tl.poll_status(dw.cache) == tl.TL_ERR_DEVICE_TIMEOUT
+    assert tl.poll_status(dw.cache) == tl.TL_OK
+    dw.step()
+    torch.cuda.synchronize()
+    assert tl.poll_status(dw.cache) == tl.TL_OK
+    out = dw.out.cpu().numpy()
+    _assert_close(out[0, 0], _oracle_lane(w, 0, 0), "after the timeout self-test")
