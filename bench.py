@@ -16,6 +16,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import re
 import math
 import os
 import statistics
@@ -148,12 +149,21 @@ def load_peaks():
 
 
 def kernel_source_sha():
+    """Hash of the streaming kernel's translation unit: k_stream_tc.cu and every header it
+    pulls in with #include "...", from the package sources or include/."""
+    dirs = [os.path.join(ROOT, "store_kv_attention_b200", "csrc"), os.path.join(ROOT, "include")]
+    seen, todo = {}, ["k_stream_tc.cu"]
+    while todo:
+        fn = todo.pop()
+        if fn in seen:
+            continue
+        path = next(os.path.join(d, fn) for d in dirs if os.path.exists(os.path.join(d, fn)))
+        with open(path, "rb") as f:
+            seen[fn] = f.read()
+        todo += re.findall(r'^\s*#\s*include\s+"([^"]+)"', seen[fn].decode(), flags=re.M)
     h = hashlib.sha256()
-    src = os.path.join(ROOT, "store_kv_attention_b200", "csrc")
-    for fn in sorted(os.listdir(src)):
-        if fn.endswith((".cu", ".cuh")):
-            with open(os.path.join(src, fn), "rb") as f:
-                h.update(fn.encode() + f.read())
+    for fn in sorted(seen):
+        h.update(fn.encode() + seen[fn])
     return h.hexdigest()[:16]
 
 

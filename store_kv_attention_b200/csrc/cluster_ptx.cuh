@@ -18,6 +18,9 @@ __device__ __forceinline__ uint32_t cluster_rank() {
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
+// The two halves of cluster_sync, for work that can run between them.
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 // Shared::cluster address of `smem_cta_addr` (a shared::cta address) in CTA `rank` of the cluster.
 __device__ __forceinline__ uint32_t dsmem_addr(uint32_t smem_cta_addr, uint32_t rank) {
   uint32_t r;
@@ -31,6 +34,11 @@ __device__ __forceinline__ float4 dsmem_ld_f4(uint32_t cluster_addr) {
                : "r"(cluster_addr)
                : "memory");
   return v;
+}
+__device__ __forceinline__ void dsmem_st_f4(uint32_t cluster_addr, float4 v) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1,%2,%3,%4};" ::"r"(cluster_addr), "f"(v.x), "f"(v.y), "f"(v.z),
+               "f"(v.w)
+               : "memory");
 }
 __device__ __forceinline__ void dsmem_st_b16(uint32_t cluster_addr, __half v) {
   asm volatile("st.shared::cluster.b16 [%0], %1;" ::"r"(cluster_addr), "h"(__half_as_ushort(v)) : "memory");

@@ -8,7 +8,7 @@
 //   (hd = 64).  Rank k of the cluster computes the K-split k of those rows into TMEM; the
 //   splits are reduced through distributed shared memory (rank k sums rows of its own
 //   share over all ranks, in rank order, into its own copy of the fp16 hi/lo B operand of
-//   the second GEMM, then every rank pulls the others' rows).  The A operand of that GEMM
+//   the second GEMM, then pushes those rows into the other ranks' copies).  The A operand of that GEMM
 //   (W_k^T, read MN-major) is loaded by TMA as soon as the first GEMM's operands are dead.
 //   Each rank then computes its share of the (head, 128-column block) items of qt and
 //   writes the streaming kernel's absorbed-query operand image directly.  With the fused
@@ -23,7 +23,7 @@
 //
 // Every reduction runs in a fixed order, so a lane's result does not depend on the
 // other lanes of the batch or on scheduling.  All mbarrier waits are bounded; every
-// thread reaches all three cluster barriers whatever happened before them.
+// thread reaches both cluster barriers of its kernel whatever happened before them.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <math_constants.h>
@@ -234,7 +234,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     }
   }
   tc_fence_before();
-  cluster_sync();  // 1: every rank's partial is in place
+  cluster_arrive();  // 1: this rank's partial is in place
 
   // ---------------------------------------------------------------- reduce the K splits through DSMEM
   // Rank k owns rows [k * 128/CL, (k+1) * 128/CL): it sums them over all ranks in rank order
@@ -249,6 +249,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   __shared__ uint64_t act_slot;
   const uint64_t act = active_mask(s, p.iter, p.loops, p.ctx_len, p.n_lanes, &act_slot);
   const int rpr = 128 / CL;
+  cluster_wait();  // 1: every rank's partial is in place
   {
     const int nq = nb / 4;
     const uint32_t part_s = smem_addr(part);
@@ -278,34 +279,24 @@ __global__ void __launch_bounds__(kProjThreads, 1)
       }
     }
   }
-  cluster_sync();  // 2: every rank's reduced rows are in its own B operand
+  __syncthreads();  // this rank's rows of the operand are complete in its own copy
   {
-    // pull the other ranks' rows: rows [r0, r0 + rpr) of operand row n are 2 rpr bytes
-    // (rpr/8 16-byte chunks) at the same swizzled offsets in every rank's copy
+    // push them into the other ranks' copies: rows [r0, r0 + rpr) of operand row n are 2 rpr
+    // bytes (rpr/8 16-byte chunks) at the same swizzled offsets in every rank's copy
     const uint32_t b2_s = smem_addr(b2);
     const int chunks = rpr / 8;
     const int per_rank = 2 * nb * chunks;
-    const int total = CL * per_rank;
-    for (int it0p = threadIdx.x; it0p < total; it0p += 4 * kProjThreads) {
-      float4 v[4];
-      uint32_t off[4];
-      bool use[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int it = it0p + u * kProjThreads;
-        const int rk = it / per_rank;
-        use[u] = it < total && rk != k;
-        const int n = (it % per_rank) / chunks, ch = it % chunks;
-        off[u] = kmajor_offset(n, rk * rpr + ch * 8, 2 * nb);  // 16-byte aligned chunk
-        if (use[u]) v[u] = dsmem_ld_f4(dsmem_addr(b2_s + off[u], (uint32_t)rk));
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (use[u]) *reinterpret_cast<float4*>(b2 + off[u]) = v[u];
+    const int total = (CL - 1) * per_rank;
+    for (int it = threadIdx.x; it < total; it += kProjThreads) {
+      const int rk = (k + 1 + it / per_rank) % CL;  // every rank but this one
+      const int n = (it % per_rank) / chunks, ch = it % chunks;
+      const uint32_t off = kmajor_offset(n, k * rpr + ch * 8, 2 * nb);  // 16-byte aligned chunk
+      dsmem_st_f4(dsmem_addr(b2_s + off, (uint32_t)rk), *reinterpret_cast<const float4*>(b2 + off));
     }
   }
   fence_proxy_async_smem();
-  cluster_sync();  // 3: no DSMEM access after this point
+  fence_proxy_async_cluster();
+  cluster_sync();  // 2: every rank's operand is complete; no DSMEM access after this point
 
   // ---------------------------------------------------------------- phase 2: qt = W_k^T q
   // item (h2, mc): head mb * heads_in_block + h2, output columns [128 mc, 128 mc + 128);
@@ -672,7 +663,7 @@ __global__ void __launch_bounds__(kOProjThreads, 1)
       }
     }
   }
-  cluster_sync();  // 2: no rank leaves while its partial may still be read
+  cluster_arrive();  // 2: this rank reads no other rank's partial any more
 
   tc_fence_before();
   __syncthreads();
@@ -681,6 +672,7 @@ __global__ void __launch_bounds__(kOProjThreads, 1)
     tc_fence_after();
     tmem_dealloc(tbase, lay.tmem_cols);
   }
+  cluster_wait();  // 2: no rank leaves while its partial may still be read
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
