@@ -40,9 +40,6 @@ __device__ __forceinline__ void dsmem_st_f4(uint32_t cluster_addr, float4 v) {
                "f"(v.w)
                : "memory");
 }
-__device__ __forceinline__ void dsmem_st_b16(uint32_t cluster_addr, __half v) {
-  asm volatile("st.shared::cluster.b16 [%0], %1;" ::"r"(cluster_addr), "h"(__half_as_ushort(v)) : "memory");
-}
 // Orders this thread's generic-proxy shared-memory writes (local or remote) before later
 // async-proxy reads (tensor-core operands) of the cluster.
 __device__ __forceinline__ void fence_proxy_async_cluster() {
