@@ -4,3 +4,4 @@ Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import this package.  The product library never does.
 """
 from .storeh_oracle import *  # noqa: F401,F403
+from . import delta_oracle  # noqa: F401  (iteration-axis delta cache)

@@ -7,6 +7,7 @@ The C library is compiled in-tree by :func:`build` (gcc, OpenMP).
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 import subprocess
 
@@ -89,6 +90,7 @@ TID_WK = 4
 TID_WV = 5
 TID_RESIDUAL = 6   # residual per (iteration, lane)
 TID_CTX = 7        # per-lane context length draws
+TID_TRAJ = 8       # loop-iteration trajectories of h (iteration-axis delta cache inputs)
 
 ROW_POS_BITS = 20  # positions per (layer, lane) in the row-id space
 ROW_LANES = 256    # lanes per layer in the row-id space
@@ -114,6 +116,29 @@ def h_rows_f16(seed: int, row_ids: np.ndarray, d: int, outlier_p: float = 0.0,
     rid = np.ascontiguousarray(row_ids, dtype=np.uint64).reshape(-1)
     out = np.empty((rid.shape[0], d), dtype=np.float16)
     h_rows_f16_into(out, seed, rid, d, outlier_p, outlier_mul)
+    return out
+
+
+def trajectory_f16(seed: int, n_tokens: int, d: int, L: int, rho_first: float = 0.68,
+                   rho_last: float = 0.04, rho_span: int = 32) -> np.ndarray:
+    """Hidden-state trajectories along the loop iterations, [L+1, n_tokens, d] fp16.
+
+    h^0 ~ N(0, 1); h^l = fp16(h^(l-1) + sigma_l z_l) with z_l ~ N(0, 1) and sigma_l set from
+    |h^(l-1)| so that |h^l - h^(l-1)| / |h^l| is about rho_l, which falls geometrically from rho_first at
+    iteration 1 to rho_last at iteration rho_span: the contraction the pages measure on
+    the 407M / 2B models (0.68 at the first iteration to 0.04 at the 32nd).  A random walk
+    with that step schedule, nothing more; every draw comes from the counter-based normals.
+    """
+    out = np.empty((L + 1, n_tokens, d), dtype=np.float16)
+    for t in range(n_tokens):
+        base = t * (L + 1) * d
+        out[0, t] = normal_f16(seed, TID_TRAJ, base, d)
+        for l in range(1, L + 1):
+            rho = rho_first * (rho_last / rho_first) ** ((l - 1) / max(rho_span - 1, 1))
+            z = normal_f64(seed, TID_TRAJ, base + l * d, d)
+            prev = out[l - 1, t].astype(np.float64)
+            sigma = rho * np.linalg.norm(prev) / math.sqrt(d * (1.0 - rho * rho))
+            out[l, t] = (prev + sigma * z).astype(np.float16)
     return out
 
 
