@@ -1,0 +1,78 @@
+/*
+ * tl_delta.h -- iteration-axis delta cache of h: the write side.
+ *
+ * [Architecture-Exclusive Features, "Iteration-axis delta-KV"; Measured benchmarks,
+ *  "iteration-axis delta-KV: full forward-path PPL A/B"]
+ * Along the loop iterations a token's hidden state h contracts, so the cache keeps, per
+ * token, one fp16 anchor (the state of loop iteration 0) and, for every later iteration i,
+ * an INT8 delta with one fp16 scale per head.  The state of iteration i is rebuilt as
+ *     h^i = anchor + sum_{j=1..i} scale_j[head] * code_j        (FP32 prefix sum)
+ * This header covers the cache layout and the writer; attention over this cache is not
+ * provided yet (the store-h decode calls of tl_storeh.h take store-h caches only).
+ *
+ * Conventions are those of tl_storeh.h: caller-owned device memory, asynchronous on a
+ * stream, host-side validation before any launch (a non-TL_OK return enqueues nothing,
+ * except TL_ERR_CUDA for a failed launch), programmatic dependent launch with stream order
+ * preserved, tl_last_error_message() for details.
+ */
+#ifndef TL_DELTA_H_
+#define TL_DELTA_H_
+
+#include "tl_storeh.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Shape of one delta cache (one loop block).  d_model = n_heads * head_dim, head_dim in
+ * {64, 128}, d_model a multiple of 256 and at most 2048; L_max loop iterations; max_ctx
+ * positions per lane. */
+typedef struct {
+  int32_t d_model, n_heads, head_dim;
+  int32_t L_max;
+  int32_t max_lanes;
+  int32_t max_ctx;
+} tl_delta_desc;
+
+/* Device buffers, caller-allocated, each 256-byte aligned:
+ *   anchor [max_lanes][max_ctx][d_model]          fp16  (state of iteration 0)
+ *   deltas [L_max-1][max_lanes][max_ctx][d_model]  int8  (iteration i >= 1 at index i-1)
+ *   scales [L_max-1][max_lanes][max_ctx][n_heads]  fp16  (one per head, same indexing)
+ * deltas and scales may be NULL when L_max == 1. */
+typedef struct {
+  void* anchor;
+  void* deltas;
+  void* scales;
+} tl_delta_cache;
+
+/* Sizes in bytes of the three buffers for `desc`.
+ * Errors: TL_ERR_INVALID_ARG (NULL pointer, non-positive size), TL_ERR_SHAPE
+ * (d_model != n_heads * head_dim), TL_ERR_UNSUPPORTED (head_dim or d_model outside the
+ * supported set). */
+TL_API tl_status tl_delta_cache_bytes(const tl_delta_desc* desc, size_t* anchor_bytes, size_t* delta_bytes,
+                                      size_t* scale_bytes);
+
+/* Writes the states of loop iteration `iter` of n_rows positions per lane.
+ *   h_rows    device fp16 [n_lanes][n_rows][d_model], 16-byte aligned: h^iter of each row
+ *   start_pos device int32 [n_lanes]: row r of lane b goes to position start_pos[b] + r
+ *   loops     device int32 [n_lanes] or NULL: lane b is skipped when iter >= loops[b]
+ * iter == 0 stores the rows as the anchor.  iter >= 1 first rebuilds h^(iter-1) of each
+ * position from the cache in FP32 (anchor, then iterations 1..iter-1 added in order, each
+ * addition rounded to fp32) and stores dh = h^iter - that rebuild, per head:
+ *   scale = fp16_rne(amax / 127.0f)  (fp32 IEEE division, amax = max |dh| over the head)
+ *   code  = clamp(rne(dh / float(scale)), -127, 127)  (fp32 IEEE division; zero scale ->
+ *           zero codes)
+ * so the rebuild error of iteration i is that of its own delta only.  Iterations of a
+ * position must therefore be written in order.  Rows whose position lies outside
+ * [0, max_ctx) are skipped on the device.
+ * Errors: TL_ERR_INVALID_ARG (NULL or misaligned pointer, bad count), TL_ERR_CAPACITY
+ * (n_lanes > max_lanes, iter outside [0, L_max)), the desc errors above, TL_ERR_CUDA. */
+TL_API tl_status tl_delta_append(const tl_delta_desc* desc, tl_delta_cache cache, int32_t iter, const void* h_rows,
+                                 int32_t n_lanes, int32_t n_rows, const int32_t* start_pos, const int32_t* loops,
+                                 tl_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TL_DELTA_H_ */

@@ -35,7 +35,8 @@ TL_H_INT4_G64 = 2
 EXPORTS = ["tl_storeh_cache_bytes", "tl_storeh_workspace_bytes", "tl_storeh_append", "tl_storeh_attn_decode",
            "tl_residual_norm_check", "tl_storeh_poll_status", "tl_status_string", "tl_last_error_message",
            "tl_storeh_abi_version", "tl_set_profile", "tl_storeh_attn_decode_static_ws",
-           "tl_storeh_append_attn_decode", "tl_storeh_selftest_wait_timeout"]
+           "tl_storeh_append_attn_decode", "tl_storeh_selftest_wait_timeout", "tl_delta_cache_bytes",
+           "tl_delta_append"]
 
 
 class TLError(RuntimeError):
@@ -57,6 +58,15 @@ class Profile(ctypes.Structure):
 
 class Cache(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
+
+
+class DeltaDescC(ctypes.Structure):
+    _fields_ = [("d_model", ctypes.c_int32), ("n_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("L_max", ctypes.c_int32), ("max_lanes", ctypes.c_int32), ("max_ctx", ctypes.c_int32)]
+
+
+class DeltaCacheC(ctypes.Structure):
+    _fields_ = [("anchor", ctypes.c_void_p), ("deltas", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
 
 
 _lib_handle = None
@@ -96,6 +106,10 @@ def _load():
     L.tl_storeh_attn_decode_static_ws.restype = ctypes.c_int
     L.tl_set_profile.argtypes = [P(Profile)]
     L.tl_set_profile.restype = ctypes.c_int
+    L.tl_delta_cache_bytes.argtypes = [P(DeltaDescC), P(sz), P(sz), P(sz)]
+    L.tl_delta_cache_bytes.restype = ctypes.c_int
+    L.tl_delta_append.argtypes = [P(DeltaDescC), DeltaCacheC, i32, vp, i32, i32, vp, vp, vp]
+    L.tl_delta_append.restype = ctypes.c_int
     _lib_handle = L
     return L
 
@@ -174,6 +188,51 @@ class StoreHCache:
 
     def c(self) -> Cache:
         return Cache(self.codes.data_ptr(), self.scales.data_ptr() if self.scales is not None else None)
+
+
+# ---------------------------------------------------------------- iteration-axis delta cache (include/tl_delta.h)
+@dataclasses.dataclass
+class DeltaDesc:
+    d_model: int
+    n_heads: int
+    head_dim: int
+    L_max: int
+    max_lanes: int
+    max_ctx: int
+
+    def c(self) -> DeltaDescC:
+        return DeltaDescC(self.d_model, self.n_heads, self.head_dim, self.L_max, self.max_lanes, self.max_ctx)
+
+
+def delta_cache_bytes(desc: DeltaDesc):
+    a, d, s = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check(_load().tl_delta_cache_bytes(ctypes.byref(desc.c()), ctypes.byref(a), ctypes.byref(d), ctypes.byref(s)),
+           "tl_delta_cache_bytes")
+    return a.value, d.value, s.value
+
+
+class DeltaCache:
+    """Device buffers of one delta cache: anchor fp16 [lanes][ctx][d], deltas int8 and
+    scales fp16 [L_max-1][lanes][ctx][d or n_heads] (torch tensors)."""
+
+    def __init__(self, desc: DeltaDesc, device="cuda"):
+        import torch
+        self.desc = desc
+        ab, db, sb = delta_cache_bytes(desc)
+        self.anchor = torch.empty(ab // 2, dtype=torch.float16, device=device)
+        self.deltas = torch.empty(max(db, 256), dtype=torch.int8, device=device)
+        self.scales = torch.empty(max(sb // 2, 128), dtype=torch.float16, device=device)
+
+    def c(self) -> DeltaCacheC:
+        return DeltaCacheC(self.anchor.data_ptr(), self.deltas.data_ptr(), self.scales.data_ptr())
+
+
+def delta_append(cache: DeltaCache, it: int, h_rows, start_pos, loops=None, stream=None) -> None:
+    """h_rows: fp16 [n_lanes, n_rows, d] (device), the states of loop iteration ``it``;
+    start_pos / loops int32 [n_lanes] (device)."""
+    n_lanes, n_rows = int(h_rows.shape[0]), int(h_rows.shape[1])
+    _check(_load().tl_delta_append(ctypes.byref(cache.desc.c()), cache.c(), it, _ptr(h_rows), n_lanes, n_rows,
+                                   _ptr(start_pos), _ptr(loops), _stream(stream)), "tl_delta_append")
 
 
 def append(cache: StoreHCache, layer: int, h_rows, start_pos, row_count=None, loops=None, stream=None) -> None:

@@ -4,6 +4,8 @@
 #include <stdio.h>
 #include <string.h>
 
+#include "delta_internal.cuh"
+#include "tl_delta.h"
 #include "tl_internal.cuh"
 
 namespace {
@@ -41,6 +43,23 @@ tl_status check_desc(const tl_storeh_desc* d, tl::Shape* s) {
   if ((int64_t)(d->n_pre + d->L_max) * d->max_lanes * d->max_ctx > ((int64_t)1 << 40))
     return fail(TL_ERR_CAPACITY, "cache has too many rows");
   *s = tl::Shape{d->d_model, d->n_heads, d->head_dim, d->n_pre, d->L_max, d->max_lanes, d->max_ctx, d->fmt};
+  return TL_OK;
+}
+
+// Validates a delta-cache descriptor (include/tl_delta.h).
+tl_status check_delta_desc(const tl_delta_desc* d, tl::DeltaShape* s) {
+  if (!d) return fail(TL_ERR_INVALID_ARG, "desc is NULL");
+  if (d->d_model <= 0 || d->n_heads <= 0 || d->head_dim <= 0 || d->L_max <= 0 || d->max_lanes <= 0 ||
+      d->max_ctx <= 0)
+    return fail(TL_ERR_INVALID_ARG, "desc has a non-positive size");
+  if ((int64_t)d->n_heads * d->head_dim != d->d_model)
+    return fail(TL_ERR_SHAPE, "d_model %d != n_heads %d * head_dim %d", d->d_model, d->n_heads, d->head_dim);
+  if (d->head_dim != 64 && d->head_dim != 128) return fail(TL_ERR_UNSUPPORTED, "head_dim %d not in {64, 128}", d->head_dim);
+  if (d->d_model % 256 != 0 || d->d_model > 2048)
+    return fail(TL_ERR_UNSUPPORTED, "d_model %d must be a multiple of 256 and at most 2048", d->d_model);
+  if ((int64_t)d->L_max * d->max_lanes * d->max_ctx > ((int64_t)1 << 40))
+    return fail(TL_ERR_CAPACITY, "cache has too many rows");
+  *s = tl::DeltaShape{d->d_model, d->n_heads, d->head_dim, d->L_max, d->max_lanes, d->max_ctx};
   return TL_OK;
 }
 
@@ -148,6 +167,42 @@ tl_status tl_storeh_append(const tl_storeh_desc* desc, tl_storeh_cache cache, in
   cudaError_t e = tl::launch_append(s, cache.codes, cache.scales, layer, (const __half*)h_rows, n_lanes, n_rows,
                                     start_pos, row_count, loops, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "tl_storeh_append launch");
+  return TL_OK;
+}
+
+tl_status tl_delta_cache_bytes(const tl_delta_desc* desc, size_t* anchor_bytes, size_t* delta_bytes,
+                               size_t* scale_bytes) {
+  tl::DeltaShape s{};
+  tl_status st = check_delta_desc(desc, &s);
+  if (st != TL_OK) return st;
+  if (!anchor_bytes || !delta_bytes || !scale_bytes) return fail(TL_ERR_INVALID_ARG, "output pointer is NULL");
+  const size_t rows = (size_t)s.max_lanes * s.max_ctx;
+  *anchor_bytes = rows * s.d * 2;
+  *delta_bytes = (size_t)(s.L_max - 1) * rows * s.d;
+  *scale_bytes = (size_t)(s.L_max - 1) * rows * s.H * 2;
+  return TL_OK;
+}
+
+tl_status tl_delta_append(const tl_delta_desc* desc, tl_delta_cache cache, int32_t iter, const void* h_rows,
+                          int32_t n_lanes, int32_t n_rows, const int32_t* start_pos, const int32_t* loops,
+                          tl_stream_t stream) {
+  tl::DeltaShape s{};
+  tl_status st = check_delta_desc(desc, &s);
+  if (st != TL_OK) return st;
+  if (!cache.anchor || (s.L_max > 1 && (!cache.deltas || !cache.scales)))
+    return fail(TL_ERR_INVALID_ARG, "cache.anchor / deltas / scales is NULL");
+  if (!aligned(cache.anchor, 256) || (cache.deltas && !aligned(cache.deltas, 256)) ||
+      (cache.scales && !aligned(cache.scales, 256)))
+    return fail(TL_ERR_INVALID_ARG, "cache buffers must be 256-byte aligned");
+  if (!h_rows || !start_pos) return fail(TL_ERR_INVALID_ARG, "h_rows / start_pos is NULL");
+  if (!aligned(h_rows, 16)) return fail(TL_ERR_INVALID_ARG, "h_rows must be 16-byte aligned");
+  if (n_lanes <= 0 || n_rows < 0) return fail(TL_ERR_INVALID_ARG, "n_lanes %d / n_rows %d", n_lanes, n_rows);
+  if (n_lanes > s.max_lanes) return fail(TL_ERR_CAPACITY, "n_lanes %d > max_lanes %d", n_lanes, s.max_lanes);
+  if (iter < 0 || iter >= s.L_max) return fail(TL_ERR_CAPACITY, "iter %d outside [0, %d)", iter, s.L_max);
+  if (n_rows == 0) return TL_OK;
+  cudaError_t e = tl::launch_delta_append(s, cache.anchor, cache.deltas, cache.scales, iter, (const __half*)h_rows,
+                                          n_lanes, n_rows, start_pos, loops, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "tl_delta_append launch");
   return TL_OK;
 }
 

@@ -107,3 +107,44 @@ def test_calls_rejected_before_launch(tl):
     assert L.tl_residual_norm_check(fake, 1, 8, float("nan"), 0, None, fake, fake, None, None) == tl.TL_ERR_INVALID_ARG
     assert b"threshold" in L.tl_last_error_message()
     assert L.tl_status_string(tl.TL_ERR_DEVICE_TIMEOUT).startswith(b"TL_ERR_DEVICE_TIMEOUT")
+
+
+# --------------------------------------------------------------------------- delta cache (tl_delta.h)
+def test_delta_cache_bytes_match_layout(tl):
+    a, d, s = tl.delta_cache_bytes(tl.DeltaDesc(2048, 16, 128, 8, 32, 4097))
+    rows = 32 * 4097
+    assert (a, d, s) == (rows * 2048 * 2, 7 * rows * 2048, 7 * rows * 16 * 2)
+    assert tl.delta_cache_bytes(tl.DeltaDesc(256, 4, 64, 1, 2, 10)) == (2 * 10 * 256 * 2, 0, 0)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(n_heads=15), 2),
+    (dict(head_dim=96, n_heads=16, d_model=1536), 4),
+    (dict(d_model=4096, n_heads=32), 4),
+    (dict(L_max=0), 1),
+    (dict(max_ctx=0), 1),
+])
+def test_delta_desc_validation(tl, kw, status):
+    base = dict(d_model=2048, n_heads=16, head_dim=128, L_max=8, max_lanes=32, max_ctx=4097)
+    base.update(kw)
+    with pytest.raises(tl.TLError) as e:
+        tl.delta_cache_bytes(tl.DeltaDesc(**base))
+    assert e.value.status == status
+
+
+def test_delta_append_rejected_before_launch(tl):
+    L = tl.lib
+    d = tl.DeltaDesc(2048, 16, 128, 4, 2, 64).c()
+    fake = ctypes.c_void_p(1 << 20)
+    cache = tl.DeltaCacheC(1 << 20, 1 << 21, 1 << 22)
+    assert L.tl_delta_append(None, cache, 0, fake, 1, 1, fake, None, None) == tl.TL_ERR_INVALID_ARG
+    assert L.tl_delta_append(ctypes.byref(d), cache, 4, fake, 1, 1, fake, None, None) == tl.TL_ERR_CAPACITY
+    assert L.tl_delta_append(ctypes.byref(d), cache, -1, fake, 1, 1, fake, None, None) == tl.TL_ERR_CAPACITY
+    assert L.tl_delta_append(ctypes.byref(d), cache, 0, fake, 3, 1, fake, None, None) == tl.TL_ERR_CAPACITY
+    bad = tl.DeltaCacheC((1 << 20) + 16, 1 << 21, 1 << 22)
+    assert L.tl_delta_append(ctypes.byref(d), bad, 0, fake, 1, 1, fake, None, None) == tl.TL_ERR_INVALID_ARG
+    no_deltas = tl.DeltaCacheC(1 << 20, None, None)
+    assert L.tl_delta_append(ctypes.byref(d), no_deltas, 1, fake, 1, 1, fake, None, None) == tl.TL_ERR_INVALID_ARG
+    assert L.tl_delta_append(ctypes.byref(d), cache, 1, ctypes.c_void_p((1 << 20) + 8), 1, 1, fake, None,
+                             None) == tl.TL_ERR_INVALID_ARG
+    assert L.tl_delta_append(ctypes.byref(d), cache, 0, fake, 1, 0, fake, None, None) == tl.TL_OK
