@@ -1,5 +1,5 @@
 /*
- * tl_delta.h -- iteration-axis delta cache of h: the write side.
+ * tl_delta.h -- iteration-axis delta cache of h: layout, writer and decode.
  *
  * [Architecture-Exclusive Features, "Iteration-axis delta-KV"; Measured benchmarks,
  *  "iteration-axis delta-KV: full forward-path PPL A/B"]
@@ -7,8 +7,9 @@
  * token, one fp16 anchor (the state of loop iteration 0) and, for every later iteration i,
  * an INT8 delta with one fp16 scale per head.  The state of iteration i is rebuilt as
  *     h^i = anchor + sum_{j=1..i} scale_j[head] * code_j        (FP32 prefix sum)
- * This header covers the cache layout and the writer; attention over this cache is not
- * provided yet (the store-h decode calls of tl_storeh.h take store-h caches only).
+ * This header covers the cache layout, the writer, and a decode over the cache: the new
+ * token's state is written, the attended rows are rebuilt, and the store-h FP16 decode
+ * kernels run over the rebuilt rows (tl_delta_attn_decode).
  *
  * Conventions are those of tl_storeh.h: caller-owned device memory, asynchronous on a
  * stream, host-side validation before any launch (a non-TL_OK return enqueues nothing,
@@ -70,6 +71,34 @@ TL_API tl_status tl_delta_cache_bytes(const tl_delta_desc* desc, size_t* anchor_
 TL_API tl_status tl_delta_append(const tl_delta_desc* desc, tl_delta_cache cache, int32_t iter, const void* h_rows,
                                  int32_t n_lanes, int32_t n_rows, const int32_t* start_pos, const int32_t* loops,
                                  tl_stream_t stream);
+
+/* Workspace bytes of tl_delta_attn_decode for n_lanes lanes: the store-h decode workspace
+ * (status word first) plus n_lanes x max_ctx x d_model fp16 rows for the rebuilt states.
+ * Errors: the desc errors, TL_ERR_INVALID_ARG (n_lanes <= 0, NULL), TL_ERR_CAPACITY
+ * (n_lanes > max_lanes), TL_ERR_UNSUPPORTED (n_lanes > 64, n_heads > 16, max_ctx > 65536). */
+TL_API tl_status tl_delta_workspace_bytes(const tl_delta_desc* desc, int32_t n_lanes, size_t* bytes);
+
+/* Decode attention of loop iteration `iter` over the delta cache, one new token per lane.
+ * Arguments as for tl_storeh_append_attn_decode (tl_storeh.h): loops / ctx_len device int32
+ * [n_lanes]; h_new fp16 [n_lanes][d] = the new token's state of iteration iter; W_q, W_k, W_v
+ * fp16 [d][d]; out fp32 [n_lanes][d]; the optional safety check (residual fp32 [n_lanes][d],
+ * threshold, abort_flags, first_abort_iter, norms_out); workspace of
+ * tl_delta_workspace_bytes bytes, 256-byte aligned, its first 256 bytes zeroed once.
+ * For every lane with iter < loops[b] (a lane whose loops / ctx_len are out of range is
+ * skipped and recorded; tl_storeh_poll_status on this workspace reports it):
+ *   1. h_new is written as the state of iteration iter at position ctx_len[b], exactly as
+ *      tl_delta_append does;
+ *   2. h^iter of positions 0..ctx_len[b] is rebuilt (FP32 prefix sum, rounded to fp16);
+ *   3. q = W_q h_new attends those rows with K = W_k h, V = W_v h (the store-h decode);
+ *   4. with a residual, the safety check of iteration iter runs as in tl_residual_norm_check.
+ * Other lanes' out rows are left unwritten.  Errors: as tl_storeh_attn_decode, plus the
+ * desc errors above. */
+TL_API tl_status tl_delta_attn_decode(const tl_delta_desc* desc, tl_delta_cache cache, int32_t iter,
+                                      const int32_t* loops, const int32_t* ctx_len, const void* h_new,
+                                      const void* W_q, const void* W_k, const void* W_v, float* out,
+                                      const float* residual, float threshold, uint8_t* abort_flags,
+                                      int32_t* first_abort_iter, float* norms_out, void* workspace,
+                                      size_t workspace_bytes, int32_t n_lanes, tl_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -36,7 +36,7 @@ EXPORTS = ["tl_storeh_cache_bytes", "tl_storeh_workspace_bytes", "tl_storeh_appe
            "tl_residual_norm_check", "tl_storeh_poll_status", "tl_status_string", "tl_last_error_message",
            "tl_storeh_abi_version", "tl_set_profile", "tl_storeh_attn_decode_static_ws",
            "tl_storeh_append_attn_decode", "tl_storeh_selftest_wait_timeout", "tl_delta_cache_bytes",
-           "tl_delta_append"]
+           "tl_delta_append", "tl_delta_workspace_bytes", "tl_delta_attn_decode"]
 
 
 class TLError(RuntimeError):
@@ -110,6 +110,11 @@ def _load():
     L.tl_delta_cache_bytes.restype = ctypes.c_int
     L.tl_delta_append.argtypes = [P(DeltaDescC), DeltaCacheC, i32, vp, i32, i32, vp, vp, vp]
     L.tl_delta_append.restype = ctypes.c_int
+    L.tl_delta_workspace_bytes.argtypes = [P(DeltaDescC), i32, P(sz)]
+    L.tl_delta_workspace_bytes.restype = ctypes.c_int
+    L.tl_delta_attn_decode.argtypes = [P(DeltaDescC), DeltaCacheC, i32, vp, vp, vp, vp, vp, vp, vp, vp, f32, vp, vp,
+                                       vp, vp, sz, i32, vp]
+    L.tl_delta_attn_decode.restype = ctypes.c_int
     _lib_handle = L
     return L
 
@@ -211,17 +216,27 @@ def delta_cache_bytes(desc: DeltaDesc):
     return a.value, d.value, s.value
 
 
+def delta_workspace_bytes(desc: DeltaDesc, n_lanes: int) -> int:
+    b = ctypes.c_size_t()
+    _check(_load().tl_delta_workspace_bytes(ctypes.byref(desc.c()), n_lanes, ctypes.byref(b)),
+           "tl_delta_workspace_bytes")
+    return b.value
+
+
 class DeltaCache:
     """Device buffers of one delta cache: anchor fp16 [lanes][ctx][d], deltas int8 and
-    scales fp16 [L_max-1][lanes][ctx][d or n_heads] (torch tensors)."""
+    scales fp16 [L_max-1][lanes][ctx][d or n_heads] (torch tensors); with ``n_lanes`` also a
+    zeroed decode workspace for that many lanes."""
 
-    def __init__(self, desc: DeltaDesc, device="cuda"):
+    def __init__(self, desc: DeltaDesc, device="cuda", n_lanes: Optional[int] = None):
         import torch
         self.desc = desc
         ab, db, sb = delta_cache_bytes(desc)
         self.anchor = torch.empty(ab // 2, dtype=torch.float16, device=device)
         self.deltas = torch.empty(max(db, 256), dtype=torch.int8, device=device)
         self.scales = torch.empty(max(sb // 2, 128), dtype=torch.float16, device=device)
+        self.ws_bytes = delta_workspace_bytes(desc, n_lanes) if n_lanes else 0
+        self.workspace = torch.zeros(self.ws_bytes, dtype=torch.uint8, device=device) if n_lanes else None
 
     def c(self) -> DeltaCacheC:
         return DeltaCacheC(self.anchor.data_ptr(), self.deltas.data_ptr(), self.scales.data_ptr())
@@ -233,6 +248,19 @@ def delta_append(cache: DeltaCache, it: int, h_rows, start_pos, loops=None, stre
     n_lanes, n_rows = int(h_rows.shape[0]), int(h_rows.shape[1])
     _check(_load().tl_delta_append(ctypes.byref(cache.desc.c()), cache.c(), it, _ptr(h_rows), n_lanes, n_rows,
                                    _ptr(start_pos), _ptr(loops), _stream(stream)), "tl_delta_append")
+
+
+def delta_attn_decode(cache: DeltaCache, it: int, loops, ctx_len, h_new, W_q, W_k, W_v, out, residual=None,
+                      threshold: float = 0.0, abort_flags=None, first_abort_iter=None, norms_out=None,
+                      stream=None) -> None:
+    """tl_delta_attn_decode: writes h_new as iteration ``it`` of each active lane's new token,
+    then attends the rebuilt rows (the cache needs a workspace: DeltaCache(..., n_lanes=N))."""
+    n_lanes = int(h_new.shape[0])
+    _check(_load().tl_delta_attn_decode(ctypes.byref(cache.desc.c()), cache.c(), it, _ptr(loops), _ptr(ctx_len),
+                                        _ptr(h_new), _ptr(W_q), _ptr(W_k), _ptr(W_v), _ptr(out), _ptr(residual),
+                                        float(threshold), _ptr(abort_flags), _ptr(first_abort_iter),
+                                        _ptr(norms_out), _ptr(cache.workspace), cache.ws_bytes, n_lanes,
+                                        _stream(stream)), "tl_delta_attn_decode")
 
 
 def append(cache: StoreHCache, layer: int, h_rows, start_pos, row_count=None, loops=None, stream=None) -> None:
@@ -276,8 +304,9 @@ def residual_norm_check(residual, threshold: float, it: int, loops, abort_flags,
            "tl_residual_norm_check")
 
 
-def poll_status(cache: StoreHCache, stream=None) -> int:
-    """Synchronise and return (and clear) the device status of the cache's workspace."""
+def poll_status(cache, stream=None) -> int:
+    """Synchronise and return (and clear) the device status of the cache's workspace
+    (a StoreHCache, or a DeltaCache made with n_lanes)."""
     return _load().tl_storeh_poll_status(cache.workspace.data_ptr(), cache.ws_bytes, _stream(stream))
 
 

@@ -17,4 +17,14 @@ cudaError_t launch_delta_append(const DeltaShape& s, void* anchor, void* deltas,
                                 const __half* h_rows, int n_lanes, int n_rows, const int32_t* start_pos,
                                 const int32_t* loops, cudaStream_t st);
 
+// One delta decode call (tl_delta_attn_decode): per-lane effective loop counts for the writer
+// and the decode, range violations recorded in *status.
+cudaError_t launch_delta_prep(int iter, int L_max, int max_ctx, int n_lanes, const int32_t* loops,
+                              const int32_t* ctx_len, int32_t* wloops, int32_t* dloops, uint32_t* status,
+                              cudaStream_t st);
+// h^iter of positions 0..ctx_len[b] of the lanes with dloops[b] = 1 into out [n_lanes][max_ctx][d] fp16.
+cudaError_t launch_delta_rebuild(const DeltaShape& s, const void* anchor, const void* deltas, const void* scales,
+                                 int iter, int n_lanes, const int32_t* ctx_len, const int32_t* dloops, __half* out,
+                                 cudaStream_t st);
+
 }  // namespace tl

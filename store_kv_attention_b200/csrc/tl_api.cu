@@ -63,6 +63,25 @@ tl_status check_delta_desc(const tl_delta_desc* d, tl::DeltaShape* s) {
   return TL_OK;
 }
 
+// A delta decode runs the store-h FP16 decode on a one-layer scratch cache of the rebuilt rows:
+// shape of that cache, and the workspace layout [decode workspace | wloops | dloops | scratch].
+tl::Shape delta_view_shape(const tl::DeltaShape& s, int n_lanes) {
+  return tl::Shape{s.d, s.H, s.hd, 0, 1, n_lanes, s.max_ctx, TL_H_FP16};
+}
+struct DeltaWorkspace {
+  tl::Workspace wl;
+  size_t wloops_off, dloops_off, scratch_off, total;
+};
+DeltaWorkspace delta_workspace(const tl::DeltaShape& s, int n_lanes) {
+  DeltaWorkspace w;
+  w.wl = tl::workspace_layout(delta_view_shape(s, n_lanes), n_lanes);
+  w.wloops_off = tl::align256(w.wl.total);
+  w.dloops_off = w.wloops_off + tl::align256((size_t)n_lanes * 4);
+  w.scratch_off = w.dloops_off + tl::align256((size_t)n_lanes * 4);
+  w.total = w.scratch_off + tl::align256((size_t)n_lanes * s.max_ctx * s.d * 2);
+  return w;
+}
+
 tl_status check_cache(const tl::Shape& s, const tl_storeh_cache& c) {
   if (!c.codes) return fail(TL_ERR_INVALID_ARG, "cache.codes is NULL");
   if (s.fmt != TL_H_FP16 && !c.scales) return fail(TL_ERR_INVALID_ARG, "cache.scales is NULL");
@@ -203,6 +222,82 @@ tl_status tl_delta_append(const tl_delta_desc* desc, tl_delta_cache cache, int32
   cudaError_t e = tl::launch_delta_append(s, cache.anchor, cache.deltas, cache.scales, iter, (const __half*)h_rows,
                                           n_lanes, n_rows, start_pos, loops, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "tl_delta_append launch");
+  return TL_OK;
+}
+
+tl_status tl_delta_workspace_bytes(const tl_delta_desc* desc, int32_t n_lanes, size_t* bytes) {
+  tl::DeltaShape s{};
+  tl_status st = check_delta_desc(desc, &s);
+  if (st != TL_OK) return st;
+  if (!bytes) return fail(TL_ERR_INVALID_ARG, "bytes is NULL");
+  if (n_lanes <= 0) return fail(TL_ERR_INVALID_ARG, "n_lanes %d <= 0", n_lanes);
+  if (n_lanes > s.max_lanes) return fail(TL_ERR_CAPACITY, "n_lanes %d > max_lanes %d", n_lanes, s.max_lanes);
+  if (n_lanes > tl::kMaxGemmLanes)
+    return fail(TL_ERR_UNSUPPORTED, "n_lanes %d > %d lanes per decode call", n_lanes, tl::kMaxGemmLanes);
+  if (s.H > tl::kMaxHeads) return fail(TL_ERR_UNSUPPORTED, "n_heads %d > %d", s.H, tl::kMaxHeads);
+  if (s.max_ctx > tl::kMaxCtx) return fail(TL_ERR_UNSUPPORTED, "max_ctx %d > %d", s.max_ctx, tl::kMaxCtx);
+  *bytes = delta_workspace(s, n_lanes).total;
+  return TL_OK;
+}
+
+tl_status tl_delta_attn_decode(const tl_delta_desc* desc, tl_delta_cache cache, int32_t iter, const int32_t* loops,
+                               const int32_t* ctx_len, const void* h_new, const void* W_q, const void* W_k,
+                               const void* W_v, float* out, const float* residual, float threshold,
+                               uint8_t* abort_flags, int32_t* first_abort_iter, float* norms_out, void* workspace,
+                               size_t workspace_bytes, int32_t n_lanes, tl_stream_t stream) {
+  tl::DeltaShape s{};
+  tl_status st = check_delta_desc(desc, &s);
+  if (st != TL_OK) return st;
+  if (!cache.anchor || (s.L_max > 1 && (!cache.deltas || !cache.scales)))
+    return fail(TL_ERR_INVALID_ARG, "cache.anchor / deltas / scales is NULL");
+  if (!aligned(cache.anchor, 256) || (cache.deltas && !aligned(cache.deltas, 256)) ||
+      (cache.scales && !aligned(cache.scales, 256)))
+    return fail(TL_ERR_INVALID_ARG, "cache buffers must be 256-byte aligned");
+  if (!loops || !ctx_len || !h_new || !W_q || !W_k || !W_v || !out || !workspace)
+    return fail(TL_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (!aligned(h_new, 16) || !aligned(W_q, 16) || !aligned(W_k, 16) || !aligned(W_v, 16) || !aligned(out, 16))
+    return fail(TL_ERR_INVALID_ARG, "h_new, W_q, W_k, W_v and out must be 16-byte aligned");
+  if (!aligned(workspace, 256)) return fail(TL_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (n_lanes <= 0) return fail(TL_ERR_INVALID_ARG, "n_lanes %d <= 0", n_lanes);
+  if (n_lanes > s.max_lanes) return fail(TL_ERR_CAPACITY, "n_lanes %d > max_lanes %d", n_lanes, s.max_lanes);
+  if (iter < 0 || iter >= s.L_max) return fail(TL_ERR_CAPACITY, "iter %d outside [0, L_max=%d)", iter, s.L_max);
+  if (n_lanes > tl::kMaxGemmLanes)
+    return fail(TL_ERR_UNSUPPORTED, "n_lanes %d > %d lanes per decode call", n_lanes, tl::kMaxGemmLanes);
+  if (s.H > tl::kMaxHeads) return fail(TL_ERR_UNSUPPORTED, "n_heads %d > %d", s.H, tl::kMaxHeads);
+  if (s.max_ctx > tl::kMaxCtx) return fail(TL_ERR_UNSUPPORTED, "max_ctx %d > %d", s.max_ctx, tl::kMaxCtx);
+  if (residual && (!abort_flags || !first_abort_iter))
+    return fail(TL_ERR_INVALID_ARG, "residual given without abort_flags / first_abort_iter");
+  if (residual && !(threshold >= 0.0f)) return fail(TL_ERR_INVALID_ARG, "threshold must be a non-negative number");
+  const DeltaWorkspace w = delta_workspace(s, n_lanes);
+  if (workspace_bytes < w.total) return fail(TL_ERR_CAPACITY, "workspace %zu bytes < %zu needed", workspace_bytes, w.total);
+
+  uint8_t* ws = (uint8_t*)workspace;
+  int32_t* wloops = (int32_t*)(ws + w.wloops_off);
+  int32_t* dloops = (int32_t*)(ws + w.dloops_off);
+  __half* scratch = (__half*)(ws + w.scratch_off);
+  cudaStream_t cs = (cudaStream_t)stream;
+  // 1. per-lane checks; 2. the new token's state of this iteration into the delta cache;
+  // 3. h^iter of every attended position into the scratch; 4. the FP16 decode over it;
+  // 5. the safety check with the real iteration
+  cudaError_t e = tl::launch_delta_prep(iter, s.L_max, s.max_ctx, n_lanes, loops, ctx_len, wloops, dloops,
+                                        (uint32_t*)(ws + w.wl.status_off), cs);
+  if (e == cudaSuccess)
+    e = tl::launch_delta_append(s, cache.anchor, cache.deltas, cache.scales, iter, (const __half*)h_new, n_lanes, 1,
+                                ctx_len, wloops, cs);
+  if (e == cudaSuccess)
+    e = tl::launch_delta_rebuild(s, cache.anchor, cache.deltas, cache.scales, iter, n_lanes, ctx_len, dloops, scratch,
+                                 cs);
+  if (e != cudaSuccess) return cuda_fail(e, "delta decode prologue launch");
+  tl::DecodeArgs a{delta_view_shape(s, n_lanes), scratch, nullptr, 0, dloops, ctx_len, (const __half*)h_new,
+                   (const __half*)W_q, (const __half*)W_k, (const __half*)W_v, out, n_lanes, ws, w.wl,
+                   nullptr, 0.0f, nullptr, nullptr, nullptr};
+  e = tl::launch_qproj(a, cs);
+  if (e == cudaSuccess) e = tl::launch_stream(a, cs);
+  if (e == cudaSuccess) e = tl::launch_oproj(a, cs);
+  if (e == cudaSuccess && residual)
+    e = tl::launch_norm_check(residual, n_lanes, s.d, threshold, iter, wloops, abort_flags, first_abort_iter,
+                              norms_out, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "delta decode launch");
   return TL_OK;
 }
 
