@@ -148,3 +148,30 @@ def test_delta_append_rejected_before_launch(tl):
     assert L.tl_delta_append(ctypes.byref(d), cache, 1, ctypes.c_void_p((1 << 20) + 8), 1, 1, fake, None,
                              None) == tl.TL_ERR_INVALID_ARG
     assert L.tl_delta_append(ctypes.byref(d), cache, 0, fake, 1, 0, fake, None, None) == tl.TL_OK
+
+
+def test_delta_workspace_and_decode_rejected_before_launch(tl):
+    desc = tl.DeltaDesc(2048, 16, 128, 4, 4, 1000)
+    ws = tl.delta_workspace_bytes(desc, 2)
+    sdesc = tl.StoreHDesc(2048, 16, 128, n_pre=0, L_max=1, max_lanes=2, max_ctx=1000, fmt=tl.TL_H_FP16)
+    assert ws >= tl.workspace_bytes(sdesc, 2) + 2 * 1000 * 2048 * 2 and ws % 256 == 0
+    with pytest.raises(tl.TLError) as e:
+        tl.delta_workspace_bytes(desc, 5)
+    assert e.value.status == tl.TL_ERR_CAPACITY
+    with pytest.raises(tl.TLError) as e:
+        tl.delta_workspace_bytes(tl.DeltaDesc(2048, 32, 64, 4, 4, 1000), 2)  # 32 heads
+    assert e.value.status == tl.TL_ERR_UNSUPPORTED
+    L = tl.lib
+    d = desc.c()
+    fake = ctypes.c_void_p(1 << 20)
+    cache = tl.DeltaCacheC(1 << 20, 1 << 21, 1 << 22)
+    args = lambda it, n, wsb, ws_ptr=fake, res=None, flags=None: (
+        ctypes.byref(d), cache, it, fake, fake, fake, fake, fake, fake, fake, res, ctypes.c_float(50.0), flags, None,
+        None, ws_ptr, wsb, n, None)
+    assert L.tl_delta_attn_decode(*args(4, 2, ws)) == tl.TL_ERR_CAPACITY          # iter outside [0, L_max)
+    assert L.tl_delta_attn_decode(*args(0, 5, ws)) == tl.TL_ERR_CAPACITY          # lanes beyond the cache
+    assert L.tl_delta_attn_decode(*args(0, 2, ws - 256)) == tl.TL_ERR_CAPACITY    # workspace too small
+    assert L.tl_delta_attn_decode(*args(0, 2, ws, ws_ptr=ctypes.c_void_p((1 << 20) + 16))) == tl.TL_ERR_INVALID_ARG
+    assert L.tl_delta_attn_decode(*args(0, 2, ws, res=fake)) == tl.TL_ERR_INVALID_ARG  # residual without flags
+    assert L.tl_delta_attn_decode(None, cache, 0, fake, fake, fake, fake, fake, fake, fake, None,
+                                  ctypes.c_float(0.0), None, None, None, fake, ws, 2, None) == tl.TL_ERR_INVALID_ARG
