@@ -5,3 +5,4 @@ Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 """
 from .storeh_oracle import *  # noqa: F401,F403
 from . import delta_oracle  # noqa: F401  (iteration-axis delta cache)
+from . import tree_oracle  # noqa: F401  (tree verification over the cache)
