@@ -92,7 +92,11 @@ TL_API tl_status tl_delta_workspace_bytes(const tl_delta_desc* desc, int32_t n_l
  *   3. q = W_q h_new attends those rows with K = W_k h, V = W_v h (the store-h decode);
  *   4. with a residual, the safety check of iteration iter runs as in tl_residual_norm_check.
  * Other lanes' out rows are left unwritten.  Errors: as tl_storeh_attn_decode, plus the
- * desc errors above. */
+ * desc errors above.
+ * Known accuracy gap of this composition: step 2 rounds the FP32 rebuild to fp16 before
+ * attention, an error the exact rebuild does not have.  At d_model 256 the outputs meet
+ * the store-h bar (max-abs 2e-3, relative L2 1e-3); at d_model 1024 one output element was
+ * measured at max-abs 2.22e-3, above that bar, and d_model 2048 has not been run. */
 TL_API tl_status tl_delta_attn_decode(const tl_delta_desc* desc, tl_delta_cache cache, int32_t iter,
                                       const int32_t* loops, const int32_t* ctx_len, const void* h_new,
                                       const void* W_q, const void* W_k, const void* W_v, float* out,

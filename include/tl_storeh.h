@@ -228,15 +228,22 @@ TL_API tl_status tl_residual_norm_check(const float* residual, int32_t n_lanes, 
  * TL_ERR_CAPACITY before anything is launched.  The call allocates nothing: no
  * cudaMalloc, cudaFree or allocating library routine.
  *
- * The first call on each device looks up the array's device address
- * (cudaGetSymbolAddress) with that device current; make that first call before
- * any stream capture.  All calls in the process share the one array and it
+ * Every call looks up the array's device address (cudaGetSymbolAddress) in the
+ * device and context current at the call.  Under CUDA's default lazy module
+ * loading the array itself is created by the first such lookup on a device, so
+ * the first call on each device is where the 32 MiB are taken and where an
+ * out-of-memory condition shows up (TL_ERR_CUDA): make one warm-up call during
+ * initialisation, and make it before any stream capture.  All calls in the
+ * process share the one array and it
  * keeps the previous call's contents (the call clears the part that must start
  * at zero itself): two calls that may overlap on the GPU — on different streams
  * without an ordering between them — race on it and give wrong results.
  *   status_out  device uint32 or NULL: receives this call's device status word
  *               (bit 0 = a lane's loops/ctx_len was out of range and the lane was
- *               skipped, bit 1 = a bounded device wait gave up).
+ *               skipped, bit 1 = a bounded device wait gave up).  The word lives in
+ *               the built-in array, which the next call clears and which
+ *               tl_storeh_poll_status cannot reach: with status_out == NULL the
+ *               range and timeout reports of this call are discarded.
  */
 TL_API tl_status tl_storeh_attn_decode_static_ws(const tl_storeh_desc* desc, tl_storeh_cache cache, int32_t iter,
                                                  const int32_t* loops, const int32_t* ctx_len, const void* h_new,

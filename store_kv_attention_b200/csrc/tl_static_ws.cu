@@ -12,10 +12,13 @@
 // The array is a file-scope __device__ variable, so every GPU that loads the
 // library holds kStaticScratchBytes of device memory until the process exits.
 // In host code its name only stands in for the symbol; the device address is
-// fetched once per device with cudaGetSymbolAddress and then passed to the
-// kernels like any other workspace pointer.
-#include <mutex>
-
+// looked up with cudaGetSymbolAddress, on the device and context current at the
+// call, on every call (a lookup costs far less than the launches it precedes),
+// and then passed to the kernels like any other workspace pointer.  Looking it up
+// each time keeps the address right after cudaDeviceReset or when another
+// context is current.  With CUDA's lazy module loading the array is only
+// created by the first lookup on a device, so that first call is where an
+// out-of-memory condition shows up (as TL_ERR_CUDA).
 #include "tl_internal.cuh"
 
 namespace {
@@ -24,24 +27,12 @@ constexpr size_t kStaticScratchBytes = 32u << 20;  // 32 MiB
 
 __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of the scratch array on the current device (looked up once per device).
+// Device address of the scratch array in the current context.
 cudaError_t scratch_address(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  void* p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_decode_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_ptr[dev] = p;
-  }
-  *out = g_scratch_ptr[dev];
+  *out = p;
   return cudaSuccess;
 }
 

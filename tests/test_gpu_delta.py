@@ -105,7 +105,7 @@ def _weights(seed, d):
 @pytest.mark.parametrize("d,H,L_max,ctx,max_ctx", [
     (256, 4, 3, [150, 37], 200),
     pytest.param(1024, 16, 3, [500, 64], 600, marks=pytest.mark.xfail(
-        reason="fp16 rounding of the rebuilt rows: max-abs 2.22e-3 > 2e-3 measured", strict=False)),
+        reason="fp16 rounding of the rebuilt rows: max-abs 2.22e-3 > 2e-3 measured", strict=True)),
 ])
 def test_decode_matches_oracle(d, H, L_max, ctx, max_ctx):
     import oracle

@@ -226,34 +226,119 @@ def test_out_of_range_lane_is_skipped_and_reported():
 
 
 # --------------------------------------------------------------------------- decode: full sizes, sampled
+# The benchmarked entry point (tl_storeh_append_attn_decode) at the benchmarked sizes, against
+# the separate append + decode calls on a copy of the same cache (whole cache byte for byte,
+# outputs bit for bit), the oracle's quantiser (every appended row), the oracle's attention
+# (sampled lanes: the forced-abort lanes, the last lane) and the oracle's safety check.
 FULL = [
     ("fp16_407m", [(it, 0) for it in range(8)]),
     ("int8_b16", [(0, 0), (3, 7), (7, 15)]),
-    ("int4_2b", [(0, 0), (4, 1), (7, 31)]),
-    ("int4_mixed", [(0, 0), (3, 15), (10, 20), (31, 47), (15, 33)]),
+    ("int4_2b", [(0, 0), (7, 1), (4, 17), (7, 31)]),
+    ("int4_mixed", [(0, 0), (3, 1), (3, 15), (10, 20), (31, 47), (15, 33)]),
 ]
+
+
+def _new_rows_from_cache(dw, it):
+    """Codes and scales of every lane's row at (layer n_pre + it, position ctx[b]), from the device."""
+    w = dw.w
+    cb = oracle.row_code_bytes(w.fmt, w.d)
+    ns = oracle.row_scale_count(w.fmt, w.d)
+    codes = dw.cache.codes[: w.n_layers * w.B * w.max_ctx * cb].view(w.n_layers, w.B, w.max_ctx, cb)
+    lanes = torch.arange(w.B, device=dw.ctx.device)
+    c = codes[w.n_pre + it, lanes, dw.ctx.long()].cpu().numpy()
+    if ns == 0:
+        return c, None
+    sdt = np.float32 if w.fmt == 1 else np.float16
+    nbytes = w.n_layers * w.B * w.max_ctx * ns * np.dtype(sdt).itemsize
+    sc = dw.cache.scales[:nbytes].view(w.n_layers, w.B, w.max_ctx, ns * np.dtype(sdt).itemsize)
+    return c, sc[w.n_pre + it, lanes, dw.ctx.long()].cpu().numpy().view(sdt)
 
 
 @pytest.mark.parametrize("name,samples", FULL, ids=[f[0] for f in FULL])
 def test_decode_full_size_sampled(name, samples):
     import store_kv_attention_b200 as tl
     w = get_workload(name)
-    dw = _dw(w)
-    dw.step()
-    torch.cuda.synchronize()
-    out = dw.out.cpu().numpy()
+    fus = _dw(w)
+    sep = _dw(w, fill=False)
+    sep.cache.codes.copy_(fus.cache.codes)
+    if fus.cache.scales is not None:
+        sep.cache.scales.copy_(fus.cache.scales)
+    act = np.array([[it < w.loops[b] for b in range(w.B)] for it in range(w.L_max)])
+    # both residual variants: literal (every lane over the threshold) and flag-mix
+    for flag_mix in (False, True):
+        res = torch.stack([torch.from_numpy(w.residual(it, flag_mix)) for it in range(w.L_max)]).cuda()
+        for dw in (fus, sep):
+            dw.residual = res
+            dw.reset_flags()
+            dw.out.fill_(float("nan"))
+        fus.step(fused_append=True)
+        sep.step()
+        torch.cuda.synchronize()
+        assert torch.equal(fus.cache.codes, sep.cache.codes)
+        if fus.cache.scales is not None:
+            assert torch.equal(fus.cache.scales, sep.cache.scales)
+        out = fus.out.cpu().numpy()
+        assert np.array_equal(out.view(np.uint32), sep.out.cpu().numpy().view(np.uint32))
+        assert torch.equal(fus.flags, sep.flags) and torch.equal(fus.first, sep.first)
+        f = np.zeros(w.B, np.uint8)
+        fi = np.full(w.B, -1, np.int32)
+        for it in range(w.L_max):
+            f, fi, _ = oracle.residual_norm_check(w.residual(it, flag_mix), w.threshold, it, np.array(w.loops), f, fi)
+        assert np.array_equal(fus.flags.cpu().numpy(), f) and np.array_equal(fus.first.cpu().numpy(), fi)
+        if flag_mix:
+            assert 0 < f.sum() < w.B
+        # every active (lane, iteration) was written, every inactive one was not
+        assert np.all(np.isfinite(out[act])) and np.all(np.isnan(out[~act]))
+    # the new token's row of every active (lane, iteration), bit-exact with the oracle's quantiser
+    for it in range(w.L_max):
+        bs = [b for b in range(w.B) if act[it, b]]
+        want_c, want_s = oracle.quantize_rows(w.h_new(it)[bs], w.fmt)
+        got_c, got_s = _new_rows_from_cache(fus, it)
+        assert np.array_equal(got_c[bs], want_c), f"{name} codes of iteration {it}"
+        if got_s is not None:
+            assert np.array_equal(got_s[bs].view(np.uint8), want_s.astype(got_s.dtype).view(np.uint8))
     for it, b in samples:
         assert it < w.loops[b]
         _assert_close(out[it, b], _oracle_lane(w, it, b, form="absorbed"), f"{name} lane {b} it {it}")
-    # every active (lane, iteration) was written, every inactive one was not
-    act = np.array([[it < w.loops[b] for b in range(w.B)] for it in range(w.L_max)])
-    assert np.all(np.isfinite(out[act])) and np.all(np.isnan(out[~act]))
-    f = np.zeros(w.B, np.uint8)
-    fi = np.full(w.B, -1, np.int32)
+    assert tl.poll_status(fus.cache) == tl.TL_OK and tl.poll_status(sep.cache) == tl.TL_OK
+
+
+@pytest.mark.parametrize("fmt", [0, 1, 2])
+def test_fused_append_more_lanes_than_ctas(fmt):
+    """d = 256 runs the projection kernel on 8 CTAs, so with 40 lanes the fused append's lane
+    loop makes several trips per CTA."""
+    import dataclasses
+    base = get_workload("tiny_fp16")
+    n = 40
+    ctx = [(53 * b * b + 17 * b) % 700 for b in range(n)]
+    ctx[3], ctx[5] = 0, 1
+    loops = [1 + (b % 3) for b in range(n)]
+    w = dataclasses.replace(base, fmt=fmt, ctx=ctx, loops=loops, L_max=3, name=f"d256_fmt{fmt}_40lanes",
+                            outlier_p=0.01 if fmt == 1 else 0.0, outlier_mul=8.0)
+    sep, fus = _dw(w, flag_mix=True, fill=False), _dw(w, flag_mix=True, fill=False)
+    for dw in (sep, fus):
+        dw.cache.codes.fill_(0x5A)
+        if dw.cache.scales is not None:
+            dw.cache.scales.fill_(0x5A)
+        dw.fill_context()
+    sep.step()
+    fus.step(fused_append=True)
+    torch.cuda.synchronize()
+    assert torch.equal(sep.cache.codes, fus.cache.codes)
+    if sep.cache.scales is not None:
+        assert torch.equal(sep.cache.scales, fus.cache.scales)
+    a = fus.out.cpu().numpy()
+    assert np.array_equal(a.view(np.uint32), sep.out.cpu().numpy().view(np.uint32))
+    assert torch.equal(sep.flags, fus.flags) and torch.equal(sep.first, fus.first)
     for it in range(w.L_max):
-        f, fi, _ = oracle.residual_norm_check(w.residual(it), w.threshold, it, np.array(w.loops), f, fi)
-    assert np.array_equal(dw.flags.cpu().numpy(), f) and np.array_equal(dw.first.cpu().numpy(), fi)
-    assert tl.poll_status(dw.cache) == tl.TL_OK
+        bs = [b for b in range(w.B) if it < w.loops[b]]
+        want_c, want_s = oracle.quantize_rows(w.h_new(it)[bs], w.fmt)
+        got_c, got_s = _new_rows_from_cache(fus, it)
+        assert np.array_equal(got_c[bs], want_c)
+        if got_s is not None:
+            assert np.array_equal(got_s[bs].view(np.uint8), want_s.astype(got_s.dtype).view(np.uint8))
+        for b in (bs[0], bs[len(bs) // 2], bs[-1]):
+            _assert_close(a[it, b], _oracle_lane(w, it, b), f"{w.name} lane {b} it {it}")
 
 
 @pytest.mark.gpu
