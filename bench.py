@@ -40,7 +40,7 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--workload", default=DEFAULT_WORKLOAD)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    p.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the CPU-baseline sample")
+    p.add_argument("--cpu-seconds", type=float, default=20.0, help="budget of the CPU-baseline sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
 
@@ -87,56 +87,73 @@ def workload_config(w, n_gpus, extra=None):
     return cfg
 
 
-def blas_threads():
+def cpu_model():
     try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
-        return max(n) if n else 1
-    except Exception:
-        return os.cpu_count() or 1
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
 
 
 class OracleSample:
-    """A bounded sample of the workload for the CPU oracle: whole (lane, iteration)
-    decodes, each with its lane's resident cache prepared once (not timed)."""
+    """A bounded sample of the workload for the plain C++ FP64 oracle: whole (lane, iteration)
+    decodes -- append of the new row, exact dequantisation, explicit K/V rebuild, softmax,
+    safety check -- each with its lane's cached rows quantised once beforehand (not timed)."""
 
     def __init__(self, w):
         self.w = w
         self.pairs = [(it, b) for it in range(w.L_max) for b in range(w.B) if it < w.loops[b]]
-        self.prepared = []
+        self.prepared = {}
         self.W = [w.weight(k) for k in "qkv"]
 
     def _prepare(self, i):
-        import oracle
-        w = self.w
-        it, b = self.pairs[i % len(self.pairs)]
-        layer = w.n_pre + it
-        cache = oracle.OracleCache(w.fmt, w.d, w.n_pre, w.L_max)
-        cache.append(layer, 0, 0, w.h_rows(layer, b, 0, w.ctx[b]))
-        return it, b, cache, w.h_new(it)[b:b + 1], w.residual(it)[b:b + 1]
+        import oracle.cpp as ocpp
+        if i not in self.prepared:
+            w = self.w
+            it, b = self.pairs[i % len(self.pairs)]
+            codes, scales = ocpp.quantize_rows(w.h_rows(w.n_pre + it, b, 0, w.ctx[b]), w.fmt)
+            self.prepared[i] = (it, b, codes, scales, w.h_new(it)[b], w.residual(it)[b])
+        return self.prepared[i]
 
-    def decode(self, i):
-        """Time the oracle as it stands on pair i: append, explicit K/V rebuild, softmax, norm check."""
-        import numpy as np
-        import oracle
-        while len(self.prepared) <= i:
-            self.prepared.append(self._prepare(len(self.prepared)))
-        it, b, cache, hn, res = self.prepared[i]
+    def decode(self, i, threads):
+        """Time the oracle as it stands on pair i with `threads` OpenMP threads (over heads)."""
+        import oracle.cpp as ocpp
+        it, b, codes, scales, hn, res = self._prepare(i)
         w = self.w
         t0 = time.perf_counter()
-        oracle.decode_iteration(cache, it, [w.loops[b]], [w.ctx[b]], hn, *self.W, w.H, w.hd, res, w.threshold,
-                                np.zeros(1, np.uint8), np.full(1, -1, np.int32))
+        ocpp.decode_lane(w.fmt, codes, scales, hn, *self.W, w.H, w.hd, residual=res, threshold=w.threshold, it=it,
+                         loops=w.loops[b], form=0, threads=threads)
         return w.ctx[b], time.perf_counter() - t0
 
-    def run(self, budget_s, max_pairs=None):
-        """Decode pairs 0, 1, ... until the budget is spent; returns (positions/s, s, description)."""
+    def run(self, budget_s, threads, max_pairs=None, first=0):
+        """Decode pairs first, first+1, ... until the budget is spent; returns (positions/s, s, n, positions)."""
         pos, spent, n = 0, 0.0, 0
         while n == 0 or (spent < budget_s and (max_pairs is None or n < max_pairs)):
-            p, t = self.decode(n)
+            p, t = self.decode(first + n, threads)
             pos, spent, n = pos + p, spent + t, n + 1
-        desc = (f"{n} (lane, iteration) decodes of {self.w.name} by the FP64 oracle (append + explicit K/V "
-                f"rebuild + softmax + norm check), {pos} cached positions, {spent:.2f} s")
-        return pos / spent, spent, desc
+        return pos / spent, spent, n, pos
+
+
+def cpu_baseline(w, budget_s):
+    """The C++ oracle on the host cores: single-threaded, and with OpenMP over the heads of a
+    lane (the (lane, head) tasks of the sample), on a bounded sample of (lane, iteration) pairs
+    of the workload, extrapolated linearly to the whole step (positions/s is per position)."""
+    import oracle.cpp as ocpp
+    sample = OracleSample(w)
+    threads = min(ocpp.max_threads(), w.H)
+    v1, s1, n1, p1 = sample.run(budget_s / 2, threads=1, max_pairs=1)
+    vm, sm, nm, pm = sample.run(budget_s / 2, threads=threads, first=1)
+    desc = (f"plain C++ FP64 oracle (append + exact dequant + explicit K/V rebuild + softmax + norm check) on "
+            f"{nm} (lane, iteration) decodes of {w.name} ({pm} cached positions, {sm:.2f} s) with {threads} OpenMP "
+            f"threads over the heads; single-threaded: {n1} decode ({p1} positions, {s1:.2f} s) = {v1:.4g} "
+            f"positions/s; rates extrapolated linearly from the sample to the whole step "
+            f"({w.cached_positions_per_step()} positions); host {os.cpu_count()} logical CPUs, {cpu_model()}")
+    return {"value": vm, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc,
+            "single_thread_value": v1, "nproc": os.cpu_count(), "cpu_model": cpu_model(), "extrapolated": True}
 
 
 def load_peaks():
@@ -199,23 +216,36 @@ class ClockSampler:
         self.proc = None
 
     def __enter__(self):
+        import threading
+        self.lines = []
         try:
             self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
-        time.sleep(0.3)
+            return self
+
+        def reader():
+            for line in self.proc.stdout:
+                if line.strip():
+                    self.lines.append(line)
+        self.thread = threading.Thread(target=reader, daemon=True)
+        self.thread.start()
+        # the first sample comes after nvidia-smi has started: wait for it (bounded), so that the
+        # timed region is covered
+        t0 = time.time()
+        while not self.lines and time.time() - t0 < 10.0 and self.proc.poll() is None:
+            time.sleep(0.05)
         return self
 
     def __exit__(self, *exc):
-        self.lines = []
         if self.proc:
+            time.sleep(0.25)  # one more sample period after the timed work
             self.proc.terminate()
             try:
-                out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
+            self.thread.join(timeout=5)
         return False
 
     def summary(self):
@@ -240,24 +270,30 @@ class ClockSampler:
 def run_reference(args, rank, world):
     if rank != 0:
         return
+    import oracle.cpp as ocpp
     w = workload_for_rank(args.workload, 0)
     sample = OracleSample(w)
-    # a step = the same bounded sample of the workload (2 lane-iteration decodes)
-    for _ in range(args.warmup):
-        sample.run(0.0, max_pairs=2)
-    t, pos = 0.0, 0.0
-    desc = ""
-    for _ in range(args.steps):
-        v, s, desc = sample.run(float("inf"), max_pairs=2)
-        t += s
-        pos += v * s
+    threads = min(ocpp.max_threads(), w.H)
+    # a step = a bounded sample of the workload: one (lane, iteration) decode, OpenMP over its heads
+    for k in range(args.warmup):
+        sample.run(0.0, threads, max_pairs=1, first=k)
+    t, pos = 0.0, 0
+    for k in range(args.steps):
+        _, s_, _, p_ = sample.run(0.0, threads, max_pairs=1, first=args.warmup + k)
+        t += s_
+        pos += p_
     value = pos / t
+    desc = (f"per step: one (lane, iteration) decode of {w.name} by the plain C++ FP64 oracle (append + exact "
+            f"dequant + explicit K/V rebuild + softmax + norm check), {threads} OpenMP threads over the heads; "
+            f"{pos} cached positions in {t:.2f} s over {args.steps} steps, extrapolated linearly to the step's "
+            f"{w.cached_positions_per_step()} positions; host {os.cpu_count()} logical CPUs, {cpu_model()}")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * t / args.steps,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000.0 * w.cached_positions_per_step() / value,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded)", "config": workload_config(w, args.gpus),
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-                             "sample": "per step: " + desc},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc,
+                             "nproc": os.cpu_count(), "cpu_model": cpu_model(), "extrapolated": True},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -288,23 +324,34 @@ def run_ours(args, rank, world, local_rank):
 
     K = args.steps
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local_rank) as clocks:
-        # headline pass: the steps alone (an event between two kernels would stop the next one
-        # from being scheduled during the previous one's tail, so none is recorded in here)
-        barrier()
-        torch.cuda.synchronize()
-        start.record(stream)
+    clocks = ClockSampler(local_rank)
+    clocks.__enter__()  # samples through every timed pass below, the end-to-end one included
+    # headline pass: the steps alone (an event between two kernels would stop the next one
+    # from being scheduled during the previous one's tail, so none is recorded in here)
+    barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(K):
+        dw.step(fused_append=True)
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    # per-step pass: the same K steps, each between its own pair of events (median reported)
+    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for a, b_ in step_ev:
+        a.record(stream)
+        dw.step(fused_append=True)
+        b_.record(stream)
+    torch.cuda.synchronize()
+    step_ms_median = statistics.median(a.elapsed_time(b_) for a, b_ in step_ev)
+    barrier()
+    # kernel pass: the same K steps again, with events around every streaming-kernel launch
+    with tl.ProfileHook(K * w.L_max) as prof:
         for _ in range(K):
             dw.step(fused_append=True)
-        end.record(stream)
         torch.cuda.synchronize()
-        barrier()
-        # kernel pass: the same K steps again, with events around every streaming-kernel launch
-        with tl.ProfileHook(K * w.L_max) as prof:
-            for _ in range(K):
-                dw.step(fused_append=True)
-            torch.cuda.synchronize()
     ms_max = max_over_ranks(start.elapsed_time(end), world, f"cuda:{local_rank}")
+    step_ms_median = max_over_ranks(step_ms_median, world, f"cuda:{local_rank}")
     pos_step = w.cached_positions_per_step()
     value = whole_job_rate(pos_step, K, ms_max, world)
 
@@ -380,6 +427,7 @@ def run_ours(args, rank, world, local_rank):
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
+    clocks.__exit__(None, None, None)
     for n in names:
         setattr(dw, n, sets[0][n])
     e2e_value = whole_job_rate(pos_step, K, max_over_ranks(e0.elapsed_time(e1), world, f"cuda:{local_rank}"), world)
@@ -388,8 +436,7 @@ def run_ours(args, rank, world, local_rank):
         return
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        v, s, desc = OracleSample(w).run(args.cpu_seconds)
-        cpu = {"value": v, "unit": UNIT, "cores": blas_threads(), "kind": "oracle", "sample": desc}
+        cpu = cpu_baseline(w, args.cpu_seconds)
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
             "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": DTYPE_OF_FMT[w.fmt] + "-h codes, fp16 tensor operands, fp32 accumulate",
@@ -397,6 +444,10 @@ def run_ours(args, rank, world, local_rank):
             "config": workload_config(w, world, {"entry_point": "tl_storeh_append_attn_decode per loop iteration",
                                                  "cached_positions_per_step_per_gpu": pos_step,
                                                  "step_roofline_ms_hbm": step_roofline_ms,
+                                                 "ms_per_step_median_of_per_step_events": step_ms_median,
+                                                 "timing": ("value and ms_per_step: K steps between one event "
+                                                            "pair (no event between kernels); the median of K "
+                                                            "per-step event pairs is reported beside it"),
                                                  "step_frac_of_hbm_roofline": step_roofline_ms / (ms_max / K)}),
             "roofline": roofline,
             "cpu_baseline": cpu,

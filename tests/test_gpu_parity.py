@@ -1,4 +1,4 @@
-"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+"""Parity of the CUDA path (through the C ABI) with the plain C++ CPU oracle (oracle/cpp.py).
 
 Bars: codes and scales bit-exact; abort flags and first-abort iterations
 identical; attention outputs within max-abs 2e-3 and relative L2 1e-3 of the
@@ -12,6 +12,7 @@ import pytest
 import torch
 
 import oracle
+import oracle.cpp
 import synth
 from synth.workloads import get_workload, select_lanes, small_variant
 
@@ -36,10 +37,10 @@ def _dw(w, **kw):
 def _oracle_lane(w, it, b, form="explicit"):
     layer = w.n_pre + it
     rows = np.concatenate([w.h_rows(layer, b, 0, w.ctx[b]), w.h_new(it)[b:b + 1]])
-    codes, scales = oracle.quantize_rows(rows, w.fmt)
-    hh = oracle.dequantize_rows(codes, scales, w.fmt, w.d)
+    codes, scales = oracle.cpp.quantize_rows(rows, w.fmt)
+    hh = oracle.cpp.dequantize_rows(codes, scales, w.fmt, w.d)
     W = [w.weight(k) for k in "qkv"]
-    f = oracle.attend_explicit if form == "explicit" else oracle.attend_absorbed
+    f = oracle.cpp.attend_explicit if form == "explicit" else oracle.attend_absorbed
     return f(hh, w.h_new(it)[b], *W, w.H, w.hd)
 
 
@@ -78,7 +79,7 @@ def test_append_codes_bit_exact(fmt):
     cb = oracle.row_code_bytes(fmt, d)
     codes = cache.codes.view(3, 2, n + 5, cb).cpu().numpy()
     for lane, src, p0 in ((0, h, 3), (1, h[::-1].copy(), 0)):
-        want_c, want_s = oracle.quantize_rows(src, fmt)
+        want_c, want_s = oracle.cpp.quantize_rows(src, fmt)
         assert np.array_equal(codes[2, lane, p0:p0 + n], want_c), f"codes lane {lane}"
         if fmt != 0:
             ns = oracle.row_scale_count(fmt, d)
@@ -125,7 +126,7 @@ def test_norm_flags_identical(flag_mix):
         r = res[it].copy()
         if it == 2:
             r *= 0.01          # a quiet iteration: flags stay sticky
-        f, fi, nrm = oracle.residual_norm_check(r, w.threshold, it, loops, f, fi)
+        f, fi, nrm = oracle.cpp.residual_norm_check(r, w.threshold, it, loops, f, fi)
         dn = torch.full((w.B,), float("nan"), device="cuda")
         tl.residual_norm_check(torch.from_numpy(r).cuda(), w.threshold, it, dl, df, dfi, norms_out=dn)
         torch.cuda.synchronize()
@@ -170,7 +171,7 @@ def test_decode_matches_oracle_small(name, ctx, loops):
                 assert np.all(np.isnan(out[it, b])), f"inactive lane {b} iteration {it} was written"
             elif it in its:
                 _assert_close(out[it, b], _oracle_lane(w, it, b), f"{name} lane {b} it {it}")
-        f, fi, _ = oracle.residual_norm_check(w.residual(it, True), w.threshold, it, np.array(w.loops), f, fi)
+        f, fi, _ = oracle.cpp.residual_norm_check(w.residual(it, True), w.threshold, it, np.array(w.loops), f, fi)
     assert np.array_equal(dw.flags.cpu().numpy(), f) and np.array_equal(dw.first.cpu().numpy(), fi)
     import store_kv_attention_b200 as tl
     assert tl.poll_status(dw.cache) == tl.TL_OK
@@ -283,16 +284,16 @@ def test_decode_full_size_sampled(name, samples):
         f = np.zeros(w.B, np.uint8)
         fi = np.full(w.B, -1, np.int32)
         for it in range(w.L_max):
-            f, fi, _ = oracle.residual_norm_check(w.residual(it, flag_mix), w.threshold, it, np.array(w.loops), f, fi)
+            f, fi, _ = oracle.cpp.residual_norm_check(w.residual(it, flag_mix), w.threshold, it, np.array(w.loops), f, fi)
         assert np.array_equal(fus.flags.cpu().numpy(), f) and np.array_equal(fus.first.cpu().numpy(), fi)
-        if flag_mix:
+        if flag_mix and w.B > 1:
             assert 0 < f.sum() < w.B
         # every active (lane, iteration) was written, every inactive one was not
         assert np.all(np.isfinite(out[act])) and np.all(np.isnan(out[~act]))
     # the new token's row of every active (lane, iteration), bit-exact with the oracle's quantiser
     for it in range(w.L_max):
         bs = [b for b in range(w.B) if act[it, b]]
-        want_c, want_s = oracle.quantize_rows(w.h_new(it)[bs], w.fmt)
+        want_c, want_s = oracle.cpp.quantize_rows(w.h_new(it)[bs], w.fmt)
         got_c, got_s = _new_rows_from_cache(fus, it)
         assert np.array_equal(got_c[bs], want_c), f"{name} codes of iteration {it}"
         if got_s is not None:
@@ -332,7 +333,7 @@ def test_fused_append_more_lanes_than_ctas(fmt):
     assert torch.equal(sep.flags, fus.flags) and torch.equal(sep.first, fus.first)
     for it in range(w.L_max):
         bs = [b for b in range(w.B) if it < w.loops[b]]
-        want_c, want_s = oracle.quantize_rows(w.h_new(it)[bs], w.fmt)
+        want_c, want_s = oracle.cpp.quantize_rows(w.h_new(it)[bs], w.fmt)
         got_c, got_s = _new_rows_from_cache(fus, it)
         assert np.array_equal(got_c[bs], want_c)
         if got_s is not None:

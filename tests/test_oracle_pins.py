@@ -17,8 +17,12 @@ import pytest
 import torch
 
 import oracle
+import oracle.cpp
 import synth
 from synth.workloads import small_variant
+
+# Both oracles, the numpy one and the plain C++ one, must pass every pin that applies to them.
+IMPLS = [pytest.param(oracle, id="numpy"), pytest.param(oracle.cpp, id="cpp")]
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -34,24 +38,26 @@ def _read_golden(name):
 
 
 # --------------------------------------------------------------------------- quantiser
-def test_int8_hand_cases():
+@pytest.mark.parametrize("ora", IMPLS)
+def test_int8_hand_cases(ora):
     for scale, xs, codes in _read_golden("quant_int8_hand.txt"):
         x = np.array([float(v) for v in xs.split()], dtype=np.float16)
         row = np.zeros((1, 64), np.float16)
         row[0, :x.size] = x
-        c, s = oracle.quantize_rows(row, oracle.FMT_INT8)
+        c, s = ora.quantize_rows(row, oracle.FMT_INT8)
         assert s.dtype == np.float32 and s[0, 0] == np.float32(float(scale))
         want = np.array([int(v) for v in codes.split()], dtype=np.int8)
         assert np.array_equal(c.view(np.int8)[0, :x.size], want), (xs, c.view(np.int8)[0, :x.size])
         assert np.all(c.view(np.int8)[0, x.size:] == 0)
 
 
-def test_int4_hand_cases_and_nibble_order():
+@pytest.mark.parametrize("ora", IMPLS)
+def test_int4_hand_cases_and_nibble_order(ora):
     for scale, xs, codes, hexbytes in _read_golden("quant_int4_hand.txt"):
         x = np.array([float(v) for v in xs.split()], dtype=np.float16)
         row = np.zeros((1, 64), np.float16)
         row[0, :x.size] = x
-        c, s = oracle.quantize_rows(row, oracle.FMT_INT4)
+        c, s = ora.quantize_rows(row, oracle.FMT_INT4)
         assert s.dtype == np.float16 and s[0, 0] == np.float16(float(scale))
         want = np.array([int(v) for v in codes.split()], dtype=np.int8)
         assert np.array_equal(oracle.unpack_int4(c)[0, :x.size], want)
@@ -60,13 +66,14 @@ def test_int4_hand_cases_and_nibble_order():
 
 
 @pytest.mark.parametrize("fmt,qmax", [(oracle.FMT_INT8, 127), (oracle.FMT_INT4, 7)])
-def test_quantiser_is_nearest_grid_point(fmt, qmax):
+@pytest.mark.parametrize("ora", IMPLS)
+def test_quantiser_is_nearest_grid_point(ora, fmt, qmax):
     """Brute force: every code is the grid point c*scale nearest to x (ties to even c),
     except where the exact quotient lies within an fp32 rounding of a tie."""
     rng = np.random.default_rng(5)
     h = (rng.standard_normal((64, 256)) * np.exp(rng.uniform(-3, 3, (64, 1)))).astype(np.float16)
     h[3, :] = 0
-    codes, scales = oracle.quantize_rows(h, fmt)
+    codes, scales = ora.quantize_rows(h, fmt)
     c = codes.view(np.int8) if fmt == oracle.FMT_INT8 else oracle.unpack_int4(codes)
     group = 256 if fmt == oracle.FMT_INT8 else 64
     sc = np.repeat(scales.astype(np.float64).reshape(64, -1), group, axis=1)
@@ -95,11 +102,12 @@ def test_quantiser_is_nearest_grid_point(fmt, qmax):
 
 
 @pytest.mark.parametrize("fmt", [oracle.FMT_FP16, oracle.FMT_INT8, oracle.FMT_INT4])
-def test_roundtrip_bound(fmt):
+@pytest.mark.parametrize("ora", IMPLS)
+def test_roundtrip_bound(ora, fmt):
     rng = np.random.default_rng(1)
     h = rng.standard_normal((32, 1024)).astype(np.float16)
-    codes, scales = oracle.quantize_rows(h, fmt)
-    hh = oracle.dequantize_rows(codes, scales, fmt, 1024)
+    codes, scales = ora.quantize_rows(h, fmt)
+    hh = ora.dequantize_rows(codes, scales, fmt, 1024)
     x = h.astype(np.float64)
     if fmt == oracle.FMT_FP16:
         assert np.array_equal(hh, x)  # FP16-h is lossless: K/V rebuilt bit-exactly
@@ -112,7 +120,8 @@ def test_roundtrip_bound(fmt):
 
 @pytest.mark.parametrize("fmt,d,lo,hi", [(oracle.FMT_INT8, 1024, 0.004, 0.010),
                                          (oracle.FMT_INT4, 2048, 0.08, 0.12)])
-def test_closed_form_kv_error(fmt, d, lo, hi):
+@pytest.mark.parametrize("ora", IMPLS)
+def test_closed_form_kv_error(ora, fmt, d, lo, hi):
     """K relative L2 error on Gaussian h equals the uniform-rounding closed form
     sqrt(sum scale^2/12 / sum h^2), and lands where the pages put it: about 0.6%
     for INT8-h and about 10% for INT4-h (Architecture-Exclusive Features,
@@ -121,8 +130,8 @@ def test_closed_form_kv_error(fmt, d, lo, hi):
     h = w.h_rows(w.n_pre, 0, 0, 512)
     if fmt == oracle.FMT_INT8:
         h = synth.h_rows_f16(w.seed, synth.row_id(w.n_pre, 0, np.arange(512)), d)  # no outliers
-    codes, scales = oracle.quantize_rows(h, fmt)
-    hh = oracle.dequantize_rows(codes, scales, fmt, d)
+    codes, scales = ora.quantize_rows(h, fmt)
+    hh = ora.dequantize_rows(codes, scales, fmt, d)
     Wk = w.weight("k").astype(np.float64)
     x = h.astype(np.float64)
     K, Kh = x @ Wk.T, hh @ Wk.T
@@ -162,12 +171,13 @@ def _library_stored_kv(h_rows64, h_new, W, H, hd):
 
 @pytest.mark.parametrize("form", ["explicit", "absorbed"])
 @pytest.mark.parametrize("fmt", [oracle.FMT_FP16, oracle.FMT_INT8, oracle.FMT_INT4])
-def test_attention_matches_library_over_stored_kv(form, fmt):
+@pytest.mark.parametrize("ora", IMPLS)
+def test_attention_matches_library_over_stored_kv(ora, form, fmt):
     H, hd = 2, 32
     d, W, h = _tiny(H=H, hd=hd, n=9, seed=fmt)
-    codes, scales = oracle.quantize_rows(h, fmt)
-    hh = oracle.dequantize_rows(codes, scales, fmt, d)
-    f = oracle.attend_explicit if form == "explicit" else oracle.attend_absorbed
+    codes, scales = ora.quantize_rows(h, fmt)
+    hh = ora.dequantize_rows(codes, scales, fmt, d)
+    f = ora.attend_explicit if form == "explicit" else ora.attend_absorbed
     got = f(hh, h[-1], *W, H, hd)
     want = _library_stored_kv(hh, h[-1], W, H, hd)
     assert np.max(np.abs(got - want)) <= 1e-12 * max(1.0, np.max(np.abs(want)))
@@ -192,37 +202,41 @@ def test_fp16_h_identical_to_stored_kv():
     assert np.max(np.abs(out[0] - _library_stored_kv(x, h[-1], W, H, hd))) < 1e-12
 
 
-def test_absorbed_equals_explicit_at_workload_shape():
+@pytest.mark.parametrize("ora", IMPLS)
+def test_absorbed_equals_explicit_at_workload_shape(ora):
     w = synth.get_workload("int4_2b")
     h = w.h_rows(w.n_pre, 0, 0, 257)
-    codes, scales = oracle.quantize_rows(h, w.fmt)
-    hh = oracle.dequantize_rows(codes, scales, w.fmt, w.d)
+    codes, scales = ora.quantize_rows(h, w.fmt)
+    hh = ora.dequantize_rows(codes, scales, w.fmt, w.d)
     W = [w.weight(k) for k in "qkv"]
-    a = oracle.attend_explicit(hh, h[-1], *W, w.H, w.hd)
-    b = oracle.attend_absorbed(hh, h[-1], *W, w.H, w.hd)
+    a = ora.attend_explicit(hh, h[-1], *W, w.H, w.hd)
+    b = ora.attend_absorbed(hh, h[-1], *W, w.H, w.hd)
     assert np.max(np.abs(a - b)) < 1e-12
 
 
-def test_single_row_gives_v_of_new_token():
+@pytest.mark.parametrize("ora", IMPLS)
+def test_single_row_gives_v_of_new_token(ora):
     """With no cached positions the softmax has one entry, so o_j = (W_v h_new)_j."""
     H, hd = 2, 16
     d, W, h = _tiny(H=H, hd=hd, n=1, seed=4)
     hh = h.astype(np.float64)
-    for f in (oracle.attend_explicit, oracle.attend_absorbed):
+    for f in (ora.attend_explicit, ora.attend_absorbed):
         o = f(hh, h[0], *W, H, hd)
         v = W[2].astype(np.float64) @ hh[0]
         assert np.max(np.abs(o.reshape(-1) - v)) < 1e-13
 
 
-def test_identical_rows_give_their_v():
+@pytest.mark.parametrize("ora", IMPLS)
+def test_identical_rows_give_their_v(ora):
     H, hd = 2, 16
     d, W, h = _tiny(H=H, hd=hd, n=1, seed=6)
     rows = np.repeat(h.astype(np.float64), 10, axis=0)
-    o = oracle.attend_explicit(rows, h[0] * np.float16(3), *W, H, hd)
+    o = ora.attend_explicit(rows, h[0] * np.float16(3), *W, H, hd)
     assert np.max(np.abs(o.reshape(-1) - W[2].astype(np.float64) @ rows[0])) < 1e-13
 
 
-def test_softmax_scale_is_inverse_sqrt_head_dim():
+@pytest.mark.parametrize("ora", IMPLS)
+def test_softmax_scale_is_inverse_sqrt_head_dim(ora):
     """Two rows whose head-0 scores differ by exactly sqrt(hd)*ln(3): weights 3/4 and 1/4."""
     H, hd = 1, 16
     d = 16
@@ -237,7 +251,7 @@ def test_softmax_scale_is_inverse_sqrt_head_dim():
     r2[0] = math.sqrt(hd) * math.log(3.0)
     r2[1] = 0.0
     rows = np.stack([r1, r2])
-    o = oracle.attend_explicit(rows, q, Wq, Wk, Wv, H, hd)
+    o = ora.attend_explicit(rows, q, Wq, Wk, Wv, H, hd)
     want = 0.25 * r1 + 0.75 * r2
     assert np.max(np.abs(o.reshape(-1) - want)) < 1e-12
 
@@ -321,40 +335,43 @@ def test_mixed_batch_lane_equals_solo_run():
 
 
 # --------------------------------------------------------------------------- safety check
-def test_norm_exact_triples_and_strictness():
+@pytest.mark.parametrize("ora", IMPLS)
+def test_norm_exact_triples_and_strictness(ora):
     r = np.zeros((3, 8), np.float32)
     r[0, :2] = [3, 4]          # norm 5
     r[1, :3] = [2, 3, 6]       # norm 7
     r[2, :2] = [30, 40]        # norm 50
-    flags, first, norms = oracle.residual_norm_check(r, 5.0, 0, np.array([4, 4, 4]),
+    flags, first, norms = ora.residual_norm_check(r, 5.0, 0, np.array([4, 4, 4]),
                                                      np.zeros(3, np.uint8), np.full(3, -1, np.int32))
     assert np.array_equal(norms, [5.0, 7.0, 50.0])
     assert list(flags) == [0, 1, 1] and list(first) == [-1, 0, 0]
-    flags, first, _ = oracle.residual_norm_check(r, 50.0, 1, np.array([4, 4, 4]),
+    flags, first, _ = ora.residual_norm_check(r, 50.0, 1, np.array([4, 4, 4]),
                                                  np.zeros(3, np.uint8), np.full(3, -1, np.int32))
     assert list(flags) == [0, 0, 0]  # exactly at the threshold is not "exceeds"
 
 
-def test_norm_sticky_and_inactive_lanes():
+@pytest.mark.parametrize("ora", IMPLS)
+def test_norm_sticky_and_inactive_lanes(ora):
     big = np.full((2, 4), 100.0, np.float32)
     small = np.zeros((2, 4), np.float32)
     loops = np.array([3, 1])
-    f, first, _ = oracle.residual_norm_check(big, 10.0, 0, loops, np.zeros(2, np.uint8),
+    f, first, _ = ora.residual_norm_check(big, 10.0, 0, loops, np.zeros(2, np.uint8),
                                              np.full(2, -1, np.int32))
     assert list(f) == [1, 1] and list(first) == [0, 0]
-    f, first, norms = oracle.residual_norm_check(small, 10.0, 1, loops, f, first)
+    f, first, norms = ora.residual_norm_check(small, 10.0, 1, loops, f, first)
     assert list(f) == [1, 1] and list(first) == [0, 0]
     assert norms[0] == 0 and np.isnan(norms[1])
-    f, first, _ = oracle.residual_norm_check(big, 10.0, 2, loops, np.zeros(2, np.uint8),
+    f, first, _ = ora.residual_norm_check(big, 10.0, 2, loops, np.zeros(2, np.uint8),
                                              np.full(2, -1, np.int32))
     assert list(f) == [1, 0] and list(first) == [2, -1]  # lane 1 has only one iteration
 
 
-def test_pages_safety_example():
+@pytest.mark.parametrize("ora", IMPLS)
+def test_pages_safety_example(ora):
     for thr, norm, it, flag, first in _read_golden("safety_check_example.txt"):
         r = np.zeros((1, 2048), np.float32)
         r[0, 0] = float(norm)
-        f, fi, n = oracle.residual_norm_check(r, float(thr), int(it), np.array([8]),
+        f, fi, n = ora.residual_norm_check(r, float(thr), int(it), np.array([8]),
                                               np.zeros(1, np.uint8), np.full(1, -1, np.int32))
         assert f[0] == int(flag) and fi[0] == int(first)
         assert abs(n[0] - float(norm)) < 1e-5
@@ -381,3 +398,68 @@ def test_generator_moments_and_determinism():
     assert 0.003 < big.mean() < 0.02   # ~1% outlier rows scaled x8
     w5 = synth.get_workload("int4_mixed")
     assert min(w5.ctx) >= 1024 and max(w5.ctx) <= 8192 and len(set(w5.ctx)) > 40
+
+
+# --------------------------------------------------------------------------- the C++ oracle
+def test_cpp_fp16_rounding_matches_ieee():
+    """The C++ oracle's binary32 -> binary16 rounding (INT4 scales) is IEEE round-to-nearest-even,
+    checked against numpy's conversion over a wide range, subnormals, ties and overflow."""
+    rng = np.random.default_rng(7)
+    x = np.concatenate([rng.standard_normal(50000) * np.exp(rng.uniform(-25, 12, 50000)),
+                        [0.0, -0.0, 65504.0, 65519.99, 65520.0, 2.0 ** -24, 2.0 ** -25, 3 * 2.0 ** -26,
+                         2.0 ** -14, 1.0 + 2.0 ** -11, 1.0 + 3 * 2.0 ** -11, -1e-9]]).astype(np.float32)
+    got = np.array([oracle.cpp.f32_to_f16_bits(v) for v in x], np.uint16)
+    with np.errstate(over="ignore"):
+        want = x.astype(np.float16).view(np.uint16)
+    assert np.array_equal(got, want)
+
+
+@pytest.mark.parametrize("fmt,d", [(oracle.FMT_FP16, 256), (oracle.FMT_INT8, 1024), (oracle.FMT_INT4, 2048)])
+def test_cpp_quantiser_and_dequant_equal_numpy(fmt, d):
+    rng = np.random.default_rng(fmt + 3)
+    h = (rng.standard_normal((80, d)) * np.exp(rng.uniform(-6, 6, (80, 1)))).astype(np.float16)
+    h[0] = 0
+    h[1, :8] = np.array([0.5, 1.5, 2.5, -2.5, 3.5, 6.5, -7, 7], np.float16)
+    h[2] = np.float16(3e-7)
+    c1, s1 = oracle.quantize_rows(h, fmt)
+    c2, s2 = oracle.cpp.quantize_rows(h, fmt)
+    assert np.array_equal(c1, c2) and s1.dtype == s2.dtype and np.array_equal(s1.view(np.uint8), s2.view(np.uint8))
+    assert np.array_equal(oracle.dequantize_rows(c1, s1, fmt, d), oracle.cpp.dequantize_rows(c2, s2, fmt, d))
+
+
+@pytest.mark.parametrize("form", ["explicit", "absorbed"])
+@pytest.mark.parametrize("H,hd,n", [(1, 8, 1), (2, 16, 9), (4, 64, 33)])
+def test_cpp_attention_equals_numpy(form, H, hd, n):
+    d, W, h = _tiny(H=H, hd=hd, n=n, seed=H + n)
+    hh = h.astype(np.float64)
+    f1 = oracle.attend_explicit if form == "explicit" else oracle.attend_absorbed
+    f2 = oracle.cpp.attend_explicit if form == "explicit" else oracle.cpp.attend_absorbed
+    a, b = f1(hh, h[-1], *W, H, hd), f2(hh, h[-1], *W, H, hd)
+    assert np.max(np.abs(a - b)) <= 1e-12 * max(1.0, np.max(np.abs(a)))
+    # the OpenMP split over heads does not change a single bit
+    assert np.array_equal(b, f2(hh, h[-1], *W, H, hd, threads=1))
+
+
+@pytest.mark.parametrize("fmt", [oracle.FMT_FP16, oracle.FMT_INT8, oracle.FMT_INT4])
+def test_cpp_decode_lane_equals_numpy_decode_iteration(fmt):
+    """One lane's whole iteration (append, dequant, explicit attention, safety check) in C++
+    against the numpy oracle's decode_iteration on the same lane."""
+    w = synth.get_workload({0: "tiny_fp16", 1: "int8_b16", 2: "int4_2b"}[fmt])
+    w = small_variant(w, ctx=[45], loops=[2])
+    it, layer = 1, w.n_pre + 1
+    ctx_rows = w.h_rows(layer, 0, 0, 45)
+    W = [w.weight(k) for k in "qkv"]
+    res = w.residual(it)
+    cache = oracle.OracleCache(w.fmt, w.d, w.n_pre, w.L_max)
+    cache.append(layer, 0, 0, ctx_rows)
+    want, wf, wfi, _ = oracle.decode_iteration(cache, it, [2], [45], w.h_new(it)[:1], *W, w.H, w.hd, res,
+                                               w.threshold, np.zeros(1, np.uint8), np.full(1, -1, np.int32))
+    cc, cs = oracle.cpp.quantize_rows(ctx_rows, fmt)
+    got, gf, gfi, codes, scales = oracle.cpp.decode_lane(fmt, cc, cs, w.h_new(it)[0], *W, w.H, w.hd, residual=res[0],
+                                                         threshold=w.threshold, it=it, loops=2)
+    assert np.max(np.abs(got - want[0])) <= 1e-12 * max(1.0, np.max(np.abs(want)))
+    assert (gf, gfi) == (int(wf[0]), int(wfi[0]))
+    rc, rs = cache.read_rows(layer, 0, 46)
+    assert np.array_equal(codes, rc)
+    if fmt != oracle.FMT_FP16:
+        assert np.array_equal(scales.view(np.uint8), rs.view(np.uint8))
