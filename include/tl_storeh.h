@@ -196,6 +196,67 @@ TL_API tl_status tl_storeh_append_attn_decode(const tl_storeh_desc* desc, tl_sto
                                 size_t workspace_bytes, int32_t n_lanes, tl_stream_t stream);
 
 /*
+ * Tree verification over the store-h cache: many query tokens per lane in one enqueue
+ * [Architecture-Exclusive Features, "Tree speculative decoding": K draft branches, each a
+ * chain of D tokens grown from the same root, are verified in one mask-gated pass].
+ * For every lane b with iter < loops[b]:
+ *   1. the K x D tree tokens' h rows are quantised into cache layer n_pre + iter at positions
+ *      ctx_len[b] + k*D + t (branch k, depth t), exactly as tl_storeh_append writes them;
+ *   2. token (k, t) attends the lane's cached positions 0 .. ctx_len[b]-1 and its own
+ *      branch's tokens (k, 0 .. t) -- itself included, no other branch -- with its query
+ *      q = W_q h_tree[b][k][t] from the unquantised row, K = W_k h, V = W_v h and the softmax
+ *      scale 1/sqrt(head_dim) of tl_storeh_attn_decode:
+ *        out[b][k][t] = sum over those rows c of softmax(s)_c V_c.
+ *   With one branch the pass equals `depth` sequential single-token decodes; token (0, t)
+ *   reads exactly the rows (and in the same order) of a decode with ctx_len[b] + t cached
+ *   positions, so its output is bit-identical to that decode's.
+ *
+ *   loops, ctx_len  device int32 [n_lanes]; ctx_len[b] + n_branches*depth <= max_ctx, or the
+ *                   lane is skipped and TL_ERR_DEVICE_RANGE recorded (its tree rows that fit
+ *                   are still written)
+ *   h_tree          device fp16 [n_lanes][n_branches][depth][d_model]
+ *   W_q, W_k, W_v   device fp16 [d_model][d_model]
+ *   out             device fp32 [n_lanes][n_branches][depth][n_heads][head_dim]; rows of
+ *                   inactive lanes are not written
+ *   workspace       tl_storeh_verify_workspace_bytes(desc, n_lanes, n_branches, depth) bytes,
+ *                   256-byte aligned, its first 256 bytes (the status word, read with
+ *                   tl_storeh_poll_status) zeroed once
+ * No safety check runs here (a verification pass has no residual of its own).
+ * Supported: 1 <= n_branches * depth <= 1024.  The n_lanes * n_branches * depth query tokens
+ * run in groups of 64 through the decode kernels, each token as a lane of its own.
+ * Errors: TL_ERR_INVALID_ARG, TL_ERR_CAPACITY (n_lanes > max_lanes, iter outside [0, L_max),
+ * workspace too small, a tree larger than max_ctx), TL_ERR_UNSUPPORTED, TL_ERR_CUDA.
+ */
+TL_API tl_status tl_storeh_verify_attn(const tl_storeh_desc* desc, tl_storeh_cache cache, int32_t iter,
+                                       const int32_t* loops, const int32_t* ctx_len, const void* h_tree,
+                                       int32_t n_branches, int32_t depth, const void* W_q, const void* W_k,
+                                       const void* W_v, float* out, void* workspace, size_t workspace_bytes,
+                                       int32_t n_lanes, tl_stream_t stream);
+
+/* Workspace bytes of tl_storeh_verify_attn / tl_storeh_prefill_attn (prefill: n_branches = 1,
+ * depth = n_tokens): a decode workspace for 64 query tokens (with one split more per token,
+ * for its branch rows) plus 24 bytes per query token for its row map.
+ * Errors: the desc errors, TL_ERR_INVALID_ARG, TL_ERR_CAPACITY, TL_ERR_UNSUPPORTED. */
+TL_API tl_status tl_storeh_verify_workspace_bytes(const tl_storeh_desc* desc, int32_t n_lanes, int32_t n_branches,
+                                                  int32_t depth, size_t* bytes);
+
+/*
+ * Chunked prefill over the store-h cache [Architecture-Exclusive Features, "What this list is
+ * not": chunked prefill runs on the same cache; "Variable-L KV cache": loop iteration i fills
+ * layer n_pre + i]: n_tokens new tokens per lane are appended at positions ctx_len[b] ..
+ * ctx_len[b] + n_tokens - 1 of layer n_pre + iter and attend causally: token t attends
+ * positions 0 .. ctx_len[b] + t.  This is tl_storeh_verify_attn with one branch of depth
+ * n_tokens (same arguments, h_chunk [n_lanes][n_tokens][d_model], out
+ * [n_lanes][n_tokens][n_heads][head_dim]); each token's output is bit-identical to the decode
+ * of that token with ctx_len[b] + t cached positions.
+ */
+TL_API tl_status tl_storeh_prefill_attn(const tl_storeh_desc* desc, tl_storeh_cache cache, int32_t iter,
+                                        const int32_t* loops, const int32_t* ctx_len, const void* h_chunk,
+                                        int32_t n_tokens, const void* W_q, const void* W_k, const void* W_v,
+                                        float* out, void* workspace, size_t workspace_bytes, int32_t n_lanes,
+                                        tl_stream_t stream);
+
+/*
  * Per-iteration safety check [Novel Contributions, "Novel: Per-Iteration
  * Safety Check"; Architecture-Exclusive Features, "Per-iteration safety check"].
  * For every lane b with iter < loops[b] (all lanes when loops is NULL):

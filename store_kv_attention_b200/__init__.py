@@ -36,7 +36,8 @@ EXPORTS = ["tl_storeh_cache_bytes", "tl_storeh_workspace_bytes", "tl_storeh_appe
            "tl_residual_norm_check", "tl_storeh_poll_status", "tl_status_string", "tl_last_error_message",
            "tl_storeh_abi_version", "tl_set_profile", "tl_storeh_attn_decode_static_ws",
            "tl_storeh_append_attn_decode", "tl_storeh_selftest_wait_timeout", "tl_delta_cache_bytes",
-           "tl_delta_append", "tl_delta_workspace_bytes", "tl_delta_attn_decode"]
+           "tl_delta_append", "tl_delta_workspace_bytes", "tl_delta_attn_decode", "tl_storeh_verify_attn",
+           "tl_storeh_verify_workspace_bytes", "tl_storeh_prefill_attn"]
 
 
 class TLError(RuntimeError):
@@ -115,6 +116,12 @@ def _load():
     L.tl_delta_attn_decode.argtypes = [P(DeltaDescC), DeltaCacheC, i32, vp, vp, vp, vp, vp, vp, vp, vp, f32, vp, vp,
                                        vp, vp, sz, i32, vp]
     L.tl_delta_attn_decode.restype = ctypes.c_int
+    L.tl_storeh_verify_attn.argtypes = [P(Desc), Cache, i32, vp, vp, vp, i32, i32, vp, vp, vp, vp, vp, sz, i32, vp]
+    L.tl_storeh_verify_attn.restype = ctypes.c_int
+    L.tl_storeh_prefill_attn.argtypes = [P(Desc), Cache, i32, vp, vp, vp, i32, vp, vp, vp, vp, vp, sz, i32, vp]
+    L.tl_storeh_prefill_attn.restype = ctypes.c_int
+    L.tl_storeh_verify_workspace_bytes.argtypes = [P(Desc), i32, i32, i32, P(sz)]
+    L.tl_storeh_verify_workspace_bytes.restype = ctypes.c_int
     _lib_handle = L
     return L
 
@@ -296,6 +303,36 @@ def attn_decode_static_ws(cache: StoreHCache, it: int, loops, ctx_len, h_new, W_
            "tl_storeh_attn_decode_static_ws")
 
 
+def verify_workspace_bytes(desc: StoreHDesc, n_lanes: int, n_branches: int, depth: int) -> int:
+    b = ctypes.c_size_t()
+    _check(_load().tl_storeh_verify_workspace_bytes(ctypes.byref(desc.c()), n_lanes, n_branches, depth,
+                                                    ctypes.byref(b)), "tl_storeh_verify_workspace_bytes")
+    return b.value
+
+
+def verify_attn(cache: StoreHCache, it: int, loops, ctx_len, h_tree, W_q, W_k, W_v, out, workspace,
+                stream=None) -> None:
+    """tl_storeh_verify_attn: h_tree fp16 [n_lanes, K, D, d] (device) is appended at positions
+    ctx_len[b] + k*D + t, then every tree token attends the context and its own branch prefix;
+    out fp32 [n_lanes, K, D, H, hd]; workspace a uint8 device tensor of verify_workspace_bytes."""
+    n_lanes, K, D = int(h_tree.shape[0]), int(h_tree.shape[1]), int(h_tree.shape[2])
+    _check(_load().tl_storeh_verify_attn(ctypes.byref(cache.desc.c()), cache.c(), it, _ptr(loops), _ptr(ctx_len),
+                                         _ptr(h_tree), K, D, _ptr(W_q), _ptr(W_k), _ptr(W_v), _ptr(out),
+                                         _ptr(workspace), int(workspace.numel()), n_lanes, _stream(stream)),
+           "tl_storeh_verify_attn")
+
+
+def prefill_attn(cache: StoreHCache, it: int, loops, ctx_len, h_chunk, W_q, W_k, W_v, out, workspace,
+                 stream=None) -> None:
+    """tl_storeh_prefill_attn: h_chunk fp16 [n_lanes, T, d] appended at ctx_len[b] .. + T - 1, token
+    t attending positions 0 .. ctx_len[b] + t; out fp32 [n_lanes, T, H, hd]."""
+    n_lanes, T = int(h_chunk.shape[0]), int(h_chunk.shape[1])
+    _check(_load().tl_storeh_prefill_attn(ctypes.byref(cache.desc.c()), cache.c(), it, _ptr(loops), _ptr(ctx_len),
+                                          _ptr(h_chunk), T, _ptr(W_q), _ptr(W_k), _ptr(W_v), _ptr(out),
+                                          _ptr(workspace), int(workspace.numel()), n_lanes, _stream(stream)),
+           "tl_storeh_prefill_attn")
+
+
 def residual_norm_check(residual, threshold: float, it: int, loops, abort_flags, first_abort_iter,
                         norms_out=None, stream=None) -> None:
     n_lanes, d = int(residual.shape[0]), int(residual.shape[1])
@@ -305,9 +342,11 @@ def residual_norm_check(residual, threshold: float, it: int, loops, abort_flags,
 
 
 def poll_status(cache, stream=None) -> int:
-    """Synchronise and return (and clear) the device status of the cache's workspace
-    (a StoreHCache, or a DeltaCache made with n_lanes)."""
-    return _load().tl_storeh_poll_status(cache.workspace.data_ptr(), cache.ws_bytes, _stream(stream))
+    """Synchronise and return (and clear) the device status of a workspace: a StoreHCache's,
+    a DeltaCache's made with n_lanes, or a workspace tensor of its own (verification, prefill)."""
+    if hasattr(cache, "workspace"):
+        return _load().tl_storeh_poll_status(cache.workspace.data_ptr(), cache.ws_bytes, _stream(stream))
+    return _load().tl_storeh_poll_status(cache.data_ptr(), int(cache.numel()), _stream(stream))
 
 
 def selftest_wait_timeout(cache: StoreHCache, limit_cycles: int, stream=None) -> None:

@@ -408,6 +408,7 @@ struct OProjParams {
   int n_lanes, nb, cl, s_max;
   const float* ml;  // [n_lanes][s_max][16][2]
   const float* U;   // [n_lanes][s_max][16][d]
+  const LaneSeg* seg;  // rows of each lane (multi-query calls), or NULL: decode lanes
   float* out;       // [n_lanes][d]
   uint32_t* status;
   const float* residual;
@@ -492,7 +493,7 @@ __global__ void __launch_bounds__(kOProjThreads, 1)
   for (int x = threadIdx.x; x < p.n_lanes * lay.hib; x += kOProjThreads) {
     const int b = x / lay.hib, h2 = x % lay.hib, j = mb * lay.hib + h2;
     if (!((act >> b) & 1)) continue;
-    const int S = splits_for_rows(p.ctx_len[b] + 1);
+    const int S = p.seg ? seg_splits(p.seg[b]) : splits_for_rows(p.ctx_len[b] + 1);
     const float2* ml = reinterpret_cast<const float2*>(p.ml + (((size_t)b * p.s_max) * kMaxHeads + j) * 2);
     float* wl = wgt + x * p.s_max;
     // (m, l) of the splits, staged in this thread's weight slots before the reductions
@@ -539,7 +540,7 @@ __global__ void __launch_bounds__(kOProjThreads, 1)
         if (x < n_items) {
           const int b = x / (lay.hib * chunks), h2 = (x / chunks) % lay.hib, ch = x % chunks;
           if (b < p.n_lanes && ((act >> b) & 1)) {
-            S2[q] = splits_for_rows(p.ctx_len[b] + 1);
+            S2[q] = p.seg ? seg_splits(p.seg[b]) : splits_for_rows(p.ctx_len[b] + 1);
             U0[q] = p.U + ((size_t)b * p.s_max * kMaxHeads + mb * lay.hib + h2) * s.d + k * lay.KS + 8 * ch;
             w2[q] = wgt + (b * lay.hib + h2) * p.s_max;
           }
@@ -768,6 +769,7 @@ cudaError_t launch_oproj(const DecodeArgs& a, cudaStream_t st) {
                 w.s_max,
                 reinterpret_cast<const float*>(a.ws + w.ml_off),
                 reinterpret_cast<const float*>(a.ws + w.u_off),
+                a.seg,
                 a.out,
                 reinterpret_cast<uint32_t*>(a.ws + w.status_off),
                 a.residual,

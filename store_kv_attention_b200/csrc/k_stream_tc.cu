@@ -150,6 +150,7 @@ struct StreamParams {
   const uint8_t* qimg;  // [n_lanes][qimg_bytes(d)] absorbed-query operand images
   float* ml;            // [n_lanes][s_max][16][2]
   float* U;             // [n_lanes][s_max][16][d]
+  const LaneSeg* seg;   // rows of each lane (multi-query calls), or NULL: rows 0..ctx_len[b] of lane b
   uint32_t* status;
   int s_max;
   int s_ring, v_ring;   // slots of the score-side and P.V-side rings
@@ -305,15 +306,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int L = p.loops[b], c = p.ctx_len[b];
     if (L < 0 || L > s.L_max || c < 0 || c >= s.max_ctx || p.iter >= L) return;
   }
-  const int n = p.ctx_len[b] + 1;
-  const int r_begin = split * kSplitRows;
-  if (r_begin >= n) return;
-  const int r_end = min(n, r_begin + kSplitRows);
+  // rows of this split: a decode lane's rows 0..ctx_len, or a segment of a multi-query lane
+  const LaneSeg g = p.seg ? p.seg[b] : LaneSeg{b, p.ctx_len[b] + 1, 0, 0};
+  int r_begin, split_rows;
+  if (!seg_split_rows(g, split, &r_begin, &split_rows)) return;
+  const int r_end = r_begin + split_rows;
   const int n_tiles = (r_end - r_begin + 127) >> 7;
   const int n_units = D >> 7;  // even: d is a multiple of 256
   const int n_chunks = D / F::kVals;
   const int layer = s.n_pre + p.iter;
-  const int row_base = (layer * s.max_lanes + b) * s.max_ctx;
+  const int row_base = (layer * s.max_lanes + g.phys) * s.max_ctx;
   const uint32_t qbytes = (uint32_t)(NS * D * 2);
   const int SR = p.s_ring, VR = p.v_ring;
   const int scale_words = D / (2 * kInt4Group);  // INT4: fp16 group scales of a row, two per word
@@ -862,6 +864,7 @@ cudaError_t launch_fmt(const DecodeArgs& a, const CUtensorMap& tmap, cudaStream_
                  a.ws + a.wl.qt_off,
                  reinterpret_cast<float*>(a.ws + a.wl.ml_off),
                  reinterpret_cast<float*>(a.ws + a.wl.u_off),
+                 a.seg,
                  reinterpret_cast<uint32_t*>(a.ws + a.wl.status_off),
                  a.wl.s_max,
                  s_ring,

@@ -65,6 +65,30 @@ __host__ __device__ inline uint32_t kmajor_offset(int row, int pos, int rows) {
 
 __host__ __device__ inline int splits_for_rows(int n_rows) { return (n_rows + kSplitRows - 1) / kSplitRows; }
 
+// Rows a (virtual) lane attends, for multi-query calls (tree verification, chunked prefill):
+// rows [0, n0) and [start1, start1 + n1) of physical lane `phys` in the iteration's layer.
+// Each segment is cut into splits of kSplitRows rows of its own, segment 0's first, so a split
+// is one contiguous run of rows.  A decode lane b is {b, ctx_len[b] + 1, 0, 0}.
+struct LaneSeg {
+  int32_t phys, n0, start1, n1;
+};
+__host__ __device__ inline int seg_splits(const LaneSeg& g) { return splits_for_rows(g.n0) + splits_for_rows(g.n1); }
+// Split `split` of a lane: first row (in the physical lane's row space) and row count; false
+// when the lane has fewer splits.
+__host__ __device__ inline bool seg_split_rows(const LaneSeg& g, int split, int* r_begin, int* n_rows) {
+  const int s0 = splits_for_rows(g.n0);
+  if (split < s0) {
+    *r_begin = split * kSplitRows;
+    *n_rows = g.n0 - *r_begin < kSplitRows ? g.n0 - *r_begin : kSplitRows;
+    return true;
+  }
+  const int s1 = split - s0;
+  if (s1 * kSplitRows >= g.n1) return false;
+  *r_begin = g.start1 + s1 * kSplitRows;
+  *n_rows = g.n1 - s1 * kSplitRows < kSplitRows ? g.n1 - s1 * kSplitRows : kSplitRows;
+  return true;
+}
+
 // ---------------------------------------------------------------- decode-step geometry
 constexpr int kMaxGemmLanes = 64;  // lanes per decode call (projection MMAs with N <= 256, 64-bit lane masks)
 
@@ -95,9 +119,11 @@ struct Workspace {
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-inline Workspace workspace_layout(const Shape& s, int n_lanes) {
+// extra_splits: splits a lane may have beyond those of max_ctx rows in one run (multi-query
+// calls, whose second row segment starts a split of its own).
+inline Workspace workspace_layout(const Shape& s, int n_lanes, int extra_splits = 0) {
   Workspace w;
-  w.s_max = splits_for_rows(s.max_ctx);
+  w.s_max = splits_for_rows(s.max_ctx) + extra_splits;
   w.nb = lanes_padded(n_lanes);
   size_t off = 0;
   w.status_off = off;
@@ -164,6 +190,8 @@ struct DecodeArgs {
   float* norms;
   // append h_new as the new token's row of every active lane first (fused into qproj_kernel)
   bool append = false;
+  // multi-query calls: the rows of each (virtual) lane (device [n_lanes]); NULL = decode lanes
+  const LaneSeg* seg = nullptr;
 };
 
 // Fused q and absorbed-query projections, one thread-block cluster per 128 rows of W_q (k_proj_tc.cu).

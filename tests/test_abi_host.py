@@ -175,3 +175,27 @@ def test_delta_workspace_and_decode_rejected_before_launch(tl):
     assert L.tl_delta_attn_decode(*args(0, 2, ws, res=fake)) == tl.TL_ERR_INVALID_ARG  # residual without flags
     assert L.tl_delta_attn_decode(None, cache, 0, fake, fake, fake, fake, fake, fake, fake, None,
                                   ctypes.c_float(0.0), None, None, None, fake, ws, 2, None) == tl.TL_ERR_INVALID_ARG
+
+
+# --------------------------------------------------------------------------- tree verification, prefill
+def test_verify_and_prefill_rejected_before_launch(tl):
+    L = tl.lib
+    desc = _desc(tl)
+    d = desc.c()
+    fake = ctypes.c_void_p(1 << 20)
+    cache = tl.Cache(1 << 20, 1 << 21)
+    ws = tl.verify_workspace_bytes(desc, 2, 3, 4)
+    assert ws >= tl.workspace_bytes(desc, 24) and ws % 256 == 0
+    args = lambda it, n, K, D, wsb: (ctypes.byref(d), cache, it, fake, fake, fake, K, D, fake, fake, fake, fake, fake,
+                                     wsb, n, None)
+    assert L.tl_storeh_verify_attn(*args(0, 2, 3, 4, ws - 256)) == tl.TL_ERR_CAPACITY   # workspace too small
+    assert L.tl_storeh_verify_attn(*args(8, 2, 3, 4, ws)) == tl.TL_ERR_CAPACITY         # iter >= L_max
+    assert L.tl_storeh_verify_attn(*args(0, 33, 3, 4, ws)) == tl.TL_ERR_CAPACITY        # lanes beyond capacity
+    assert L.tl_storeh_verify_attn(*args(0, 2, 0, 4, ws)) == tl.TL_ERR_INVALID_ARG
+    assert L.tl_storeh_verify_attn(*args(0, 2, 33, 32, ws)) == tl.TL_ERR_UNSUPPORTED    # > 1024 tree tokens
+    nul = (ctypes.byref(d), cache, 0, fake, fake, None, 3, 4, fake, fake, fake, fake, fake, ws, 2, None)
+    assert L.tl_storeh_verify_attn(*nul) == tl.TL_ERR_INVALID_ARG                       # h_tree NULL
+    assert L.tl_storeh_prefill_attn(ctypes.byref(d), cache, 0, fake, fake, fake, 0, fake, fake, fake, fake, fake, ws,
+                                    2, None) == tl.TL_ERR_INVALID_ARG                    # no tokens
+    with pytest.raises(tl.TLError):
+        tl.verify_workspace_bytes(desc, 2, 40, 40)
