@@ -114,14 +114,26 @@ typedef struct {
   void* scales;
 } tl_storeh_cache;
 
-/* Bytes the caller must allocate for the cache described by `desc`.
- * Errors: TL_ERR_INVALID_ARG (NULL), TL_ERR_SHAPE / TL_ERR_UNSUPPORTED (desc). */
+/* Bytes the caller must allocate for the cache described by `desc`: the variable-L cache
+ * holds n_pre + L_max layers [Architecture-Exclusive Features, "Variable-L KV cache"] of
+ * max_lanes x max_ctx rows, each row stored in its mode's size [Architecture-Exclusive
+ * Features, "Store-h KV cache", mode table: D (FP16-h), D/2 + e (INT8-h), D/4 + e (INT4-h)
+ * per K+V pair of fp16 elements; here 2d, d + 4 and d/2 + 2 d/64 bytes, scales in
+ * scales_bytes], laid out as tl_storeh_cache describes.
+ * Errors: TL_ERR_INVALID_ARG (NULL), TL_ERR_SHAPE / TL_ERR_UNSUPPORTED (desc).
+ * tl_storeh_desc.fmt is an int32_t holding a tl_h_format value rather than the enum type,
+ * so that the struct's size and layout do not depend on the compiler's enum width. */
 TL_API tl_status tl_storeh_cache_bytes(const tl_storeh_desc* desc, size_t* codes_bytes, size_t* scales_bytes);
 
 /* Bytes of device workspace tl_storeh_attn_decode needs for up to `n_lanes`
- * lanes (256-byte aligned, contents need no initialisation, must not be shared
- * by two calls in flight at once).  One decode call takes at most 64 lanes
- * (TL_ERR_UNSUPPORTED above); larger batches are split into several calls. */
+ * lanes (256-byte aligned, contents need no initialisation apart from the status
+ * word described at tl_storeh_poll_status, must not be shared by two calls in flight
+ * at once).  It holds, per lane, the absorbed query q_j^T W_k[j] of every head and the
+ * partial softmax results (running max, sum and sum_c p_c h_c) of each 1024-row split
+ * of the lane's context: the absorbed form of the pages' K = W_k h rebuild
+ * [Novel Contributions, "Novel Mechanism: Store-h KV Cache"], split so that the
+ * context of one lane streams on several SMs at once.  One decode call takes at most
+ * 64 lanes (TL_ERR_UNSUPPORTED above); larger batches are split into several calls. */
 TL_API tl_status tl_storeh_workspace_bytes(const tl_storeh_desc* desc, int32_t n_lanes, size_t* bytes);
 
 /*

@@ -458,7 +458,12 @@ __global__ void __launch_bounds__(kOProjThreads, 1)
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
 
-  pdl_wait();  // the split partials come from the streaming kernel just before
+  // This kernel is launched (programmatic dependent launch) only once every CTA of the streaming
+  // kernel has passed its own griddepcontrol.wait, i.e. once the projection kernel before it has
+  // completed, which itself waited for everything enqueued before the decode call.  So the call's
+  // inputs -- W_v, loops / ctx_len, the residual, the sticky flags -- are complete here already;
+  // only the split partials, written by the streaming kernel, need the wait below.  The weight
+  // tiles, the active-lane mask and the safety check therefore overlap the streaming kernel's tail.
   if (threadIdx.x == 0) {
     mbar_init(&bar_ld, 1);
     mbar_init(&bar_m, 1);
@@ -475,7 +480,6 @@ __global__ void __launch_bounds__(kOProjThreads, 1)
   tc_fence_after();
   const uint32_t tbase = tmem_base;
   volatile int* abort_p = &abort_flag;
-  pdl_trigger();  // TMEM is held
 
   if (threadIdx.x == 0) {
     mbar_expect_tx(&bar_ld, (uint32_t)lay.nk * kTileBytes);
@@ -488,6 +492,9 @@ __global__ void __launch_bounds__(kOProjThreads, 1)
   const int nl = mb * CL + k;
   if (p.residual && nl < p.n_lanes && ((act >> nl) & 1))
     norm_check_lane<kOProjThreads>(p.residual, nl, s.d, p.threshold, p.iter, p.flags, p.first, p.norms);
+
+  pdl_wait();     // the split partials come from the streaming kernel just before
+  pdl_trigger();  // TMEM is held
 
   // ---------------------------------------------------------------- merge weights
   for (int x = threadIdx.x; x < p.n_lanes * lay.hib; x += kOProjThreads) {

@@ -47,8 +47,13 @@
 // hi + lo parts (N doubles, which costs nothing at these N), so the scores
 // and P.V carry ~22 bits.
 //
-// INT4 codes are unpacked eight at a time with the magic-number fp16 method
-// (OR the nibble into the mantissa of 1024.0 or 64.0, subtract the bias), which
+// INT4 codes are unpacked eight at a time with the exponent-bias ("magic number")
+// integer-to-fp16 conversion -- an identity of IEEE binary16: a small integer n placed in
+// the low mantissa bits of the fp16 constant 2^k reads as 2^k + n * ulp(2^k), so one lop3
+// (mask, OR the constant, flip the sign bit of the code) and one subtraction give the exact
+// value; the method as used for INT4/INT8 weight dequantisation is described by Kim et al.,
+// "Who Says Elephants Can't Run" (2022, arXiv:2211.10017).  Here the nibble goes into the
+// mantissa of 1024.0 (bits 0-3) or 64.0 (bits 4-7), which
 // yields the pairs (e0,e4),(e1,e5),(e2,e6),(e3,e7) of every 32-bit word; the
 // d-order inside each group of 8 is therefore permuted, identically for H, QT
 // and the rows of U^T, and undone when the partial is written.
