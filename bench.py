@@ -42,6 +42,8 @@ def parse_args():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--cpu-seconds", type=float, default=20.0, help="budget of the CPU-baseline sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--split-rows", type=int, default=0,
+                   help="context rows per split of every decode call (tl_decode_opts.split_rows; 0 = the default 1024)")
     return p.parse_args()
 
 
@@ -309,7 +311,7 @@ def run_ours(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     w = workload_for_rank(args.workload, rank)
-    dw = DeviceWorkload(w, device=f"cuda:{local_rank}")
+    dw = DeviceWorkload(w, device=f"cuda:{local_rank}", split_rows=args.split_rows)
     stream = torch.cuda.current_stream()
 
     def barrier():
@@ -441,7 +443,11 @@ def run_ours(args, rank, world, local_rank):
             "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": DTYPE_OF_FMT[w.fmt] + "-h codes, fp16 tensor operands, fp32 accumulate",
             "data": "synthetic (seeded generator: SplitMix64 + Box-Muller)",
-            "config": workload_config(w, world, {"entry_point": "tl_storeh_append_attn_decode per loop iteration",
+            "config": workload_config(w, world, {"entry_point": ("tl_storeh_append_attn_decode per loop iteration" if not
+                                                                 args.split_rows else
+                                                                 "tl_storeh_decode_ex (append=1, split_rows=%d) per "
+                                                                 "loop iteration" % args.split_rows),
+                                                 "split_rows": args.split_rows or 1024,
                                                  "cached_positions_per_step_per_gpu": pos_step,
                                                  "step_roofline_ms_hbm": step_roofline_ms,
                                                  "ms_per_step_median_of_per_step_events": step_ms_median,

@@ -269,6 +269,44 @@ TL_API tl_status tl_storeh_prefill_attn(const tl_storeh_desc* desc, tl_storeh_ca
                                         tl_stream_t stream);
 
 /*
+ * Options of tl_storeh_decode_ex.  Zero-initialise the struct, then set what is needed.
+ *   append      0: the decode of tl_storeh_attn_decode; 1: tl_storeh_append_attn_decode
+ *               (h_new appended as the new token's row first).
+ *   split_rows  context rows per split: 0 (the default, 1024) or one of 128, 256, 512, 1024.
+ *               Each lane's context is cut into splits of this many rows, each streamed by
+ *               its own CTA and merged exactly at the end.  A lane's result depends only on
+ *               its own rows and on split_rows, never on the other lanes of the call
+ *               [Architecture-Exclusive Features, "L-aware batching": mixed lanes give the
+ *               bits of solo runs], so runs that are compared must use the same value.
+ *               Shorter splits put more SMs on a lane, which pays when the call has few
+ *               lanes or few active lanes (single-sequence decode, the deep iterations of
+ *               an L-aware batch); they write more partial results (16 x d_model fp32 per
+ *               split).  TL_ERR_UNSUPPORTED when the splits of max_ctx rows for n_lanes
+ *               lanes would not fit the merge kernel's shared memory.
+ *   reserved    must be zero.
+ */
+typedef struct {
+  int32_t append;
+  int32_t split_rows;
+  int32_t reserved[7];
+} tl_decode_opts;
+
+/* tl_storeh_workspace_bytes for a call made with these options (NULL = defaults). */
+TL_API tl_status tl_storeh_workspace_bytes_ex(const tl_storeh_desc* desc, int32_t n_lanes, const tl_decode_opts* opts,
+                                              size_t* bytes);
+
+/* tl_storeh_attn_decode / tl_storeh_append_attn_decode with options (see tl_decode_opts);
+ * same arguments, results and errors, the workspace sized by tl_storeh_workspace_bytes_ex
+ * with the same options.  TL_ERR_INVALID_ARG for a bad option. */
+TL_API tl_status tl_storeh_decode_ex(const tl_storeh_desc* desc, tl_storeh_cache cache, int32_t iter,
+                                     const int32_t* loops, const int32_t* ctx_len, const void* h_new,
+                                     const void* W_q, const void* W_k, const void* W_v, float* out,
+                                     const float* residual, float threshold, uint8_t* abort_flags,
+                                     int32_t* first_abort_iter, float* norms_out, void* workspace,
+                                     size_t workspace_bytes, int32_t n_lanes, const tl_decode_opts* opts,
+                                     tl_stream_t stream);
+
+/*
  * Per-iteration safety check [Novel Contributions, "Novel: Per-Iteration
  * Safety Check"; Architecture-Exclusive Features, "Per-iteration safety check"].
  * For every lane b with iter < loops[b] (all lanes when loops is NULL):

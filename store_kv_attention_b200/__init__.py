@@ -37,7 +37,8 @@ EXPORTS = ["tl_storeh_cache_bytes", "tl_storeh_workspace_bytes", "tl_storeh_appe
            "tl_storeh_abi_version", "tl_set_profile", "tl_storeh_attn_decode_static_ws",
            "tl_storeh_append_attn_decode", "tl_storeh_selftest_wait_timeout", "tl_delta_cache_bytes",
            "tl_delta_append", "tl_delta_workspace_bytes", "tl_delta_attn_decode", "tl_storeh_verify_attn",
-           "tl_storeh_verify_workspace_bytes", "tl_storeh_prefill_attn"]
+           "tl_storeh_verify_workspace_bytes", "tl_storeh_prefill_attn", "tl_storeh_decode_ex",
+           "tl_storeh_workspace_bytes_ex"]
 
 
 class TLError(RuntimeError):
@@ -55,6 +56,10 @@ class Desc(ctypes.Structure):
 class Profile(ctypes.Structure):
     _fields_ = [("begin_events", ctypes.POINTER(ctypes.c_void_p)), ("end_events", ctypes.POINTER(ctypes.c_void_p)),
                 ("capacity", ctypes.c_int32), ("recorded", ctypes.c_int32), ("launches", ctypes.c_int64)]
+
+
+class DecodeOpts(ctypes.Structure):
+    _fields_ = [("append", ctypes.c_int32), ("split_rows", ctypes.c_int32), ("reserved", ctypes.c_int32 * 7)]
 
 
 class Cache(ctypes.Structure):
@@ -121,6 +126,11 @@ def _load():
     L.tl_storeh_prefill_attn.argtypes = [P(Desc), Cache, i32, vp, vp, vp, i32, vp, vp, vp, vp, vp, sz, i32, vp]
     L.tl_storeh_prefill_attn.restype = ctypes.c_int
     L.tl_storeh_verify_workspace_bytes.argtypes = [P(Desc), i32, i32, i32, P(sz)]
+    L.tl_storeh_decode_ex.argtypes = [P(Desc), Cache, i32, vp, vp, vp, vp, vp, vp, vp, vp, f32, vp, vp, vp, vp, sz,
+                                      i32, P(DecodeOpts), vp]
+    L.tl_storeh_decode_ex.restype = ctypes.c_int
+    L.tl_storeh_workspace_bytes_ex.argtypes = [P(Desc), i32, P(DecodeOpts), P(sz)]
+    L.tl_storeh_workspace_bytes_ex.restype = ctypes.c_int
     L.tl_storeh_verify_workspace_bytes.restype = ctypes.c_int
     _lib_handle = L
     return L
@@ -178,24 +188,31 @@ def cache_bytes(desc: StoreHDesc):
     return cb.value, sb.value
 
 
-def workspace_bytes(desc: StoreHDesc, n_lanes: int) -> int:
+def workspace_bytes(desc: StoreHDesc, n_lanes: int, split_rows: int = 0) -> int:
+    """tl_storeh_workspace_bytes, or with split_rows != 0 tl_storeh_workspace_bytes_ex."""
     b = ctypes.c_size_t()
-    _check(_load().tl_storeh_workspace_bytes(ctypes.byref(desc.c()), n_lanes, ctypes.byref(b)),
-           "tl_storeh_workspace_bytes")
+    if split_rows:
+        opts = DecodeOpts(0, split_rows)
+        _check(_load().tl_storeh_workspace_bytes_ex(ctypes.byref(desc.c()), n_lanes, ctypes.byref(opts),
+                                                    ctypes.byref(b)), "tl_storeh_workspace_bytes_ex")
+    else:
+        _check(_load().tl_storeh_workspace_bytes(ctypes.byref(desc.c()), n_lanes, ctypes.byref(b)),
+               "tl_storeh_workspace_bytes")
     return b.value
 
 
 class StoreHCache:
     """Device buffers of one cache (torch uint8 tensors) plus a decode workspace."""
 
-    def __init__(self, desc: StoreHDesc, device="cuda", n_lanes: Optional[int] = None):
+    def __init__(self, desc: StoreHDesc, device="cuda", n_lanes: Optional[int] = None, split_rows: int = 0):
         import torch
         self.desc = desc
+        self.split_rows = split_rows
         cb, sb = cache_bytes(desc)
         self.codes = torch.empty(cb, dtype=torch.uint8, device=device)
         self.scales = torch.empty(max(sb, 256), dtype=torch.uint8, device=device) if sb else None
         n = n_lanes or desc.max_lanes
-        self.ws_bytes = workspace_bytes(desc, n)
+        self.ws_bytes = workspace_bytes(desc, n, split_rows)
         self.workspace = torch.zeros(self.ws_bytes, dtype=torch.uint8, device=device)
 
     def c(self) -> Cache:
@@ -281,8 +298,17 @@ def attn_decode(cache: StoreHCache, it: int, loops, ctx_len, h_new, W_q, W_k, W_
                 residual=None, threshold: float = 0.0, abort_flags=None, first_abort_iter=None,
                 norms_out=None, stream=None, append: bool = False) -> None:
     """tl_storeh_attn_decode, or with append=True tl_storeh_append_attn_decode (h_new is first
-    written as the new token's row of every active lane, in the same enqueue)."""
+    written as the new token's row of every active lane, in the same enqueue); through
+    tl_storeh_decode_ex when the cache was made with a split length of its own."""
     n_lanes = int(h_new.shape[0])
+    if cache.split_rows:  # the cache's workspace was sized for this split length: tl_storeh_decode_ex
+        opts = DecodeOpts(1 if append else 0, cache.split_rows)
+        _check(_load().tl_storeh_decode_ex(ctypes.byref(cache.desc.c()), cache.c(), it, _ptr(loops), _ptr(ctx_len),
+                                           _ptr(h_new), _ptr(W_q), _ptr(W_k), _ptr(W_v), _ptr(out), _ptr(residual),
+                                           float(threshold), _ptr(abort_flags), _ptr(first_abort_iter),
+                                           _ptr(norms_out), cache.workspace.data_ptr(), cache.ws_bytes, n_lanes,
+                                           ctypes.byref(opts), _stream(stream)), "tl_storeh_decode_ex")
+        return
     name = "tl_storeh_append_attn_decode" if append else "tl_storeh_attn_decode"
     _check(getattr(_load(), name)(ctypes.byref(cache.desc.c()), cache.c(), it, _ptr(loops), _ptr(ctx_len),
                                   _ptr(h_new), _ptr(W_q), _ptr(W_k), _ptr(W_v), _ptr(out), _ptr(residual),

@@ -406,6 +406,7 @@ struct OProjParams {
   const int32_t* loops;
   const int32_t* ctx_len;
   int n_lanes, nb, cl, s_max;
+  int split;        // context rows per split
   const float* ml;  // [n_lanes][s_max][16][2]
   const float* U;   // [n_lanes][s_max][16][d]
   const LaneSeg* seg;  // rows of each lane (multi-query calls), or NULL: decode lanes
@@ -500,7 +501,7 @@ __global__ void __launch_bounds__(kOProjThreads, 1)
   for (int x = threadIdx.x; x < p.n_lanes * lay.hib; x += kOProjThreads) {
     const int b = x / lay.hib, h2 = x % lay.hib, j = mb * lay.hib + h2;
     if (!((act >> b) & 1)) continue;
-    const int S = p.seg ? seg_splits(p.seg[b]) : splits_for_rows(p.ctx_len[b] + 1);
+    const int S = p.seg ? seg_splits(p.seg[b], p.split) : splits_for_rows(p.ctx_len[b] + 1, p.split);
     const float2* ml = reinterpret_cast<const float2*>(p.ml + (((size_t)b * p.s_max) * kMaxHeads + j) * 2);
     float* wl = wgt + x * p.s_max;
     // (m, l) of the splits, staged in this thread's weight slots before the reductions
@@ -547,7 +548,7 @@ __global__ void __launch_bounds__(kOProjThreads, 1)
         if (x < n_items) {
           const int b = x / (lay.hib * chunks), h2 = (x / chunks) % lay.hib, ch = x % chunks;
           if (b < p.n_lanes && ((act >> b) & 1)) {
-            S2[q] = p.seg ? seg_splits(p.seg[b]) : splits_for_rows(p.ctx_len[b] + 1);
+            S2[q] = p.seg ? seg_splits(p.seg[b], p.split) : splits_for_rows(p.ctx_len[b] + 1, p.split);
             U0[q] = p.U + ((size_t)b * p.s_max * kMaxHeads + mb * lay.hib + h2) * s.d + k * lay.KS + 8 * ch;
             w2[q] = wgt + (b * lay.hib + h2) * p.s_max;
           }
@@ -715,6 +716,11 @@ bool make_tmap_f16(void* tmap, const void* base, uint64_t rows, uint64_t cols, u
 // Cluster size of the projection kernels: K splits of d, each a multiple of 64 wide.
 int proj_cluster(int d) { return d / 64 < 8 ? d / 64 : 8; }
 
+// Dynamic shared memory oproj_kernel needs for a call (its merge weights grow with the splits).
+size_t oproj_smem_bytes(const Shape& s, int n_lanes, int s_max) {
+  return OProjLayout(s, lanes_padded(n_lanes), proj_cluster(s.d), n_lanes, s_max).total;
+}
+
 cudaError_t launch_qproj(const DecodeArgs& a, cudaStream_t st) {
   const Shape& s = a.s;
   const Workspace& w = a.wl;
@@ -774,6 +780,7 @@ cudaError_t launch_oproj(const DecodeArgs& a, cudaStream_t st) {
                 w.nb,
                 CL,
                 w.s_max,
+                w.split,
                 reinterpret_cast<const float*>(a.ws + w.ml_off),
                 reinterpret_cast<const float*>(a.ws + w.u_off),
                 a.seg,

@@ -158,6 +158,7 @@ struct StreamParams {
   const LaneSeg* seg;   // rows of each lane (multi-query calls), or NULL: rows 0..ctx_len[b] of lane b
   uint32_t* status;
   int s_max;
+  int split;            // context rows per split
   int s_ring, v_ring;   // slots of the score-side and P.V-side rings
 };
 
@@ -314,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // rows of this split: a decode lane's rows 0..ctx_len, or a segment of a multi-query lane
   const LaneSeg g = p.seg ? p.seg[b] : LaneSeg{b, p.ctx_len[b] + 1, 0, 0};
   int r_begin, split_rows;
-  if (!seg_split_rows(g, split, &r_begin, &split_rows)) return;
+  if (!seg_split_rows(g, split, p.split, &r_begin, &split_rows)) return;
   const int r_end = r_begin + split_rows;
   const int n_tiles = (r_end - r_begin + 127) >> 7;
   const int n_units = D >> 7;  // even: d is a multiple of 256
@@ -872,6 +873,7 @@ cudaError_t launch_fmt(const DecodeArgs& a, const CUtensorMap& tmap, cudaStream_
                  a.seg,
                  reinterpret_cast<uint32_t*>(a.ws + a.wl.status_off),
                  a.wl.s_max,
+                 a.wl.split,
                  s_ring,
                  v_ring};
   // lanes vary fastest, so every lane's first splits are scheduled before any lane's last

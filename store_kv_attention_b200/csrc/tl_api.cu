@@ -156,7 +156,27 @@ tl_status tl_storeh_cache_bytes(const tl_storeh_desc* desc, size_t* codes_bytes,
   return TL_OK;
 }
 
-tl_status tl_storeh_workspace_bytes(const tl_storeh_desc* desc, int32_t n_lanes, size_t* bytes) {
+// Split length of a call's options (0 = default); TL_OK or an error for a bad value or one whose
+// merge state would not fit the epilogue kernel's shared memory.
+static tl_status check_split(const tl::Shape& s, int32_t n_lanes, const tl_decode_opts* opts, int* split) {
+  *split = tl::kSplitRows;
+  if (opts && opts->split_rows != 0) {
+    if (!tl::valid_split_rows(opts->split_rows))
+      return fail(TL_ERR_INVALID_ARG, "split_rows %d not in {0, 128, 256, 512, 1024}", opts->split_rows);
+    *split = opts->split_rows;
+  }
+  if (opts)
+    for (int i = 0; i < 7; ++i)
+      if (opts->reserved[i] != 0) return fail(TL_ERR_INVALID_ARG, "tl_decode_opts.reserved[%d] is not zero", i);
+  const int s_max = tl::splits_for_rows(s.max_ctx, *split);
+  if (tl::oproj_smem_bytes(s, n_lanes, s_max) > 227u * 1024u)
+    return fail(TL_ERR_UNSUPPORTED, "split_rows %d: %d splits per lane for %d lanes exceed the merge kernel's shared memory",
+                *split, s_max, n_lanes);
+  return TL_OK;
+}
+
+static tl_status workspace_bytes_impl(const tl_storeh_desc* desc, int32_t n_lanes, const tl_decode_opts* opts,
+                                      size_t* bytes) {
   tl::Shape s{};
   tl_status st = check_desc(desc, &s);
   if (st != TL_OK) return st;
@@ -165,8 +185,19 @@ tl_status tl_storeh_workspace_bytes(const tl_storeh_desc* desc, int32_t n_lanes,
   if (n_lanes > s.max_lanes) return fail(TL_ERR_CAPACITY, "n_lanes %d > max_lanes %d", n_lanes, s.max_lanes);
   if (n_lanes > tl::kMaxGemmLanes)
     return fail(TL_ERR_UNSUPPORTED, "n_lanes %d > %d lanes per decode call", n_lanes, tl::kMaxGemmLanes);
-  *bytes = tl::workspace_layout(s, n_lanes).total;
+  int split;
+  if ((st = check_split(s, n_lanes, opts, &split)) != TL_OK) return st;
+  *bytes = tl::workspace_layout(s, n_lanes, 0, split).total;
   return TL_OK;
+}
+
+tl_status tl_storeh_workspace_bytes(const tl_storeh_desc* desc, int32_t n_lanes, size_t* bytes) {
+  return workspace_bytes_impl(desc, n_lanes, nullptr, bytes);
+}
+
+tl_status tl_storeh_workspace_bytes_ex(const tl_storeh_desc* desc, int32_t n_lanes, const tl_decode_opts* opts,
+                                       size_t* bytes) {
+  return workspace_bytes_impl(desc, n_lanes, opts, bytes);
 }
 
 tl_status tl_storeh_append(const tl_storeh_desc* desc, tl_storeh_cache cache, int32_t layer,
@@ -321,7 +352,7 @@ tl_status decode_impl(const tl_storeh_desc* desc, tl_storeh_cache cache, int32_t
                       const int32_t* ctx_len, const void* h_new, const void* W_q, const void* W_k, const void* W_v,
                       float* out, const float* residual, float threshold, uint8_t* abort_flags,
                       int32_t* first_abort_iter, float* norms_out, void* workspace, size_t workspace_bytes,
-                      int32_t n_lanes, tl_stream_t stream, bool append) {
+                      int32_t n_lanes, tl_stream_t stream, bool append, const tl_decode_opts* opts = nullptr) {
   tl::Shape s{};
   tl_status st = check_desc(desc, &s);
   if (st != TL_OK) return st;
@@ -339,7 +370,9 @@ tl_status decode_impl(const tl_storeh_desc* desc, tl_storeh_cache cache, int32_t
   if (residual && (!abort_flags || !first_abort_iter))
     return fail(TL_ERR_INVALID_ARG, "residual given without abort_flags / first_abort_iter");
   if (residual && !(threshold >= 0.0f)) return fail(TL_ERR_INVALID_ARG, "threshold must be a non-negative number");
-  tl::Workspace wl = tl::workspace_layout(s, n_lanes);
+  int split;
+  if ((st = check_split(s, n_lanes, opts, &split)) != TL_OK) return st;
+  tl::Workspace wl = tl::workspace_layout(s, n_lanes, 0, split);
   if (workspace_bytes < wl.total)
     return fail(TL_ERR_CAPACITY, "workspace %zu bytes < %zu needed", workspace_bytes, wl.total);
 
@@ -376,6 +409,18 @@ tl_status tl_storeh_append_attn_decode(const tl_storeh_desc* desc, tl_storeh_cac
                                 int32_t* first_abort_iter, float* norms_out, void* workspace,
                                 size_t workspace_bytes, int32_t n_lanes, tl_stream_t stream) {
   return decode_impl(desc, cache, iter, loops, ctx_len, h_new, W_q, W_k, W_v, out, residual, threshold, abort_flags, first_abort_iter, norms_out, workspace, workspace_bytes, n_lanes, stream, true);
+}
+
+tl_status tl_storeh_decode_ex(const tl_storeh_desc* desc, tl_storeh_cache cache, int32_t iter, const int32_t* loops,
+                              const int32_t* ctx_len, const void* h_new, const void* W_q, const void* W_k,
+                              const void* W_v, float* out, const float* residual, float threshold,
+                              uint8_t* abort_flags, int32_t* first_abort_iter, float* norms_out, void* workspace,
+                              size_t workspace_bytes, int32_t n_lanes, const tl_decode_opts* opts,
+                              tl_stream_t stream) {
+  if (!opts) return fail(TL_ERR_INVALID_ARG, "opts is NULL");
+  if (opts->append != 0 && opts->append != 1) return fail(TL_ERR_INVALID_ARG, "opts->append %d not 0 or 1", opts->append);
+  return decode_impl(desc, cache, iter, loops, ctx_len, h_new, W_q, W_k, W_v, out, residual, threshold, abort_flags,
+                     first_abort_iter, norms_out, workspace, workspace_bytes, n_lanes, stream, opts->append == 1, opts);
 }
 
 tl_status tl_storeh_selftest_wait_timeout(void* workspace, size_t workspace_bytes, int64_t limit_cycles,

@@ -19,7 +19,7 @@ enum : uint32_t {
 
 constexpr int kInt4Group = 64;
 constexpr int kMaxHeads = 16;        // heads are padded to 16 in the kernels
-constexpr int kSplitRows = 1024;     // context rows per split (a function of the lane's own ctx only)
+constexpr int kSplitRows = 1024;     // default context rows per split (a call may choose 128, 256, 512 or 1024)
 constexpr int kMaxCtx = 65536;       // positions per (layer, lane) the kernels support
 constexpr int kMaxSplits = kMaxCtx / kSplitRows;
 
@@ -63,7 +63,10 @@ __host__ __device__ inline uint32_t kmajor_offset(int row, int pos, int rows) {
   return (uint32_t)(a * rows * 128 + row * 128 + ((((c >> 3) ^ (row & 7)) << 4) | ((c & 7) << 1)));
 }
 
-__host__ __device__ inline int splits_for_rows(int n_rows) { return (n_rows + kSplitRows - 1) / kSplitRows; }
+__host__ __device__ inline int splits_for_rows(int n_rows, int split = kSplitRows) { return (n_rows + split - 1) / split; }
+__host__ __device__ inline bool valid_split_rows(int split) {
+  return split == 128 || split == 256 || split == 512 || split == 1024;
+}
 
 // Rows a (virtual) lane attends, for multi-query calls (tree verification, chunked prefill):
 // rows [0, n0) and [start1, start1 + n1) of physical lane `phys` in the iteration's layer.
@@ -72,20 +75,22 @@ __host__ __device__ inline int splits_for_rows(int n_rows) { return (n_rows + kS
 struct LaneSeg {
   int32_t phys, n0, start1, n1;
 };
-__host__ __device__ inline int seg_splits(const LaneSeg& g) { return splits_for_rows(g.n0) + splits_for_rows(g.n1); }
-// Split `split` of a lane: first row (in the physical lane's row space) and row count; false
-// when the lane has fewer splits.
-__host__ __device__ inline bool seg_split_rows(const LaneSeg& g, int split, int* r_begin, int* n_rows) {
-  const int s0 = splits_for_rows(g.n0);
-  if (split < s0) {
-    *r_begin = split * kSplitRows;
-    *n_rows = g.n0 - *r_begin < kSplitRows ? g.n0 - *r_begin : kSplitRows;
+__host__ __device__ inline int seg_splits(const LaneSeg& g, int split) {
+  return splits_for_rows(g.n0, split) + splits_for_rows(g.n1, split);
+}
+// Split `split_idx` of a lane (splits of `split` rows): first row (in the physical lane's row
+// space) and row count; false when the lane has fewer splits.
+__host__ __device__ inline bool seg_split_rows(const LaneSeg& g, int split_idx, int split, int* r_begin, int* n_rows) {
+  const int s0 = splits_for_rows(g.n0, split);
+  if (split_idx < s0) {
+    *r_begin = split_idx * split;
+    *n_rows = g.n0 - *r_begin < split ? g.n0 - *r_begin : split;
     return true;
   }
-  const int s1 = split - s0;
-  if (s1 * kSplitRows >= g.n1) return false;
-  *r_begin = g.start1 + s1 * kSplitRows;
-  *n_rows = g.n1 - s1 * kSplitRows < kSplitRows ? g.n1 - s1 * kSplitRows : kSplitRows;
+  const int s1 = split_idx - s0;
+  if (s1 * split >= g.n1) return false;
+  *r_begin = g.start1 + s1 * split;
+  *n_rows = g.n1 - s1 * split < split ? g.n1 - s1 * split : split;
   return true;
 }
 
@@ -115,15 +120,17 @@ struct Workspace {
   size_t u_off;        // fp32 [n_lanes][S_max][16][d]   per-split unnormalised sum_c p_c h_c
   size_t total;
   int s_max, nb;
+  int split;           // context rows per split
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 // extra_splits: splits a lane may have beyond those of max_ctx rows in one run (multi-query
 // calls, whose second row segment starts a split of its own).
-inline Workspace workspace_layout(const Shape& s, int n_lanes, int extra_splits = 0) {
+inline Workspace workspace_layout(const Shape& s, int n_lanes, int extra_splits = 0, int split = kSplitRows) {
   Workspace w;
-  w.s_max = splits_for_rows(s.max_ctx) + extra_splits;
+  w.split = split;
+  w.s_max = splits_for_rows(s.max_ctx, split) + extra_splits;
   w.nb = lanes_padded(n_lanes);
   size_t off = 0;
   w.status_off = off;
@@ -199,6 +206,7 @@ cudaError_t launch_qproj(const DecodeArgs& a, cudaStream_t st);
 // Fused split merge, value projection and safety check on thread-block clusters (k_proj_tc.cu).
 cudaError_t launch_oproj(const DecodeArgs& a, cudaStream_t st);
 int proj_cluster(int d);
+size_t oproj_smem_bytes(const Shape& s, int n_lanes, int s_max);
 
 // fp16 2D tensor map [rows][cols] (row pitch `pitch_elems`), box [box_cols x box_rows], 128-byte swizzle
 // (k_proj_tc.cu).

@@ -19,11 +19,11 @@ from .workloads import Workload
 
 class DeviceWorkload:
     def __init__(self, w: Workload, device: str = "cuda", flag_mix: bool = False, fill: bool = True,
-                 n_lanes_ws: Optional[int] = None, max_ctx: Optional[int] = None):
+                 n_lanes_ws: Optional[int] = None, max_ctx: Optional[int] = None, split_rows: int = 0):
         self.w = w
         self.device = device
         self.desc = tl.StoreHDesc(w.d, w.H, w.hd, w.n_pre, w.L_max, w.B, max_ctx or w.max_ctx, w.fmt)
-        self.cache = tl.StoreHCache(self.desc, device=device, n_lanes=n_lanes_ws)
+        self.cache = tl.StoreHCache(self.desc, device=device, n_lanes=n_lanes_ws, split_rows=split_rows)
         self.W = {k: self._f16(w.weight(k)).to(device) for k in "qkv"}
         self.loops = torch.tensor(w.loops, dtype=torch.int32, device=device)
         self.ctx = torch.tensor(w.ctx, dtype=torch.int32, device=device)

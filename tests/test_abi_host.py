@@ -199,3 +199,34 @@ def test_verify_and_prefill_rejected_before_launch(tl):
                                     2, None) == tl.TL_ERR_INVALID_ARG                    # no tokens
     with pytest.raises(tl.TLError):
         tl.verify_workspace_bytes(desc, 2, 40, 40)
+
+
+def test_decode_options_rejected_before_launch(tl):
+    L = tl.lib
+    desc = _desc(tl)
+    d = desc.c()
+    fake = ctypes.c_void_p(1 << 20)
+    cache = tl.Cache(1 << 20, 1 << 21)
+    b = ctypes.c_size_t()
+    for split, want in ((0, tl.TL_OK), (128, tl.TL_OK), (512, tl.TL_OK), (100, tl.TL_ERR_INVALID_ARG),
+                        (2048, tl.TL_ERR_INVALID_ARG), (-1, tl.TL_ERR_INVALID_ARG)):
+        opts = tl.DecodeOpts(0, split)
+        assert L.tl_storeh_workspace_bytes_ex(ctypes.byref(d), 4, ctypes.byref(opts), ctypes.byref(b)) == want, split
+    # shorter splits need more partial results
+    assert tl.workspace_bytes(desc, 4, 128) > tl.workspace_bytes(desc, 4, 1024) == tl.workspace_bytes(desc, 4)
+    opts = tl.DecodeOpts(0, 128)
+    opts.reserved[3] = 1
+    assert L.tl_storeh_workspace_bytes_ex(ctypes.byref(d), 4, ctypes.byref(opts), ctypes.byref(b)) == tl.TL_ERR_INVALID_ARG
+    ws = tl.workspace_bytes(desc, 4, 128)
+    args = lambda o, wsb: (ctypes.byref(d), cache, 0, fake, fake, fake, fake, fake, fake, fake, None, 0.0, None, None,
+                           None, fake, wsb, 4, o, None)
+    assert L.tl_storeh_decode_ex(*args(None, ws)) == tl.TL_ERR_INVALID_ARG
+    assert L.tl_storeh_decode_ex(*args(ctypes.byref(tl.DecodeOpts(2, 128)), ws)) == tl.TL_ERR_INVALID_ARG
+    # the default-split workspace is too small for 128-row splits
+    assert L.tl_storeh_decode_ex(*args(ctypes.byref(tl.DecodeOpts(0, 128)), tl.workspace_bytes(desc, 4))) == \
+        tl.TL_ERR_CAPACITY
+    # 65536 positions in splits of 128 rows for 64 lanes: the merge state does not fit
+    big = tl.StoreHDesc(2048, 16, 128, n_pre=1, L_max=2, max_lanes=64, max_ctx=65536, fmt=2)
+    with pytest.raises(tl.TLError) as e:
+        tl.workspace_bytes(big, 64, 128)
+    assert e.value.status == tl.TL_ERR_UNSUPPORTED

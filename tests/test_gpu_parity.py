@@ -450,3 +450,37 @@ def test_device_timeout_is_reported_and_cleared():
     assert tl.poll_status(dw.cache) == tl.TL_OK
     out = dw.out.cpu().numpy()
     _assert_close(out[0, 0], _oracle_lane(w, 0, 0), "after the timeout self-test")
+
+
+# --------------------------------------------------------------------------- per-call split length
+@pytest.mark.parametrize("name,ctx,loops,split", [
+    ("fp16_407m", [2048], [8], 128),
+    ("int8_b16", [0, 255, 1100, 2049], [8, 3, 8, 5], 256),
+    ("int4_mixed", [1, 129, 700, 1024, 2500, 64], [4, 16, 32, 4, 16, 32], 512),
+], ids=["fp16_split128", "int8_split256", "int4_split512"])
+def test_split_rows_option_matches_oracle_and_solo(name, ctx, loops, split):
+    """tl_storeh_decode_ex with a shorter split: outputs against the oracle, flags identical, and
+    each lane bit-identical to its solo run with the same split length (batch independence)."""
+    import store_kv_attention_b200 as tl
+    w = _small(name, ctx, loops)
+    dw = _dw(w, flag_mix=True, split_rows=split)
+    dw.step(fused_append=True)
+    torch.cuda.synchronize()
+    assert tl.poll_status(dw.cache) == tl.TL_OK
+    out = dw.out.cpu().numpy()
+    f = np.zeros(w.B, np.uint8)
+    fi = np.full(w.B, -1, np.int32)
+    its = range(w.L_max) if w.L_max <= 8 else [0, 3, 4, 15, 16, 31]
+    for it in range(w.L_max):
+        for b in range(w.B):
+            if it >= w.loops[b]:
+                assert np.all(np.isnan(out[it, b]))
+            elif it in its:
+                _assert_close(out[it, b], _oracle_lane(w, it, b, form="absorbed"), f"{name} split {split} lane {b} it {it}")
+        f, fi, _ = oracle.cpp.residual_norm_check(w.residual(it, True), w.threshold, it, np.array(w.loops), f, fi)
+    assert np.array_equal(dw.flags.cpu().numpy(), f) and np.array_equal(dw.first.cpu().numpy(), fi)
+    for b in sorted({0, w.B - 1}):
+        solo = _dw(select_lanes(w, [b]), flag_mix=True, split_rows=split, max_ctx=w.max_ctx)
+        solo.step(fused_append=True)
+        torch.cuda.synchronize()
+        assert np.array_equal(out[:, b].view(np.uint32), solo.out[:, 0].cpu().numpy().view(np.uint32)), f"lane {b}"
