@@ -307,6 +307,37 @@ TL_API tl_status tl_storeh_decode_ex(const tl_storeh_desc* desc, tl_storeh_cache
                                      tl_stream_t stream);
 
 /*
+ * RoPE-compatible variant of tl_storeh_attn_decode, for models that put rotary position
+ * embeddings on q and K.  The pages give K = W_k h with no positional encoding [Novel
+ * Contributions, "Novel Mechanism: Store-h KV Cache"]; a rotation between the rebuild and the
+ * score breaks the absorbed form for K, so this call rebuilds K = W_k h explicitly for every
+ * attended row (a dense contraction, on the tensor cores) and rotates it.  Per head j:
+ *   q' = R(ctx_len[b]) q_j,  K'_c = R(c) K_cj,  s_c = q' . K'_c / sqrt(head_dim),
+ *   out[b][j] = sum_c softmax(s)_c V_cj   (V = W_v h, not rotated),
+ * where R(t) rotates the pairs (i, i + head_dim/2), i < head_dim/2, by the angle
+ * t * rope_base^(-2i/head_dim) (the "rotate half" form of rotary embeddings): row c of the
+ * cache sits at position c and the new token's query at its own row, ctx_len[b].
+ * Arguments, results and errors as tl_storeh_attn_decode (the new row already appended), plus
+ *   rope_base  the rotary base (10000 in most models), > 1;
+ *   workspace  tl_storeh_rope_workspace_bytes(desc, n_lanes) bytes, 256-byte aligned, its first
+ *              256 bytes (the status word) zeroed once.
+ * The explicit rebuild costs 2 d_model^2 FLOPs per attended row, head_dim times the absorbed
+ * decode's; this call is compute-bound where tl_storeh_attn_decode is memory-bound.
+ */
+TL_API tl_status tl_storeh_attn_decode_rope(const tl_storeh_desc* desc, tl_storeh_cache cache, int32_t iter,
+                                            const int32_t* loops, const int32_t* ctx_len, const void* h_new,
+                                            const void* W_q, const void* W_k, const void* W_v, float* out,
+                                            const float* residual, float threshold, uint8_t* abort_flags,
+                                            int32_t* first_abort_iter, float* norms_out, float rope_base,
+                                            void* workspace, size_t workspace_bytes, int32_t n_lanes,
+                                            tl_stream_t stream);
+
+/* Workspace bytes of tl_storeh_attn_decode_rope: the decode workspace plus the cos / sin table
+ * of the cache's positions, the rotated queries and the scores (64 bytes per position and lane).
+ * Errors: as tl_storeh_workspace_bytes. */
+TL_API tl_status tl_storeh_rope_workspace_bytes(const tl_storeh_desc* desc, int32_t n_lanes, size_t* bytes);
+
+/*
  * Per-iteration safety check [Novel Contributions, "Novel: Per-Iteration
  * Safety Check"; Architecture-Exclusive Features, "Per-iteration safety check"].
  * For every lane b with iter < loops[b] (all lanes when loops is NULL):

@@ -38,7 +38,7 @@ EXPORTS = ["tl_storeh_cache_bytes", "tl_storeh_workspace_bytes", "tl_storeh_appe
            "tl_storeh_append_attn_decode", "tl_storeh_selftest_wait_timeout", "tl_delta_cache_bytes",
            "tl_delta_append", "tl_delta_workspace_bytes", "tl_delta_attn_decode", "tl_storeh_verify_attn",
            "tl_storeh_verify_workspace_bytes", "tl_storeh_prefill_attn", "tl_storeh_decode_ex",
-           "tl_storeh_workspace_bytes_ex"]
+           "tl_storeh_workspace_bytes_ex", "tl_storeh_attn_decode_rope", "tl_storeh_rope_workspace_bytes"]
 
 
 class TLError(RuntimeError):
@@ -131,6 +131,11 @@ def _load():
     L.tl_storeh_decode_ex.restype = ctypes.c_int
     L.tl_storeh_workspace_bytes_ex.argtypes = [P(Desc), i32, P(DecodeOpts), P(sz)]
     L.tl_storeh_workspace_bytes_ex.restype = ctypes.c_int
+    L.tl_storeh_attn_decode_rope.argtypes = [P(Desc), Cache, i32, vp, vp, vp, vp, vp, vp, vp, vp, f32, vp, vp, vp, f32,
+                                             vp, sz, i32, vp]
+    L.tl_storeh_attn_decode_rope.restype = ctypes.c_int
+    L.tl_storeh_rope_workspace_bytes.argtypes = [P(Desc), i32, P(sz)]
+    L.tl_storeh_rope_workspace_bytes.restype = ctypes.c_int
     L.tl_storeh_verify_workspace_bytes.restype = ctypes.c_int
     _lib_handle = L
     return L
@@ -357,6 +362,27 @@ def prefill_attn(cache: StoreHCache, it: int, loops, ctx_len, h_chunk, W_q, W_k,
                                           _ptr(h_chunk), T, _ptr(W_q), _ptr(W_k), _ptr(W_v), _ptr(out),
                                           _ptr(workspace), int(workspace.numel()), n_lanes, _stream(stream)),
            "tl_storeh_prefill_attn")
+
+
+def rope_workspace_bytes(desc: StoreHDesc, n_lanes: int) -> int:
+    b = ctypes.c_size_t()
+    _check(_load().tl_storeh_rope_workspace_bytes(ctypes.byref(desc.c()), n_lanes, ctypes.byref(b)),
+           "tl_storeh_rope_workspace_bytes")
+    return b.value
+
+
+def attn_decode_rope(cache: StoreHCache, it: int, loops, ctx_len, h_new, W_q, W_k, W_v, out, workspace,
+                     rope_base: float = 10000.0, residual=None, threshold: float = 0.0, abort_flags=None,
+                     first_abort_iter=None, norms_out=None, stream=None) -> None:
+    """tl_storeh_attn_decode_rope: the decode with rotary embeddings on q and K (the new rows
+    already appended); workspace a uint8 device tensor of rope_workspace_bytes."""
+    n_lanes = int(h_new.shape[0])
+    _check(_load().tl_storeh_attn_decode_rope(ctypes.byref(cache.desc.c()), cache.c(), it, _ptr(loops), _ptr(ctx_len),
+                                              _ptr(h_new), _ptr(W_q), _ptr(W_k), _ptr(W_v), _ptr(out),
+                                              _ptr(residual), float(threshold), _ptr(abort_flags),
+                                              _ptr(first_abort_iter), _ptr(norms_out), float(rope_base),
+                                              _ptr(workspace), int(workspace.numel()), n_lanes, _stream(stream)),
+           "tl_storeh_attn_decode_rope")
 
 
 def residual_norm_check(residual, threshold: float, it: int, loops, abort_flags, first_abort_iter,

@@ -22,9 +22,12 @@ cudaError_t launch_delta_append(const DeltaShape& s, void* anchor, void* deltas,
 cudaError_t launch_delta_prep(int iter, int L_max, int max_ctx, int n_lanes, const int32_t* loops,
                               const int32_t* ctx_len, int32_t* wloops, int32_t* dloops, uint32_t* status,
                               cudaStream_t st);
-// h^iter of positions 0..ctx_len[b] of the lanes with dloops[b] = 1 into out [n_lanes][max_ctx][d] fp16.
-cudaError_t launch_delta_rebuild(const DeltaShape& s, const void* anchor, const void* deltas, const void* scales,
-                                 int iter, int n_lanes, const int32_t* ctx_len, const int32_t* dloops, __half* out,
-                                 cudaStream_t st);
+struct Workspace;
+// The decode's streaming stage over the delta cache (k_delta_stream.cu): rows 0..ctx_len[b] of
+// every lane with dloops[b] = 1 rebuilt by the FP32 prefix sum of levels 1..iter, attended with
+// the absorbed-query images of the decode workspace `ws` (layout wl), split partials into ws.
+cudaError_t launch_delta_stream(const DeltaShape& s, const void* anchor, const void* deltas, const void* scales,
+                                int iter, int n_lanes, const int32_t* dloops, const int32_t* ctx_len, uint8_t* ws,
+                                const Workspace& wl, cudaStream_t st);
 
 }  // namespace tl

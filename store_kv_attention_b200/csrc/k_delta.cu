@@ -119,43 +119,6 @@ __global__ void delta_prep_kernel(int iter, int L_max, int max_ctx, int n_lanes,
   dloops[b] = ok && iter < L ? 1 : 0;
 }
 
-// h^iter of positions 0..ctx_len[b] of every lane with dloops[b] = 1, as fp16 rows of a
-// [n_lanes][max_ctx][d] scratch: the FP32 prefix sum (anchor, then deltas 1..iter in order,
-// one rounding per addition) rounded to fp16.
-__global__ void __launch_bounds__(kDThreads)
-    delta_rebuild_kernel(DeltaShape s, const __half* __restrict__ anchor, const int8_t* __restrict__ deltas,
-                         const __half* __restrict__ scales, int iter, const int32_t* __restrict__ ctx_len,
-                         const int32_t* __restrict__ dloops, __half* out) {
-  ptx::pdl_wait();  // the new token's row comes from the writer just before
-  ptx::pdl_trigger();
-  const int p = blockIdx.x, b = blockIdx.y;
-  if (!dloops[b] || p > ctx_len[b]) return;  // ctx_len[b] < max_ctx when dloops[b] = 1
-  const int k0 = threadIdx.x * 16;
-  if (k0 >= s.d) return;
-  const size_t row = (size_t)b * s.max_ctx + (size_t)p;
-  const size_t level_rows = (size_t)s.max_lanes * s.max_ctx;
-  const int head = k0 / s.hd;
-  float acc[16];
-  load16_f32(anchor + row * s.d + k0, acc);
-  for (int i = 1; i <= iter; ++i) {
-    const size_t lr = (size_t)(i - 1) * level_rows + row;
-    const uint4 cv = *reinterpret_cast<const uint4*>(deltas + lr * s.d + k0);
-    const float sc = __half2float(scales[lr * s.H + head]);
-    const int8_t* c = reinterpret_cast<const int8_t*>(&cv);
-#pragma unroll
-    for (int j = 0; j < 16; ++j) acc[j] = __fadd_rn(acc[j], __fmul_rn((float)c[j], sc));
-  }
-  uint32_t w[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const __half2 h2 = __floats2half2_rn(acc[2 * i], acc[2 * i + 1]);
-    w[i] = *reinterpret_cast<const uint32_t*>(&h2);
-  }
-  uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)b * s.max_ctx + p) * s.d + k0);
-  dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-  dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-}
-
 }  // namespace
 
 cudaError_t launch_delta_prep(int iter, int L_max, int max_ctx, int n_lanes, const int32_t* loops,
@@ -171,24 +134,6 @@ cudaError_t launch_delta_prep(int iter, int L_max, int max_ctx, int n_lanes, con
   cfg.numAttrs = 1;
   cudaError_t e = cudaLaunchKernelEx(&cfg, delta_prep_kernel, iter, L_max, max_ctx, n_lanes, loops, ctx_len, wloops,
                                      dloops, status);
-  count_launch();
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
-}
-
-cudaError_t launch_delta_rebuild(const DeltaShape& s, const void* anchor, const void* deltas, const void* scales,
-                                 int iter, int n_lanes, const int32_t* ctx_len, const int32_t* dloops, __half* out,
-                                 cudaStream_t st) {
-  if (n_lanes > 65535) return cudaErrorInvalidValue;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(s.max_ctx, n_lanes, 1);
-  cfg.blockDim = dim3(kDThreads, 1, 1);
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1] = {pdl_attribute()};
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, delta_rebuild_kernel, s, (const __half*)anchor, (const int8_t*)deltas,
-                                     (const __half*)scales, iter, ctx_len, dloops, out);
   count_launch();
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

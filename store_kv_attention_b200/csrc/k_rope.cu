@@ -1,0 +1,344 @@
+// RoPE-compatible variant of store-h decode attention: the scores with rotary position
+// embeddings, on 5th-generation tensor cores (tcgen05 + TMEM), sm_100a.
+// [Novel Contributions, "Novel Mechanism: Store-h KV Cache": K = W_k h rebuilt from the cached
+//  h; the pages give no positional encoding, and this variant applies the standard rotary one]
+//
+// A rotary embedding rotates q and every K row by angles that depend on their positions, between
+// the rebuild K = W_k h and the score, so the absorbed query of the store-h decode no longer
+// applies to K: every attended row needs its K rebuilt explicitly, a dense [rows x d] x [d x d]
+// contraction.  Three kernels:
+//   rope_table_kernel   cos / sin of position * base^(-2i/hd) for i < hd/2, evaluated in FP64
+//                       (full range reduction) and stored as fp32 pairs
+//   rope_query_kernel   q = W_q h_new per lane (fp32), rotated to the query's position and scaled
+//                       by log2(e)/sqrt(hd) (the softmax runs in base 2)
+//   rope_score_kernel   per (lane, 128-row tile, block of up to 512 K columns): K = h W_k^T with
+//                       tcgen05 (A = the tile's rows dequantised into shared memory, B = W_k
+//                       tiles by TMA, D in TMEM), then in the epilogue every row rotates its K by
+//                       its own position and takes the dot product with each head's rotated q
+// The value side is not rotated, so the streaming kernel's P.V stage and the split merge run as
+// in the decode, with these scores given (k_stream_tc.cu, k_proj_tc.cu).
+//
+// Rotary form ("rotate half" pairing): for head vector x at position t and i < hd/2,
+//   x'_i = x_i cos(t theta_i) - x_{i+hd/2} sin(t theta_i),
+//   x'_{i+hd/2} = x_{i+hd/2} cos(t theta_i) + x_i sin(t theta_i),   theta_i = base^(-2i/hd).
+// Row c sits at position c; the query of a lane with ctx_len cached positions at position ctx_len.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "tc_ptx.cuh"
+#include "tl_internal.cuh"
+
+namespace tl {
+namespace {
+
+using namespace ptx;
+
+constexpr int kRThreads = 128;
+constexpr int kATile = 128 * 64 * 2;  // 128 rows x 64 fp16, K-major, 128-byte swizzle
+constexpr long long kRWait = 4000000000ll;
+
+__global__ void rope_table_kernel(int rows, int half, int hd, double base, float2* cs) {
+  ptx::pdl_wait();
+  ptx::pdl_trigger();
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= rows * half) return;
+  const int c = idx / half, i = idx % half;
+  const double theta = pow(base, -2.0 * (double)i / (double)hd);
+  double sn, cn;
+  sincos((double)c * theta, &sn, &cn);
+  cs[idx] = make_float2((float)cn, (float)sn);
+}
+
+// grid (n_heads, n_lanes), block 128: warp w computes rows w, w + 4, ... of the head with the
+// lanes striding over d, then the head is rotated to the lane's query position.
+__global__ void rope_query_kernel(Shape s, int iter, const int32_t* loops, const int32_t* ctx_len,
+                                  const __half* __restrict__ h_new, const __half* __restrict__ Wq, const float2* cs,
+                                  float* qrot) {
+  ptx::pdl_wait();
+  ptx::pdl_trigger();
+  const int j = blockIdx.x, b = blockIdx.y;
+  int nr;
+  if (!lane_active(s, iter, loops, ctx_len, b, &nr)) return;
+  __shared__ float q[128];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const __half* h = h_new + (size_t)b * s.d;
+  for (int m = warp; m < s.hd; m += 4) {
+    const __half* w = Wq + (size_t)(j * s.hd + m) * s.d;
+    float acc = 0.0f;
+    for (int k = lane * 8; k < s.d; k += 256) {
+      const uint4 wv = *reinterpret_cast<const uint4*>(w + k);
+      const uint4 hv = *reinterpret_cast<const uint4*>(h + k);
+      const __half2* w2 = reinterpret_cast<const __half2*>(&wv);
+      const __half2* h2 = reinterpret_cast<const __half2*>(&hv);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 a = __half22float2(w2[i]), c = __half22float2(h2[i]);
+        acc = fmaf(a.x, c.x, acc);
+        acc = fmaf(a.y, c.y, acc);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) q[m] = acc;
+  }
+  __syncthreads();
+  const int half = s.hd / 2;
+  const float scale = 1.4426950408889634f / sqrtf((float)s.hd);
+  const int pos = ctx_len[b];  // the query's position (its own row)
+  for (int i = threadIdx.x; i < half; i += blockDim.x) {
+    const float2 c = cs[(size_t)pos * half + i];
+    const float x1 = q[i], x2 = q[i + half];
+    qrot[(size_t)b * s.d + j * s.hd + i] = (x1 * c.x - x2 * c.y) * scale;
+    qrot[(size_t)b * s.d + j * s.hd + i + half] = (x2 * c.x + x1 * c.y) * scale;
+  }
+}
+
+struct RopeScoreParams {
+  Shape s;
+  int iter;
+  const int32_t* loops;
+  const int32_t* ctx_len;
+  const uint8_t* codes;
+  const uint8_t* scales;
+  const float* qrot;   // [n_lanes][d]
+  const float2* cs;    // [max_ctx][hd/2]
+  float* scores;       // [n_lanes][max_ctx][16]
+  uint32_t* status;
+  int n_pass;          // K columns per CTA (a multiple of hd, at most 512)
+};
+
+// The 64 values [k0, k0 + 64) of one cached row as fp16 pairs into a K-major swizzled A tile.
+// FP16 rows are copied, INT8 codes are converted exactly (the row scale is applied to the
+// scores), INT4 codes are multiplied by their group scale (rounded once to fp16).
+__device__ __forceinline__ void stage_row(const Shape& s, const uint8_t* codes, const uint8_t* scales, size_t row,
+                                          bool valid, int k0, uint8_t* tile, int r) {
+  uint32_t h[32];
+  if (!valid) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) h[i] = 0u;
+  } else if (s.fmt == TL_H_FP16) {
+    const uint4* src = reinterpret_cast<const uint4*>(codes + row * (size_t)(2 * s.d) + 2 * k0);
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+      const uint4 w = __ldg(src + v);
+      h[4 * v] = w.x;
+      h[4 * v + 1] = w.y;
+      h[4 * v + 2] = w.z;
+      h[4 * v + 3] = w.w;
+    }
+  } else if (s.fmt == TL_H_INT8_TOKEN) {
+    const uint4* src = reinterpret_cast<const uint4*>(codes + row * (size_t)s.d + k0);
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const uint4 w = __ldg(src + v);
+      const int8_t* c = reinterpret_cast<const int8_t*>(&w);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const __half2 p = __halves2half2(__int2half_rn(c[2 * i]), __int2half_rn(c[2 * i + 1]));
+        h[8 * v + i] = *reinterpret_cast<const uint32_t*>(&p);
+      }
+    }
+  } else {
+    const uint4* src = reinterpret_cast<const uint4*>(codes + row * (size_t)(s.d / 2) + k0 / 2);
+    const __half sc = reinterpret_cast<const __half*>(scales)[row * (size_t)(s.d / kInt4Group) + k0 / kInt4Group];
+    const __half2 s2 = __halves2half2(sc, sc);
+#pragma unroll
+    for (int v = 0; v < 2; ++v) {
+      const uint4 w = __ldg(src + v);
+      const uint8_t* by = reinterpret_cast<const uint8_t*>(&w);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int lo = (int)(by[i] & 0xF), hi = (int)(by[i] >> 4);
+        const __half2 p = __halves2half2(__int2half_rn(lo >= 8 ? lo - 16 : lo), __int2half_rn(hi >= 8 ? hi - 16 : hi));
+        const __half2 x = __hmul2(p, s2);
+        h[16 * v + i] = *reinterpret_cast<const uint32_t*>(&x);
+      }
+    }
+  }
+#pragma unroll
+  for (int v = 0; v < 8; ++v)
+    *reinterpret_cast<uint4*>(tile + r * 128 + ((v ^ (r & 7)) << 4)) = make_uint4(h[4 * v], h[4 * v + 1], h[4 * v + 2], h[4 * v + 3]);
+}
+
+__device__ __forceinline__ bool block_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  const bool w = mbar_wait(bar, parity, abort, kRWait);
+  return __syncthreads_and(w) != 0;
+}
+
+// grid (tiles of 128 rows, column blocks of n_pass, lanes), block 128 (thread r = tile row r)
+__global__ void __launch_bounds__(kRThreads, 1)
+    rope_score_kernel(const __grid_constant__ CUtensorMap tmWk, const RopeScoreParams p) {
+  const Shape& s = p.s;
+  pdl_wait();
+  const int tile = blockIdx.x, cb = blockIdx.y, b = blockIdx.z;
+  int n;
+  if (!lane_active(s, p.iter, p.loops, p.ctx_len, b, &n)) return;
+  if (tile * 128 >= n) return;
+  const int NP = p.n_pass;
+  const int n_ks = s.d / 64;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
+  uint8_t* A[2] = {base, base + kATile};
+  uint8_t* B[2] = {base + 2 * kATile, base + 2 * kATile + NP * 128};
+  float* qs = reinterpret_cast<float*>(base + 2 * kATile + 2 * NP * 128);  // this block's NP rotated q values
+  __shared__ uint64_t full[2], empty[2], fin;
+  __shared__ uint32_t tmem_base;
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5, r = threadIdx.x;
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(&fin, 1);
+    abort_flag = 0;
+    mbar_fence_init();
+    tma_prefetch_desc(&tmWk);
+  }
+  if (warp == 0) {
+    tmem_alloc(&tmem_base, NP <= 256 ? 256 : 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = tmem_base;
+  volatile int* abort_p = &abort_flag;
+  pdl_trigger();  // TMEM is held
+
+  for (int i = threadIdx.x; i < NP; i += kRThreads) qs[i] = p.qrot[(size_t)b * s.d + cb * NP + i];
+  const int row = tile * 128 + r;
+  const bool valid = row < n;
+  const size_t grow = ((size_t)(s.n_pre + p.iter) * s.max_lanes + b) * s.max_ctx + (size_t)row;
+  const uint32_t idesc = idesc_f16_f32(128, 256, false, false);
+  bool ok = true, issued = false;
+  for (int ks = 0; ks < n_ks && ok; ++ks) {
+    const int st = ks & 1, use = ks >> 1;
+    if (ks >= 2 && !(ok = block_wait(&empty[st], (use - 1) & 1, abort_p))) break;
+    if (threadIdx.x == 0) {
+      mbar_expect_tx(&full[st], (uint32_t)NP * 128);
+      for (int nb = 0; nb < NP / 128; ++nb)
+        tma_load_2d(B[st] + nb * 16384, &tmWk, ks * 64, cb * NP + nb * 128, &full[st]);
+    }
+    stage_row(s, p.codes, p.scales, grow, valid, ks * 64, A[st], r);
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (warp == 0) {
+      const bool got = __all_sync(0xffffffffu, mbar_wait(&full[st], use & 1, abort_p, kRWait));
+      if (got) {
+        tc_fence_after();
+        if (elect_one()) {
+          const uint64_t ad = sdesc_sw128(smem_addr(A[st]), 16, 1024);
+          for (int nh = 0; nh < NP / 256 + (NP % 256 ? 1 : 0); ++nh) {
+            const uint64_t bd = sdesc_sw128(smem_addr(B[st] + nh * 256 * 128), 16, 1024);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ss(tbase + nh * 256, ad + (uint64_t)((kk * 32) >> 4), bd + (uint64_t)((kk * 32) >> 4), idesc,
+                     (ks | kk) != 0);
+          }
+          mma_commit(&empty[st]);
+        }
+        __syncwarp();
+      }
+    }
+    issued = true;
+    ok = __syncthreads_and(!*abort_p) != 0;
+  }
+  // the last K-step's MMAs complete on empty[(n_ks - 1) & 1]
+  if (ok) ok = block_wait(&empty[(n_ks - 1) & 1], ((n_ks - 1) >> 1) & 1, abort_p);
+
+  if (ok) {
+    // every thread of a warp runs the TMEM loads (they are warp-collective); rows past the
+    // lane's end read position 0's angles and store nothing
+    tc_fence_after();
+    const int half = s.hd / 2;
+    const float2* cs = p.cs + (size_t)(valid ? row : 0) * half;
+    const float sr = (s.fmt == TL_H_INT8_TOKEN && valid) ? reinterpret_cast<const float*>(p.scales)[grow] : 1.0f;
+    for (int h = 0; h < NP / s.hd; ++h) {
+      float acc = 0.0f;
+      for (int i0 = 0; i0 < half; i0 += 16) {
+        uint32_t k1[16], k2[16];
+        tmem_ld16(tbase + lane_off + h * s.hd + i0, k1);
+        tmem_ld16(tbase + lane_off + h * s.hd + half + i0, k2);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float2 c = cs[i0 + i];
+          const float a1 = __uint_as_float(k1[i]), a2 = __uint_as_float(k2[i]);
+          const float r1 = a1 * c.x - a2 * c.y, r2 = a2 * c.x + a1 * c.y;
+          acc = fmaf(qs[h * s.hd + i0 + i], r1, acc);
+          acc = fmaf(qs[h * s.hd + half + i0 + i], r2, acc);
+        }
+      }
+      const int j = (cb * NP) / s.hd + h;
+      if (valid) p.scores[((size_t)b * s.max_ctx + row) * kMaxHeads + j] = acc * sr;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && abort_flag) atomicOr(p.status, kStatusTimeout);
+  if (warp == 0) {
+    if (issued && !ok) {
+      // an abandoned pipeline: nothing may still be writing TMEM when it is freed
+      if (elect_one()) mma_commit(&fin);  // arrives once every MMA this warp issued is done
+      __syncwarp();
+      const long long t0 = clock64();
+      while (!mbar_try_wait(&fin, 0) && clock64() - t0 < kRWait) {
+      }
+    }
+    tc_fence_after();
+    tmem_dealloc(tbase, NP <= 256 ? 256 : 512);
+  }
+}
+
+}  // namespace
+
+bool make_tmap_f16(void* tmap, const void* base, uint64_t rows, uint64_t cols, uint64_t pitch_elems,
+                   uint32_t box_cols, uint32_t box_rows);
+
+int rope_pass_cols(const Shape& s) { return s.d < 512 ? s.d : 512; }
+
+cudaError_t launch_rope_scores(const DecodeArgs& a, float rope_base, float2* cs, float* qrot, float* scores,
+                               cudaStream_t st) {
+  const Shape& s = a.s;
+  const int half = s.hd / 2;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1] = {pdl_attribute()};
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cfg.stream = st;
+  // 1. the cos / sin table of every position of the cache
+  cfg.gridDim = dim3((unsigned)((s.max_ctx * half + 255) / 256), 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, rope_table_kernel, s.max_ctx, half, s.hd, (double)rope_base, cs);
+  count_launch();
+  if (e != cudaSuccess) return e;
+  // 2. the rotated queries
+  cfg.gridDim = dim3(s.H, a.n_lanes, 1);
+  cfg.blockDim = dim3(128, 1, 1);
+  e = cudaLaunchKernelEx(&cfg, rope_query_kernel, s, a.iter, a.loops, a.ctx_len, a.h_new, a.Wq, (const float2*)cs, qrot);
+  count_launch();
+  if (e != cudaSuccess) return e;
+  // 3. the scores: K rebuilt on the tensor cores, rotated and dotted in the epilogue
+  const int NP = rope_pass_cols(s);
+  alignas(64) CUtensorMap tmWk;
+  if (!make_tmap_f16(&tmWk, a.Wk, s.d, s.d, s.d, 64, 128)) return cudaErrorInvalidValue;
+  const size_t smem = 1024 + 2 * (size_t)kATile + 2 * (size_t)NP * 128 + (size_t)NP * 4;
+  e = cudaFuncSetAttribute(rope_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  RopeScoreParams p{s, a.iter, a.loops, a.ctx_len, (const uint8_t*)a.codes, (const uint8_t*)a.scales, qrot,
+                    (const float2*)cs, scores, reinterpret_cast<uint32_t*>(a.ws + a.wl.status_off), NP};
+  cfg.gridDim = dim3((unsigned)((s.max_ctx + 127) / 128), (unsigned)(s.d / NP), (unsigned)a.n_lanes);
+  cfg.blockDim = dim3(kRThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  e = cudaLaunchKernelEx(&cfg, rope_score_kernel, tmWk, p);
+  count_launch();
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace tl

@@ -156,6 +156,10 @@ struct StreamParams {
   float* ml;            // [n_lanes][s_max][16][2]
   float* U;             // [n_lanes][s_max][16][d]
   const LaneSeg* seg;   // rows of each lane (multi-query calls), or NULL: rows 0..ctx_len[b] of lane b
+  // Scores given (RoPE variant): fp32 [n_lanes][max_ctx][16], already in the base-2 units of the
+  // softmax (and with the INT8 row scale applied).  The score ring and the score MMAs are then
+  // not used; NULL = the scores are computed here from the absorbed-query images.
+  const float* scores;
   uint32_t* status;
   int s_max;
   int split;            // context rows per split
@@ -382,7 +386,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   volatile int* s_issued_p = &s_issued;
   const int total_chunks = n_tiles * n_chunks;
-  if (warp == 0) {
+  if (warp == 0 && p.scores) {
+    // scores given: no score-side loads; the P.V side may load every chunk
+    if (lane == 0) *s_issued_p = total_chunks;
+  } else if (warp == 0) {
     // ------------------------------------------------------------ TMA producer, score-side ring
     if (lane == 0) {
       // the lane's absorbed-query operand image, straight into place
@@ -431,6 +438,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       drain_ring<FMT>(bars.v_full, VR, g);
     }
+  } else if (warp == 1 && p.scores) {
+    // scores given: no score MMAs
   } else if (warp == 1) {
     // ------------------------------------------------------------ score-MMA issuer
     // The whole warp runs the loop, so descriptors and TMEM addresses stay warp-uniform, and one
@@ -558,7 +567,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ------------------------------------------------ this half's units of tile t -> TMEM staging
       // Rows past the lane's end are not zeroed: a score row depends on its own operand row
       // only, and its score is masked to -inf below.
-      for (int u = half; u < n_units; u += 2) {
+      for (int u = half; u < n_units && !p.scores; u += 2) {
         const uint32_t sw = (FMT == TL_H_INT4_G64 && valid) ? __ldg(srow + u) : 0u;  // groups 2u | 2u+1
         const int k_use = t * (n_units >> 1) + (u >> 1);
         const uint32_t ta = tbase + lane_off + kColStg + half * 64;
@@ -615,22 +624,29 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       // ------------------------------------------------ online softmax of tile t, this half's heads
       const int sb = t & 1;
-      if (!mbar_wait(&bars.sc_full[sb], (t >> 1) & 1, abort_p, kWaitLimit)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t sv[16];
-      tmem_ld8(tbase + lane_off + kColS + sb * 32 + h0, sv);
-      if (NS == 32) tmem_ld8(tbase + lane_off + kColS + sb * 32 + 16 + h0, sv + 8);
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.sc_empty[sb]);
       float sc[8];
+      if (p.scores) {
+        // scores given: this row's scores of this half's heads (padded heads read as 0)
+        const float* srow_s = p.scores + ((size_t)b * s.max_ctx + (r_begin + t * 128 + r)) * kMaxHeads + h0;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        float v = __uint_as_float(sv[j]);
-        if (NS == 32) v += __uint_as_float(sv[8 + j]);
-        if (FMT == TL_H_INT8_TOKEN) v *= scale_row;
-        sc[j] = valid ? v : -CUDART_INF_F;
+        for (int j = 0; j < 8; ++j) sc[j] = valid ? (h0 + j < s.H ? srow_s[j] : 0.0f) : -CUDART_INF_F;
+      } else {
+        if (!mbar_wait(&bars.sc_full[sb], (t >> 1) & 1, abort_p, kWaitLimit)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t sv[16];
+        tmem_ld8(tbase + lane_off + kColS + sb * 32 + h0, sv);
+        if (NS == 32) tmem_ld8(tbase + lane_off + kColS + sb * 32 + 16 + h0, sv + 8);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.sc_empty[sb]);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          float v = __uint_as_float(sv[j]);
+          if (NS == 32) v += __uint_as_float(sv[8 + j]);
+          if (FMT == TL_H_INT8_TOKEN) v *= scale_row;
+          sc[j] = valid ? v : -CUDART_INF_F;
+        }
       }
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
@@ -871,6 +887,7 @@ cudaError_t launch_fmt(const DecodeArgs& a, const CUtensorMap& tmap, cudaStream_
                  reinterpret_cast<float*>(a.ws + a.wl.ml_off),
                  reinterpret_cast<float*>(a.ws + a.wl.u_off),
                  a.seg,
+                 a.scores,
                  reinterpret_cast<uint32_t*>(a.ws + a.wl.status_off),
                  a.wl.s_max,
                  a.wl.split,

@@ -63,22 +63,22 @@ tl_status check_delta_desc(const tl_delta_desc* d, tl::DeltaShape* s) {
   return TL_OK;
 }
 
-// A delta decode runs the store-h FP16 decode on a one-layer scratch cache of the rebuilt rows:
-// shape of that cache, and the workspace layout [decode workspace | wloops | dloops | scratch].
+// A delta decode uses the store-h decode's projection kernels with the rows in natural d order
+// (the FP16 layout): the shape they see (one loop iteration, the lane's 0/1 flag as its loop
+// count) and the workspace layout [decode workspace | wloops | dloops].
 tl::Shape delta_view_shape(const tl::DeltaShape& s, int n_lanes) {
   return tl::Shape{s.d, s.H, s.hd, 0, 1, n_lanes, s.max_ctx, TL_H_FP16};
 }
 struct DeltaWorkspace {
   tl::Workspace wl;
-  size_t wloops_off, dloops_off, scratch_off, total;
+  size_t wloops_off, dloops_off, total;
 };
 DeltaWorkspace delta_workspace(const tl::DeltaShape& s, int n_lanes) {
   DeltaWorkspace w;
   w.wl = tl::workspace_layout(delta_view_shape(s, n_lanes), n_lanes);
   w.wloops_off = tl::align256(w.wl.total);
   w.dloops_off = w.wloops_off + tl::align256((size_t)n_lanes * 4);
-  w.scratch_off = w.dloops_off + tl::align256((size_t)n_lanes * 4);
-  w.total = w.scratch_off + tl::align256((size_t)n_lanes * s.max_ctx * s.d * 2);
+  w.total = w.dloops_off + tl::align256((size_t)n_lanes * 4);
   return w;
 }
 
@@ -305,25 +305,27 @@ tl_status tl_delta_attn_decode(const tl_delta_desc* desc, tl_delta_cache cache, 
   uint8_t* ws = (uint8_t*)workspace;
   int32_t* wloops = (int32_t*)(ws + w.wloops_off);
   int32_t* dloops = (int32_t*)(ws + w.dloops_off);
-  __half* scratch = (__half*)(ws + w.scratch_off);
   cudaStream_t cs = (cudaStream_t)stream;
   // 1. per-lane checks; 2. the new token's state of this iteration into the delta cache;
-  // 3. h^iter of every attended position into the scratch; 4. the FP16 decode over it;
-  // 5. the safety check with the real iteration
+  // 3. q and the absorbed-query images; 4. the streaming stage, whose dequantisation is the FP32
+  // prefix sum of the anchor and the deltas 1..iter; 5. the split merge and W_v; 6. the safety
+  // check with the real iteration
   cudaError_t e = tl::launch_delta_prep(iter, s.L_max, s.max_ctx, n_lanes, loops, ctx_len, wloops, dloops,
                                         (uint32_t*)(ws + w.wl.status_off), cs);
   if (e == cudaSuccess)
     e = tl::launch_delta_append(s, cache.anchor, cache.deltas, cache.scales, iter, (const __half*)h_new, n_lanes, 1,
                                 ctx_len, wloops, cs);
-  if (e == cudaSuccess)
-    e = tl::launch_delta_rebuild(s, cache.anchor, cache.deltas, cache.scales, iter, n_lanes, ctx_len, dloops, scratch,
-                                 cs);
   if (e != cudaSuccess) return cuda_fail(e, "delta decode prologue launch");
-  tl::DecodeArgs a{delta_view_shape(s, n_lanes), scratch, nullptr, 0, dloops, ctx_len, (const __half*)h_new,
+  tl::DecodeArgs a{delta_view_shape(s, n_lanes), nullptr, nullptr, 0, dloops, ctx_len, (const __half*)h_new,
                    (const __half*)W_q, (const __half*)W_k, (const __half*)W_v, out, n_lanes, ws, w.wl,
                    nullptr, 0.0f, nullptr, nullptr, nullptr};
   e = tl::launch_qproj(a, cs);
-  if (e == cudaSuccess) e = tl::launch_stream(a, cs);
+  if (e == cudaSuccess) {
+    tl::profile_stream_begin(cs);
+    e = tl::launch_delta_stream(s, cache.anchor, cache.deltas, cache.scales, iter, n_lanes, dloops, ctx_len, ws, w.wl,
+                                cs);
+    tl::profile_stream_end(cs);
+  }
   if (e == cudaSuccess) e = tl::launch_oproj(a, cs);
   if (e == cudaSuccess && residual)
     e = tl::launch_norm_check(residual, n_lanes, s.d, threshold, iter, wloops, abort_flags, first_abort_iter,

@@ -199,6 +199,8 @@ struct DecodeArgs {
   bool append = false;
   // multi-query calls: the rows of each (virtual) lane (device [n_lanes]); NULL = decode lanes
   const LaneSeg* seg = nullptr;
+  // RoPE variant: scores computed before the streaming kernel (device fp32 [n_lanes][max_ctx][16])
+  const float* scores = nullptr;
 };
 
 // Fused q and absorbed-query projections, one thread-block cluster per 128 rows of W_q (k_proj_tc.cu).
@@ -213,6 +215,10 @@ size_t oproj_smem_bytes(const Shape& s, int n_lanes, int s_max);
 bool make_tmap_f16(void* tmap, const void* base, uint64_t rows, uint64_t cols, uint64_t pitch_elems,
                    uint32_t box_cols, uint32_t box_rows);
 cudaError_t launch_stream(const DecodeArgs& a, cudaStream_t st);
+// RoPE variant (k_rope.cu): cos / sin table [max_ctx][hd/2], rotated queries [n_lanes][d] and the
+// scores [n_lanes][max_ctx][16] the streaming kernel then takes (DecodeArgs::scores).
+cudaError_t launch_rope_scores(const DecodeArgs& a, float rope_base, float2* cs, float* qrot, float* scores,
+                               cudaStream_t st);
 // Self-test of the timeout path: one wait that cannot complete, bounded by limit_cycles (k_selftest.cu).
 cudaError_t launch_wait_selftest(uint32_t* status, long long limit_cycles, cudaStream_t st);
 

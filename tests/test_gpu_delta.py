@@ -98,14 +98,14 @@ def _weights(seed, d):
     return [synth.normal_f16(seed, 40 + i, 0, d * d, scale=1.0 / np.sqrt(d)).reshape(d, d) for i in range(3)]
 
 
-# The decode rounds the rebuilt rows to fp16 before the store-h FP16 decode runs over them, an
-# error the exact rebuild does not have.  At d = 1024 it was measured at max-abs 2.22e-3
-# (iteration 2, lane 0; typical elements 1.5e-4 to 6e-4), over the 2e-3 bar.  The case stays
-# in the suite, marked, until the rebuild keeps its FP32 precision into the operands.
+# The streaming stage rebuilds every attended row by the FP32 prefix sum and feeds it to the
+# tensor cores as fp16 hi + lo parts, so the outputs carry the FP32 rebuild.  (The earlier
+# composition rounded the rebuilt rows to fp16 first and missed the bar at d = 1024.)
 @pytest.mark.parametrize("d,H,L_max,ctx,max_ctx", [
     (256, 4, 3, [150, 37], 200),
-    pytest.param(1024, 16, 3, [500, 64], 600, marks=pytest.mark.xfail(
-        reason="fp16 rounding of the rebuilt rows: max-abs 2.22e-3 > 2e-3 measured", strict=True)),
+    (1024, 16, 3, [500, 64], 600),
+    (1024, 16, 8, [1030, 5], 1100),      # deep levels, a context over two splits
+    (2048, 16, 4, [1100, 300], 1200),    # the 2B-like shape
 ])
 def test_decode_matches_oracle(d, H, L_max, ctx, max_ctx):
     import oracle
