@@ -10,17 +10,19 @@
 // deltas of levels 1..iter (each product code * scale is exact in fp32, each addition rounded
 // to fp32, in level order).  The fp32 result x is split into two fp16 operands
 // hi = fp16(x), lo = fp16(x - hi), about 22 significant bits together, so the tensor cores see
-// the FP32 rebuild rather than an fp16 rounding of it; every MMA is issued twice, once per
-// part, into the same fp32 accumulators.
+// the FP32 rebuild rather than an fp16 rounding of it; every MMA is issued once per part into
+// the same fp32 accumulators.  The other operands are split the same way at every d_model: the
+// absorbed query image has hi and lo rows (qproj writes 32 rows for this call), and P is
+// written as hi and lo rows that two N = 16 MMAs accumulate into the same U^T columns.
 //
 // The absorbed form is that of the store-h decode (k_stream_tc.cu): per head j the scores
 // s_cj = qt_j . h_c with the absorbed query image written by qproj_kernel, an online base-2
 // softmax, U_j = sum_c p_cj h_c accumulated as U^T in TMEM, and the (m, l, U) partial of the
 // split in the workspace layout that oproj_kernel merges.  Per tile:
 //   score pass: for each 128-value unit, rebuild -> hi / lo into TMEM -> 2 x 8 TS MMAs into S
-//   softmax:    S -> P (fp16, hi / lo when d <= 1024), lazy rescale of U^T
+//   softmax:    S -> P (fp16 hi / lo), lazy rescale of U^T
 //   P.V pass:   for each unit, rebuild again -> hi / lo into shared memory (MN-major) ->
-//               2 x 8 SS MMAs into U^T
+//               4 x 8 SS MMAs (h hi / lo times P hi / lo) into U^T
 // The passes run one after the other in all four warps (no warp specialisation): the delta
 // cache reads (1 + iter) rows per position, and this kernel is written for clarity of the
 // rebuild first.  Every wait is bounded; on expiry the kernel records a timeout in the status
@@ -48,7 +50,7 @@ struct DeltaStreamParams {
   const __half* anchor;         // [max_lanes][max_ctx][d]
   const int8_t* deltas;         // [L_max-1][max_lanes][max_ctx][d]
   const __half* scales;         // [L_max-1][max_lanes][max_ctx][H]
-  const uint8_t* qimg;          // [n_lanes][qimg_bytes(d)] absorbed-query operand images
+  const uint8_t* qimg;          // [n_lanes][32 x d] absorbed-query operand images, hi and lo rows
   float* ml;                    // [n_lanes][s_max][16][2]
   float* U;                     // [n_lanes][s_max][16][d]
   uint32_t* status;
@@ -113,10 +115,10 @@ __device__ __forceinline__ bool block_wait(uint64_t* bar, uint32_t parity, volat
   return __syncthreads_and(w) != 0;
 }
 
-template <bool SPLIT>
 __global__ void __launch_bounds__(kDSThreads, 1) delta_stream_kernel(const DeltaStreamParams p) {
-  constexpr int NS = SPLIT ? 32 : 16;
-  constexpr int NP = SPLIT ? 32 : 16;
+  constexpr int NS = 32;  // query image rows: hi (0-15) and lo (16-31) of each head
+  constexpr int NP = 16;  // U^T columns per unit (P hi and lo accumulate into the same ones)
+  constexpr int PR = 32;  // P rows: hi (0-15) and lo (16-31)
   constexpr uint32_t kIdS = idesc_f16_f32(128, NS, false, false);
   constexpr uint32_t kIdP = idesc_f16_f32(128, NP, true, false);
   // TMEM columns: S at 0, the score operand's hi / lo staging at 64 / 128, U^T at 256
@@ -139,7 +141,7 @@ __global__ void __launch_bounds__(kDSThreads, 1) delta_stream_kernel(const Delta
   uint8_t* qs = base;                        // NS x D fp16, K-major swizzled (the qproj image)
   uint8_t* pv_hi = qs + qbytes;              // one unit, hi part, MN-major
   uint8_t* pv_lo = pv_hi + kStageBytes;      // one unit, lo part
-  uint8_t* ps = pv_lo + kStageBytes;         // NP x 128 fp16, K-major swizzled
+  uint8_t* ps = pv_lo + kStageBytes;         // PR x 128 fp16, K-major swizzled
   __shared__ uint64_t bar_q, bar_mma;
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
@@ -248,12 +250,10 @@ __global__ void __launch_bounds__(kDSThreads, 1) delta_stream_kernel(const Delta
       tmem_ld_wait();
 #pragma unroll
       for (int j = 0; j < 16; ++j) sc[j] = __uint_as_float(v[j]);
-      if (NS == 32) {
-        tmem_ld16(tbase + lane_off + kColS + 16, v);
-        tmem_ld_wait();
+      tmem_ld16(tbase + lane_off + kColS + 16, v);
+      tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 16; ++j) sc[j] += __uint_as_float(v[j]);
-      }
+      for (int j = 0; j < 16; ++j) sc[j] += __uint_as_float(v[j]);
     }
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
@@ -289,21 +289,19 @@ __global__ void __launch_bounds__(kDSThreads, 1) delta_stream_kernel(const Delta
       // the P.V MMAs of the earlier tiles are complete (each was waited for)
       for (int u = 0; u < n_units; ++u) {
         uint32_t uv[16];
-        for (int h = 0; h < NP; h += 16) {
-          tmem_ld16(tbase + lane_off + kColU + u * NP + h, uv);
-          tmem_ld_wait();
+        tmem_ld16(tbase + lane_off + kColU + u * NP, uv);
+        tmem_ld_wait();
 #pragma unroll
-          for (int c = 0; c < 16; ++c) uv[c] = __float_as_uint(__uint_as_float(uv[c]) * alpha[c]);
-          tmem_st16(tbase + lane_off + kColU + u * NP + h, uv);
-        }
+        for (int c = 0; c < 16; ++c) uv[c] = __float_as_uint(__uint_as_float(uv[c]) * alpha[c]);
+        tmem_st16(tbase + lane_off + kColU + u * NP, uv);
       }
       tmem_st_wait();
     }
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       const __half hi = __float2half_rn(pr[j]);
-      *reinterpret_cast<__half*>(ps + kmajor_offset(j, r, NP)) = hi;
-      if (NP == 32) *reinterpret_cast<__half*>(ps + kmajor_offset(16 + j, r, NP)) = __float2half_rn(pr[j] - __half2float(hi));
+      *reinterpret_cast<__half*>(ps + kmajor_offset(j, r, PR)) = hi;
+      *reinterpret_cast<__half*>(ps + kmajor_offset(16 + j, r, PR)) = __float2half_rn(pr[j] - __half2float(hi));
     }
 
     // ---------------------------------------------------------------- P.V pass
@@ -331,12 +329,17 @@ __global__ void __launch_bounds__(kDSThreads, 1) delta_stream_kernel(const Delta
           const uint32_t du = tbase + kColU + u * NP;
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
-            const uint64_t pk = p_desc + (uint64_t)((((k * 16) >> 6) * NP * 128 + ((k * 16) & 63) * 2) >> 4);
+            // P rows of K-step k: hi at rows 0-15, lo 16 rows (2048 bytes) further
+            const uint64_t pk = p_desc + (uint64_t)((((k * 16) >> 6) * PR * 128 + ((k * 16) & 63) * 2) >> 4);
+            const uint64_t pl = pk + (uint64_t)(2048 >> 4);
+            const uint64_t ah = hi_desc + (uint64_t)((k * 2048) >> 4), al = lo_desc + (uint64_t)((k * 2048) >> 4);
             if (t == 0 && k == 0)
-              mma_ss_first(du, hi_desc, pk, kIdP);
+              mma_ss_first(du, ah, pk, kIdP);
             else
-              mma_ss_acc(du, hi_desc + (uint64_t)((k * 2048) >> 4), pk, kIdP);
-            mma_ss_acc(du, lo_desc + (uint64_t)((k * 2048) >> 4), pk, kIdP);
+              mma_ss_acc(du, ah, pk, kIdP);
+            mma_ss_acc(du, ah, pl, kIdP);
+            mma_ss_acc(du, al, pk, kIdP);
+            mma_ss_acc(du, al, pl, kIdP);
           }
           mma_commit(&bar_mma);
         }
@@ -350,17 +353,13 @@ __global__ void __launch_bounds__(kDSThreads, 1) delta_stream_kernel(const Delta
   if (ok) {
     const size_t part = (size_t)b * p.s_max + split;
     for (int u = 0; u < n_units; ++u) {
-      uint32_t uv[16], ul[16];
+      uint32_t uv[16];
       tmem_ld16(tbase + lane_off + kColU + u * NP, uv);
-      if (NP == 32) tmem_ld16(tbase + lane_off + kColU + u * NP + 16, ul);
       tmem_ld_wait();
       const int d = u * 128 + r;
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        float v = __uint_as_float(uv[j]);
-        if (NP == 32) v += __uint_as_float(ul[j]);
-        if (j < s.H) p.U[(part * kMaxHeads + j) * D + d] = v;
-      }
+      for (int j = 0; j < 16; ++j)
+        if (j < s.H) p.U[(part * kMaxHeads + j) * D + d] = __uint_as_float(uv[j]);
     }
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
@@ -398,10 +397,9 @@ __global__ void __launch_bounds__(kDSThreads, 1) delta_stream_kernel(const Delta
   }
 }
 
-template <bool SPLIT>
-cudaError_t launch_split(const DeltaStreamParams& p, int n_lanes, cudaStream_t st) {
-  const size_t smem = 1024 + qimg_bytes(p.s.d) + 2 * (size_t)kStageBytes + (size_t)(SPLIT ? 32 : 16) * 256;
-  auto kern = delta_stream_kernel<SPLIT>;
+cudaError_t launch_kernel(const DeltaStreamParams& p, int n_lanes, cudaStream_t st) {
+  const size_t smem = 1024 + 32 * (size_t)p.s.d * 2 + 2 * (size_t)kStageBytes + 32 * 256;
+  auto kern = delta_stream_kernel;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -435,7 +433,8 @@ cudaError_t launch_delta_stream(const DeltaShape& s, const void* anchor, const v
                       reinterpret_cast<float*>(ws + wl.u_off),
                       reinterpret_cast<uint32_t*>(ws + wl.status_off),
                       wl.s_max};
-  return split_operands(s.d) ? launch_split<true>(p, n_lanes, st) : launch_split<false>(p, n_lanes, st);
+  if (wl.qrows != 32) return cudaErrorInvalidValue;  // the workspace must hold hi / lo query images
+  return launch_kernel(p, n_lanes, st);
 }
 
 }  // namespace tl

@@ -78,7 +78,8 @@ struct QProjParams {
   int n_lanes, nb;
   int cl;            // cluster size = K splits of q
   uint32_t* status;
-  uint8_t* qimg;     // [n_lanes][qimg_bytes(d)]
+  uint8_t* qimg;     // [n_lanes][qrows x d] fp16
+  int qrows;         // 32: fp16 hi + lo rows per head, 16: fp16 rows
   // fused append (codes == NULL: none): h_new of every active lane becomes its new token's row
   const __half* h_new;
   uint8_t* codes;
@@ -329,9 +330,9 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   // Image epilogue, one item at a time: fp16 hi/lo values are staged in shared memory in the
   // image's physical position order (the dead phase-1 region), then copied out as 16-byte
   // chunks at their swizzled image offsets.  The item loop count is the same for all threads.
-  const bool split = split_operands(s.d);
+  const bool split = p.qrows == 32;
   const int nhl = split ? 2 : 1;
-  const int rows_img = qimg_rows(s.d);
+  const int rows_img = p.qrows;
   __half* stg = reinterpret_cast<__half*>(base);  // [hl][nb][128]
   const bool ok2 = has_items && mbar_wait(&bar_m2, 0, abort_p, kProjWaitLimit);
   const float scale = 1.4426950408889634f / sqrtf((float)s.hd);
@@ -361,7 +362,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         const int hl = x / (nb * 16), b = (x / 16) % nb, g = x % 16;
         if (!((act >> b) & 1)) continue;
         const uint4 v = *reinterpret_cast<const uint4*>(stg + (hl * nb + b) * 128 + 8 * g);
-        uint8_t* img = p.qimg + (size_t)b * qimg_bytes(s.d);
+        uint8_t* img = p.qimg + (size_t)b * rows_img * s.d * 2;
         *reinterpret_cast<uint4*>(img + kmajor_offset(16 * hl + j, mc * 128 + 8 * g, rows_img)) = v;
       }
     }
@@ -376,7 +377,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
       if (!((act >> b) & 1)) continue;
       const int y = x % per_lane;
       const int j = s.H + y / (nhl * groups), hl = (y / groups) % nhl, g = y % groups;
-      uint8_t* img = p.qimg + (size_t)b * qimg_bytes(s.d);
+      uint8_t* img = p.qimg + (size_t)b * rows_img * s.d * 2;
       *reinterpret_cast<uint4*>(img + kmajor_offset(16 * hl + j, k * cs + 8 * g, rows_img)) = make_uint4(0, 0, 0, 0);
     }
   }
@@ -741,6 +742,7 @@ cudaError_t launch_qproj(const DecodeArgs& a, cudaStream_t st) {
                 CL,
                 reinterpret_cast<uint32_t*>(a.ws + w.status_off),
                 a.ws + w.qt_off,
+                w.qrows,
                 a.h_new,
                 a.append ? (uint8_t*)a.codes : nullptr,
                 a.append ? (uint8_t*)a.scales : nullptr};

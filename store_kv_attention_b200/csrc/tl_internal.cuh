@@ -115,28 +115,32 @@ __device__ __forceinline__ bool lane_active(const Shape& s, int iter, const int3
 // All offsets are 256-byte aligned.
 struct Workspace {
   size_t status_off;   // uint32 status word (+ padding to 256 bytes)
-  size_t qt_off;       // fp16 [n_lanes][qimg_rows(d) x d] absorbed query operand images (stream kernel)
+  size_t qt_off;       // fp16 [n_lanes][qrows x d] absorbed query operand images (stream kernel)
   size_t ml_off;       // fp32 [n_lanes][S_max][16][2]   per-split running max and sum
   size_t u_off;        // fp32 [n_lanes][S_max][16][d]   per-split unnormalised sum_c p_c h_c
   size_t total;
   int s_max, nb;
   int split;           // context rows per split
+  int qrows;           // rows of a query image: 16 (fp16) or 32 (fp16 hi + lo)
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 // extra_splits: splits a lane may have beyond those of max_ctx rows in one run (multi-query
 // calls, whose second row segment starts a split of its own).
-inline Workspace workspace_layout(const Shape& s, int n_lanes, int extra_splits = 0, int split = kSplitRows) {
+// qt_split: hi / lo query images at every d (otherwise only where split_operands(d)).
+inline Workspace workspace_layout(const Shape& s, int n_lanes, int extra_splits = 0, int split = kSplitRows,
+                                  bool qt_split = false) {
   Workspace w;
   w.split = split;
+  w.qrows = (qt_split || split_operands(s.d)) ? 32 : 16;
   w.s_max = splits_for_rows(s.max_ctx, split) + extra_splits;
   w.nb = lanes_padded(n_lanes);
   size_t off = 0;
   w.status_off = off;
   off += 256;
   w.qt_off = off;
-  off = align256(off + (size_t)n_lanes * qimg_bytes(s.d));
+  off = align256(off + (size_t)n_lanes * w.qrows * (size_t)s.d * 2);
   w.ml_off = off;
   off = align256(off + (size_t)n_lanes * w.s_max * kMaxHeads * 2 * 4);
   w.u_off = off;
