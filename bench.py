@@ -42,6 +42,13 @@ def parse_args():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--cpu-seconds", type=float, default=20.0, help="budget of the CPU-baseline sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--path", default="decode", choices=["decode", "verify", "prefill", "delta", "rope"],
+                   help="decode (the headline); verify / prefill: tree verification / chunked prefill over the "
+                        "cache; delta: the iteration-axis delta cache; rope: the rotary-embedding variant")
+    p.add_argument("--branches", type=int, default=4, help="verify: draft branches per lane")
+    p.add_argument("--depth", type=int, default=4, help="verify: tokens per branch")
+    p.add_argument("--tokens", type=int, default=16, help="prefill: tokens per lane per chunk")
+    p.add_argument("--lanes", type=int, default=8, help="delta: lanes (the workload's shape otherwise)")
     p.add_argument("--split-rows", type=int, default=0,
                    help="context rows per split of every decode call (tl_decode_opts.split_rows; 0 = the default 1024)")
     return p.parse_args()
@@ -463,6 +470,146 @@ def run_ours(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------- other paths
+def load_tensor_peak():
+    """Dense fp16/bf16 tensor TFLOP/s (the two have the same nominal rate on B200)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["bf16_tflops"]), "measured (bf16 burst; fp16 has the same nominal dense rate)"
+    return 1590.0, "fallback"
+
+
+def run_path(args, rank, world, local_rank):
+    """One JSON line for a path other than the headline decode: its own units, the step time, and
+    the roofline of its dominant kernel (events around every launch of it)."""
+    import numpy as np
+    import torch
+    import store_kv_attention_b200 as tl
+    from synth.device import DeviceWorkload
+
+    torch.cuda.set_device(local_rank)
+    dev = f"cuda:{local_rank}"
+    w = workload_for_rank(args.workload, rank)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1000 + w.seed)
+    rb = row_bytes(w)
+    extra = {}
+    if args.path in ("verify", "prefill"):
+        K, D = (args.branches, args.depth) if args.path == "verify" else (1, args.tokens)
+        dw = DeviceWorkload(w, device=dev, max_ctx=max(w.ctx) + K * D + 1)
+        # tree / chunk states: seeded normals on the device (timing inputs only)
+        trees = [torch.randn((w.B, K, D, w.d), generator=gen, device=dev).half() for _ in range(w.L_max)]
+        ws = torch.zeros(tl.verify_workspace_bytes(dw.desc, w.B, K, D), dtype=torch.uint8, device=dev)
+        out = torch.empty((w.B, K, D, w.H, w.hd), dtype=torch.float32, device=dev)
+
+        def step():
+            for it in range(w.L_max):
+                tl.verify_attn(dw.cache, it, dw.loops, dw.ctx, trees[it], dw.W["q"], dw.W["k"], dw.W["v"], out, ws)
+
+        act = [[b for b in range(w.B) if it < w.loops[b]] for it in range(w.L_max)]
+        units = sum(w.ctx[b] * K * D + K * D * (D + 1) // 2 for it in range(w.L_max) for b in act[it])
+        unit_name = "attended (query, row) pairs/s"
+        launch_bytes = [sum((w.ctx[b] + K * D) * rb for b in act[it]) for it in range(w.L_max)]
+        launches_per_it = -(-w.B * K * D // 64)
+        extra = {"branches": K, "depth": D, "query_tokens_per_lane": K * D,
+                 "roofline_note": "unique cache bytes (each row once from HBM) over the streaming launches of "
+                                  "an iteration; every query token streams its rows as a lane of its own"}
+        bound, peak, peak_kind, unit = "hbm", *load_peaks(), "GB/s"
+    elif args.path == "delta":
+        B = min(args.lanes, w.B)
+        ctx = w.ctx[0]
+        L = w.L_max
+        desc = tl.DeltaDesc(w.d, w.H, w.hd, L, B, ctx + 1)
+        cache = tl.DeltaCache(desc, device=dev, n_lanes=B)
+        # trajectories on the device: h^0 ~ N(0,1), h^l = h^(l-1) + sigma_l z with the contraction
+        # schedule of the synthetic generator (|dh|/|h| from 0.68 down to 0.04 over 32 iterations)
+        traj = [torch.randn((B, ctx + 1, w.d), generator=gen, device=dev)]
+        for l in range(1, L):
+            rho = 0.68 * (0.04 / 0.68) ** ((l - 1) / 31)
+            prev = traj[-1]
+            sigma = rho * prev.norm(dim=2, keepdim=True) / math.sqrt(w.d * (1 - rho * rho))
+            traj.append(prev + sigma * torch.randn(prev.shape, generator=gen, device=dev))
+        traj = [t.half() for t in traj]
+        zeros = torch.zeros(B, dtype=torch.int32, device=dev)
+        for it in range(L):
+            tl.delta_append(cache, it, traj[it][:, :ctx].contiguous(), zeros)
+        loops = torch.full((B,), L, dtype=torch.int32, device=dev)
+        ctx_d = torch.full((B,), ctx, dtype=torch.int32, device=dev)
+        h_new = [traj[it][:, ctx].contiguous() for it in range(L)]
+        W = [torch.from_numpy(np.ascontiguousarray(w.weight(k)).view(np.int16)).view(torch.float16).to(dev)
+             for k in "qkv"]
+        out = torch.empty((B, w.d), dtype=torch.float32, device=dev)
+
+        def step():
+            for it in range(L):
+                tl.delta_attn_decode(cache, it, loops, ctx_d, h_new[it], *W, out)
+
+        units = B * ctx * L
+        unit_name = UNIT
+        launch_bytes = [B * (ctx + 1) * (2 * w.d + it * (w.d + 2 * w.H)) for it in range(L)]
+        launches_per_it = 1
+        extra = {"lanes": B, "delta_rows_per_position_at_iteration_l": "anchor (2d B) + l x (d + 2 H) B",
+                 "inputs": "trajectories drawn on the device (seeded torch normals, the generator's schedule)"}
+        bound, peak, peak_kind, unit = "hbm", *load_peaks(), "GB/s"
+    else:  # rope
+        dw = DeviceWorkload(w, device=dev)
+        ws = torch.zeros(tl.rope_workspace_bytes(dw.desc, w.B), dtype=torch.uint8, device=dev)
+
+        def step():
+            for it in range(w.L_max):
+                dw.append_new(it)
+                tl.attn_decode_rope(dw.cache, it, dw.loops, dw.ctx, dw.h_new[it], dw.W["q"], dw.W["k"],
+                                    dw.W["v"], dw.out[it], ws, residual=dw.residual[it], threshold=w.threshold,
+                                    abort_flags=dw.flags, first_abort_iter=dw.first)
+
+        units = w.cached_positions_per_step()
+        unit_name = UNIT
+        # the score kernel's contraction: K = h W_k^T for every attended row (2 d^2 FLOPs per row)
+        launch_bytes = [sum(2.0 * (w.ctx[b] + 1) * w.d * w.d for b in range(w.B) if it < w.loops[b])
+                        for it in range(w.L_max)]
+        launches_per_it = 1
+        extra = {"rope_base": 10000.0}
+        bound, (peak, peak_kind), unit = "tensor", load_tensor_peak(), "TFLOP/s"
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    K_ = args.steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    clocks.__enter__()
+    e0.record()
+    for _ in range(K_):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    with tl.ProfileHook(K_ * w.L_max * launches_per_it) as prof:
+        for _ in range(K_):
+            step()
+        torch.cuda.synchronize()
+    clocks.__exit__(None, None, None)
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    kms = prof.stream_kernel_ms()
+    per_it = [sum(kms[i * launches_per_it:(i + 1) * launches_per_it]) for i in range(len(kms) // launches_per_it)]
+    total = sum(launch_bytes[i % w.L_max] for i in range(len(per_it)))
+    achieved = total / (sum(per_it) / 1000.0) / (1e9 if unit == "GB/s" else 1e12)
+    if rank != 0:
+        return
+    line = {"metric": f"{args.path} over the store-h cache: {unit_name} on 1 B200", "value":
+            world * K_ * units / (ms / 1000.0), "unit": unit_name, "n_gpus": world, "steps": K_,
+            "warmup": args.warmup, "ms_per_step": ms / K_, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "path": args.path,
+            "config": workload_config(w, world, extra),
+            "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+                         "traffic": None, "peak_source": peak_kind,
+                         "algorithmic_per_iteration": statistics.mean(launch_bytes),
+                         "kernel_ms_per_iteration": statistics.mean(per_it)},
+            "gpu_launches": prof.launches, "clocks": clocks.summary()}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -481,6 +628,8 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, rank, world)
+        elif args.path != "decode":
+            run_path(args, rank, world, local_rank)
         else:
             run_ours(args, rank, world, local_rank)
     finally:

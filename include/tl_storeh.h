@@ -426,8 +426,9 @@ TL_API tl_status tl_storeh_selftest_wait_timeout(void* workspace, size_t workspa
  * thread, every tl_storeh_* call made from that thread counts the kernels it
  * launches in `launches`, and records begin_events[k] / end_events[k]
  * (cudaEvent_t handles created by the caller) on the call's stream right before
- * and right after each launch of the context-streaming kernel of
- * tl_storeh_attn_decode, for k = recorded++ while recorded < capacity.
+ * and right after each launch of the call's dominant kernel -- the context-streaming
+ * kernel of the decode, verification, prefill and delta calls, the score kernel (the
+ * K rebuild) of tl_storeh_attn_decode_rope -- for k = recorded++ while recorded < capacity.
  * Pass NULL to uninstall.  The struct must outlive its installation.  The events
  * sit between kernels, which stops a kernel from being scheduled during the tail
  * of the one before it, so a step timed with the hook installed runs a little

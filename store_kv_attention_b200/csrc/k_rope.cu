@@ -323,7 +323,8 @@ cudaError_t launch_rope_scores(const DecodeArgs& a, float rope_base, float2* cs,
   e = cudaLaunchKernelEx(&cfg, rope_query_kernel, s, a.iter, a.loops, a.ctx_len, a.h_new, a.Wq, (const float2*)cs, qrot);
   count_launch();
   if (e != cudaSuccess) return e;
-  // 3. the scores: K rebuilt on the tensor cores, rotated and dotted in the epilogue
+  // 3. the scores: K rebuilt on the tensor cores, rotated and dotted in the epilogue (the
+  // measurement hook brackets this launch, the call's dominant kernel)
   const int NP = rope_pass_cols(s);
   alignas(64) CUtensorMap tmWk;
   if (!make_tmap_f16(&tmWk, a.Wk, s.d, s.d, s.d, 64, 128)) return cudaErrorInvalidValue;
@@ -335,7 +336,9 @@ cudaError_t launch_rope_scores(const DecodeArgs& a, float rope_base, float2* cs,
   cfg.gridDim = dim3((unsigned)((s.max_ctx + 127) / 128), (unsigned)(s.d / NP), (unsigned)a.n_lanes);
   cfg.blockDim = dim3(kRThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
+  profile_stream_begin(st);
   e = cudaLaunchKernelEx(&cfg, rope_score_kernel, tmWk, p);
+  profile_stream_end(st);
   count_launch();
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

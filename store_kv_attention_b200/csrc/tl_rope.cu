@@ -79,11 +79,7 @@ tl_status tl_storeh_attn_decode_rope(const tl_storeh_desc* desc, tl_storeh_cache
   cudaStream_t cs = (cudaStream_t)stream;
   cudaError_t e = launch_rope_scores(a, rope_base, (float2*)(ws + w.cs_off), (float*)(ws + w.qrot_off),
                                      (float*)(ws + w.scores_off), cs);
-  if (e == cudaSuccess) {
-    profile_stream_begin(cs);
-    e = launch_stream(a, cs);
-    profile_stream_end(cs);
-  }
+  if (e == cudaSuccess) e = launch_stream(a, cs);
   if (e == cudaSuccess) e = launch_oproj(a, cs);
   if (e != cudaSuccess) return set_error(TL_ERR_CUDA, "rope decode launch: %s", cudaGetErrorString(e));
   return TL_OK;

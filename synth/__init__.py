@@ -129,16 +129,32 @@ def trajectory_f16(seed: int, n_tokens: int, d: int, L: int, rho_first: float = 
     the 407M / 2B models (0.68 at the first iteration to 0.04 at the 32nd).  A random walk
     with that step schedule, nothing more; every draw comes from the counter-based normals.
     """
+    # token t's draws are the counters [t (L+1) d, (t+1) (L+1) d): one contiguous block for all
+    # tokens, so the recurrence runs over all tokens at once
+    z = normal_f64(seed, TID_TRAJ, 0, n_tokens * (L + 1) * d).reshape(n_tokens, L + 1, d)
+    out = np.empty((L + 1, n_tokens, d), dtype=np.float16)
+    out[0] = z[:, 0].astype(np.float16)  # round to nearest even, as normal_f16
+    for l in range(1, L + 1):
+        rho = rho_first * (rho_last / rho_first) ** ((l - 1) / max(rho_span - 1, 1))
+        prev = out[l - 1].astype(np.float64)
+        sigma = rho * np.linalg.norm(prev, axis=1, keepdims=True) / math.sqrt(d * (1.0 - rho * rho))
+        out[l] = (prev + sigma * z[:, l]).astype(np.float16)
+    return out
+
+
+def _trajectory_f16_per_token(seed: int, n_tokens: int, d: int, L: int, rho_first: float = 0.68,
+                              rho_last: float = 0.04, rho_span: int = 32) -> np.ndarray:
+    """The same trajectories one token at a time (the definition the vectorised form follows)."""
     out = np.empty((L + 1, n_tokens, d), dtype=np.float16)
     for t in range(n_tokens):
         base = t * (L + 1) * d
         out[0, t] = normal_f16(seed, TID_TRAJ, base, d)
         for l in range(1, L + 1):
             rho = rho_first * (rho_last / rho_first) ** ((l - 1) / max(rho_span - 1, 1))
-            z = normal_f64(seed, TID_TRAJ, base + l * d, d)
+            zz = normal_f64(seed, TID_TRAJ, base + l * d, d)
             prev = out[l - 1, t].astype(np.float64)
             sigma = rho * np.linalg.norm(prev) / math.sqrt(d * (1.0 - rho * rho))
-            out[l, t] = (prev + sigma * z).astype(np.float16)
+            out[l, t] = (prev + sigma * zz).astype(np.float16)
     return out
 
 

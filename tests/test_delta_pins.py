@@ -199,3 +199,11 @@ def test_storage_bytes():
     assert a.nbytes + c.nbytes + s.nbytes == D.delta_cache_bytes(d, H, L, n)
     # the same storage class as INT8-h (d + 4 bytes per token and iteration) plus the anchor
     assert D.delta_cache_bytes(d, H, L, n) - n * L * (d + 4) == n * (2 * d + L * (2 * H - 4))
+
+
+def test_trajectory_generator_vectorised_equals_per_token():
+    """The trajectories drawn for all tokens at once are the per-token recurrence, bit for bit."""
+    for args in [(3, 17, 256, 5), (31, 9, 1024, 8)]:
+        a = synth.trajectory_f16(*args)
+        b = synth._trajectory_f16_per_token(*args)
+        assert np.array_equal(a.view(np.uint16), b.view(np.uint16))
