@@ -55,6 +55,7 @@ struct DeltaStreamParams {
   float* U;                     // [n_lanes][s_max][16][d]
   uint32_t* status;
   int s_max;
+  int split;                    // context rows per split
 };
 
 __device__ __forceinline__ uint32_t pack_h2(__half a, __half b) {
@@ -129,9 +130,9 @@ __global__ void __launch_bounds__(kDSThreads, 1) delta_stream_kernel(const Delta
   const int b = blockIdx.x, split = blockIdx.y;
   if (!p.dloops[b]) return;
   const int n = p.ctx_len[b] + 1;  // < max_ctx + 1: the prep kernel checked ctx_len
-  const int r_begin = split * kSplitRows;
+  const int r_begin = split * p.split;
   if (r_begin >= n) return;
-  const int r_end = min(n, r_begin + kSplitRows);
+  const int r_end = min(n, r_begin + p.split);
   const int n_tiles = (r_end - r_begin + 127) >> 7;
   const int n_units = D >> 7;
   const uint32_t qbytes = (uint32_t)(NS * D * 2);
@@ -432,7 +433,8 @@ cudaError_t launch_delta_stream(const DeltaShape& s, const void* anchor, const v
                       reinterpret_cast<float*>(ws + wl.ml_off),
                       reinterpret_cast<float*>(ws + wl.u_off),
                       reinterpret_cast<uint32_t*>(ws + wl.status_off),
-                      wl.s_max};
+                      wl.s_max,
+                      wl.split};
   if (wl.qrows != 32) return cudaErrorInvalidValue;  // the workspace must hold hi / lo query images
   return launch_kernel(p, n_lanes, st);
 }

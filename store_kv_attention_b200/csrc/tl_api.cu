@@ -75,7 +75,9 @@ struct DeltaWorkspace {
 };
 DeltaWorkspace delta_workspace(const tl::DeltaShape& s, int n_lanes) {
   DeltaWorkspace w;
-  w.wl = tl::workspace_layout(delta_view_shape(s, n_lanes), n_lanes, 0, tl::kSplitRows, /*qt_split=*/true);
+  // 256-row splits: this path's streaming kernel works through a split sequentially, so a lane
+  // is spread over more SMs; the plan still depends on the lane's own context only
+  w.wl = tl::workspace_layout(delta_view_shape(s, n_lanes), n_lanes, 0, tl::kDeltaSplitRows, /*qt_split=*/true);
   w.wloops_off = tl::align256(w.wl.total);
   w.dloops_off = w.wloops_off + tl::align256((size_t)n_lanes * 4);
   w.total = w.dloops_off + tl::align256((size_t)n_lanes * 4);

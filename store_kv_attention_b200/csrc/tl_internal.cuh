@@ -21,6 +21,7 @@ constexpr int kInt4Group = 64;
 constexpr int kMaxHeads = 16;        // heads are padded to 16 in the kernels
 constexpr int kSplitRows = 1024;     // default context rows per split (a call may choose 128, 256, 512 or 1024)
 constexpr int kMaxCtx = 65536;       // positions per (layer, lane) the kernels support
+constexpr int kDeltaSplitRows = 256;  // context rows per split of the delta-cache decode
 constexpr int kMaxSplits = kMaxCtx / kSplitRows;
 
 // ---------------------------------------------------------------- shapes

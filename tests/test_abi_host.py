@@ -156,7 +156,7 @@ def test_delta_workspace_and_decode_rejected_before_launch(tl):
     sdesc = tl.StoreHDesc(2048, 16, 128, n_pre=0, L_max=1, max_lanes=2, max_ctx=1000, fmt=tl.TL_H_FP16)
     # the decode workspace (with hi and lo query images: 2 lanes x 16 more rows x d fp16) and two
     # small per-lane arrays; the rows are rebuilt inside the streaming kernel, with no scratch copy
-    base = tl.workspace_bytes(sdesc, 2) + 2 * 16 * 2048 * 2
+    base = tl.workspace_bytes(sdesc, 2, split_rows=256) + 2 * 16 * 2048 * 2  # 256-row splits
     assert base < ws < base + 4096 and ws % 256 == 0
     with pytest.raises(tl.TLError) as e:
         tl.delta_workspace_bytes(desc, 5)
