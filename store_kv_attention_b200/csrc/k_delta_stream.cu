@@ -23,9 +23,10 @@
 //   softmax:    S -> P (fp16 hi / lo), lazy rescale of U^T
 //   P.V pass:   for each unit, rebuild again -> hi / lo into shared memory (MN-major) ->
 //               4 x 8 SS MMAs (h hi / lo times P hi / lo) into U^T
-// The passes run one after the other in all four warps (no warp specialisation): the delta
-// cache reads (1 + iter) rows per position, and this kernel is written for clarity of the
-// rebuild first.  Every wait is bounded; on expiry the kernel records a timeout in the status
+// The passes run one after the other in all eight warps (no warp specialisation): warps w and
+// w + 4 own the same 32 rows (TMEM lane quarter w) and rebuild alternate 32-value chunks of each
+// unit; the softmax and the epilogue run in warps 0-3.  The delta cache reads (1 + iter) rows
+// per position, and this kernel is written for clarity of the rebuild first.  Every wait is bounded; on expiry the kernel records a timeout in the status
 // word, waits (bounded) for its MMAs in flight, frees its TMEM and returns.
 #include <math_constants.h>
 
@@ -38,7 +39,7 @@ namespace {
 
 using namespace ptx;
 
-constexpr int kDSThreads = 128;                 // four warps = four TMEM lane quarters = 128 rows
+constexpr int kDSThreads = 256;                 // eight warps: two per TMEM lane quarter (32 rows)
 constexpr int kStageBytes = 128 * 256;          // one unit of one part, 128 rows x 128 fp16, MN-major
 constexpr long long kDWait = 4000000000ll;      // ~2 s of SM clocks
 
@@ -149,9 +150,10 @@ __global__ void __launch_bounds__(kDSThreads, 1) delta_stream_kernel(const Delta
   __shared__ float red[4][16];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = threadIdx.x;  // this thread's row of a tile = its TMEM lane
+  const int quarter = warp & 3, grp = warp >> 2;  // grp 0 also runs the softmax and the epilogue
+  const int r = quarter * 32 + lane;              // this thread's row of a tile = its TMEM lane
   const int xr = r & 7;
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
   if (threadIdx.x == 0) {
     mbar_init(&bar_q, 1);
     mbar_init(&bar_mma, 1);
@@ -213,7 +215,8 @@ __global__ void __launch_bounds__(kDSThreads, 1) delta_stream_kernel(const Delta
     for (int u = 0; u < n_units && ok; ++u) {
       uint32_t hi[16], lo[16];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int qq = 0; qq < 2; ++qq) {
+        const int q = grp + 2 * qq;  // this warp's 32-value chunks of the unit
         rebuild32(p, row, valid, u * 128 + q * 32, hi, lo);
         tmem_st16(tbase + lane_off + kColHi + q * 16, hi);
         tmem_st16(tbase + lane_off + kColLo + q * 16, lo);
@@ -244,8 +247,10 @@ __global__ void __launch_bounds__(kDSThreads, 1) delta_stream_kernel(const Delta
     if (!ok) break;
 
     // ---------------------------------------------------------------- online softmax of the tile
-    float sc[16];
-    {
+    // warps 0-3 (one thread per row); warps 4-7 only pass the block barriers
+    float sc[16], alpha[16];
+    bool rescale = false;
+    if (grp == 0) {
       uint32_t v[16];
       tmem_ld16(tbase + lane_off + kColS, v);
       tmem_ld_wait();
@@ -255,60 +260,63 @@ __global__ void __launch_bounds__(kDSThreads, 1) delta_stream_kernel(const Delta
       tmem_ld_wait();
 #pragma unroll
       for (int j = 0; j < 16; ++j) sc[j] += __uint_as_float(v[j]);
-    }
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      if (!valid || j >= s.H) sc[j] = -CUDART_INF_F;
-      float m = sc[j];
+      for (int j = 0; j < 16; ++j) {
+        if (!valid || j >= s.H) sc[j] = -CUDART_INF_F;
+        float m = sc[j];
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      if (lane == 0) red[warp][j] = m;
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) red[warp][j] = m;
+      }
     }
     __syncthreads();
-    float alpha[16];
-    bool rescale = false;
+    if (grp == 0) {
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const float tm = fmaxf(fmaxf(red[0][j], red[1][j]), fmaxf(red[2][j], red[3][j]));
-      alpha[j] = 1.0f;
-      if (tm > m_used[j] + 8.0f) {  // lazy rescale: P stays below 2^8 otherwise
-        if (m_used[j] != -CUDART_INF_F) {
-          alpha[j] = exp2f(m_used[j] - tm);
-          rescale = true;
+      for (int j = 0; j < 16; ++j) {
+        const float tm = fmaxf(fmaxf(red[0][j], red[1][j]), fmaxf(red[2][j], red[3][j]));
+        alpha[j] = 1.0f;
+        if (tm > m_used[j] + 8.0f) {  // lazy rescale: P stays below 2^8 otherwise
+          if (m_used[j] != -CUDART_INF_F) {
+            alpha[j] = exp2f(m_used[j] - tm);
+            rescale = true;
+          }
+          m_used[j] = tm;
         }
-        m_used[j] = tm;
       }
     }
     __syncthreads();  // red is reused below
-    float pr[16];
+    if (grp == 0) {
+      float pr[16];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      pr[j] = (valid && j < s.H) ? exp2f(sc[j] - m_used[j]) : 0.0f;
-      l_part[j] = l_part[j] * alpha[j] + pr[j];
-    }
-    if (rescale && t > 0) {
-      // the P.V MMAs of the earlier tiles are complete (each was waited for)
-      for (int u = 0; u < n_units; ++u) {
-        uint32_t uv[16];
-        tmem_ld16(tbase + lane_off + kColU + u * NP, uv);
-        tmem_ld_wait();
-#pragma unroll
-        for (int c = 0; c < 16; ++c) uv[c] = __float_as_uint(__uint_as_float(uv[c]) * alpha[c]);
-        tmem_st16(tbase + lane_off + kColU + u * NP, uv);
+      for (int j = 0; j < 16; ++j) {
+        pr[j] = (valid && j < s.H) ? exp2f(sc[j] - m_used[j]) : 0.0f;
+        l_part[j] = l_part[j] * alpha[j] + pr[j];
       }
-      tmem_st_wait();
-    }
+      if (__any_sync(0xffffffffu, rescale) && t > 0) {
+        // the P.V MMAs of the earlier tiles are complete (each was waited for)
+        for (int u = 0; u < n_units; ++u) {
+          uint32_t uv[16];
+          tmem_ld16(tbase + lane_off + kColU + u * NP, uv);
+          tmem_ld_wait();
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const __half hi = __float2half_rn(pr[j]);
-      *reinterpret_cast<__half*>(ps + kmajor_offset(j, r, PR)) = hi;
-      *reinterpret_cast<__half*>(ps + kmajor_offset(16 + j, r, PR)) = __float2half_rn(pr[j] - __half2float(hi));
+          for (int c = 0; c < 16; ++c) uv[c] = __float_as_uint(__uint_as_float(uv[c]) * alpha[c]);
+          tmem_st16(tbase + lane_off + kColU + u * NP, uv);
+        }
+        tmem_st_wait();
+      }
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const __half hi = __float2half_rn(pr[j]);
+        *reinterpret_cast<__half*>(ps + kmajor_offset(j, r, PR)) = hi;
+        *reinterpret_cast<__half*>(ps + kmajor_offset(16 + j, r, PR)) = __float2half_rn(pr[j] - __half2float(hi));
+      }
     }
 
     // ---------------------------------------------------------------- P.V pass
     for (int u = 0; u < n_units && ok; ++u) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int qq = 0; qq < 2; ++qq) {
+        const int q = grp + 2 * qq;  // this warp's 32-value chunks of the unit
         uint32_t hi[16], lo[16];
         rebuild32(p, row, valid, u * 128 + q * 32, hi, lo);
         // values q*32 .. q*32+31 of the unit: atom-column q / 2, 16-byte vectors 4 (q & 1) .. + 3
@@ -351,7 +359,7 @@ __global__ void __launch_bounds__(kDSThreads, 1) delta_stream_kernel(const Delta
   }
 
   // ---------------------------------------------------------------- partial (m, l, U) of this split
-  if (ok) {
+  if (ok && grp == 0) {
     const size_t part = (size_t)b * p.s_max + split;
     for (int u = 0; u < n_units; ++u) {
       uint32_t uv[16];
@@ -369,16 +377,17 @@ __global__ void __launch_bounds__(kDSThreads, 1) delta_stream_kernel(const Delta
       for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
       if (lane == 0) red[warp][j] = v;
     }
-    __syncthreads();
-    if (threadIdx.x < 16) {
-      const int j = threadIdx.x;
-      float m = 0.0f;
+  }
+  __syncthreads();
+  if (ok && threadIdx.x < 16) {
+    const size_t part = (size_t)b * p.s_max + split;
+    const int j = threadIdx.x;
+    float m = 0.0f;
 #pragma unroll
-      for (int i = 0; i < 16; ++i)
-        if (i == j) m = m_used[i];
-      p.ml[(part * kMaxHeads + j) * 2 + 0] = m;
-      p.ml[(part * kMaxHeads + j) * 2 + 1] = red[0][j] + red[1][j] + red[2][j] + red[3][j];
-    }
+    for (int i = 0; i < 16; ++i)
+      if (i == j) m = m_used[i];
+    p.ml[(part * kMaxHeads + j) * 2 + 0] = m;
+    p.ml[(part * kMaxHeads + j) * 2 + 1] = red[0][j] + red[1][j] + red[2][j] + red[3][j];
   }
 
   tc_fence_before();

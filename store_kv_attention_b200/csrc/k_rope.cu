@@ -107,31 +107,51 @@ struct RopeScoreParams {
   int n_pass;          // K columns per CTA (a multiple of hd, at most 512)
 };
 
-// The 64 values [k0, k0 + 64) of one cached row as fp16 pairs into a K-major swizzled A tile.
-// FP16 rows are copied, INT8 codes are converted exactly (the row scale is applied to the
-// scores), INT4 codes are multiplied by their group scale (rounded once to fp16).
-__device__ __forceinline__ void stage_row(const Shape& s, const uint8_t* codes, const uint8_t* scales, size_t row,
-                                          bool valid, int k0, uint8_t* tile, int r) {
+// The raw codes of the 64 values [k0, k0 + 64) of one cached row (and, for INT4, their group
+// scale), loaded one K-step ahead of their use so that the loads are in flight during the MMAs.
+struct RowSlice {
+  uint4 v[8];
+  __half sc;
+};
+__device__ __forceinline__ void load_row(const Shape& s, const uint8_t* codes, const uint8_t* scales, size_t row,
+                                         bool valid, int k0, RowSlice& x) {
+  if (!valid) return;
+  if (s.fmt == TL_H_FP16) {
+    const uint4* src = reinterpret_cast<const uint4*>(codes + row * (size_t)(2 * s.d) + 2 * k0);
+#pragma unroll
+    for (int v = 0; v < 8; ++v) x.v[v] = __ldg(src + v);
+  } else if (s.fmt == TL_H_INT8_TOKEN) {
+    const uint4* src = reinterpret_cast<const uint4*>(codes + row * (size_t)s.d + k0);
+#pragma unroll
+    for (int v = 0; v < 4; ++v) x.v[v] = __ldg(src + v);
+  } else {
+    const uint4* src = reinterpret_cast<const uint4*>(codes + row * (size_t)(s.d / 2) + k0 / 2);
+    x.v[0] = __ldg(src);
+    x.v[1] = __ldg(src + 1);
+    x.sc = reinterpret_cast<const __half*>(scales)[row * (size_t)(s.d / kInt4Group) + k0 / kInt4Group];
+  }
+}
+
+// The loaded slice as fp16 pairs into a K-major swizzled A tile.  FP16 rows are copied, INT8
+// codes are converted exactly (the row scale is applied to the scores), INT4 codes are
+// multiplied by their group scale (rounded once to fp16).  Rows outside the lane give zeros.
+__device__ __forceinline__ void stage_row(const Shape& s, const RowSlice& x, bool valid, uint8_t* tile, int r) {
   uint32_t h[32];
   if (!valid) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) h[i] = 0u;
   } else if (s.fmt == TL_H_FP16) {
-    const uint4* src = reinterpret_cast<const uint4*>(codes + row * (size_t)(2 * s.d) + 2 * k0);
 #pragma unroll
     for (int v = 0; v < 8; ++v) {
-      const uint4 w = __ldg(src + v);
-      h[4 * v] = w.x;
-      h[4 * v + 1] = w.y;
-      h[4 * v + 2] = w.z;
-      h[4 * v + 3] = w.w;
+      h[4 * v] = x.v[v].x;
+      h[4 * v + 1] = x.v[v].y;
+      h[4 * v + 2] = x.v[v].z;
+      h[4 * v + 3] = x.v[v].w;
     }
   } else if (s.fmt == TL_H_INT8_TOKEN) {
-    const uint4* src = reinterpret_cast<const uint4*>(codes + row * (size_t)s.d + k0);
 #pragma unroll
     for (int v = 0; v < 4; ++v) {
-      const uint4 w = __ldg(src + v);
-      const int8_t* c = reinterpret_cast<const int8_t*>(&w);
+      const int8_t* c = reinterpret_cast<const int8_t*>(&x.v[v]);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const __half2 p = __halves2half2(__int2half_rn(c[2 * i]), __int2half_rn(c[2 * i + 1]));
@@ -139,19 +159,16 @@ __device__ __forceinline__ void stage_row(const Shape& s, const uint8_t* codes, 
       }
     }
   } else {
-    const uint4* src = reinterpret_cast<const uint4*>(codes + row * (size_t)(s.d / 2) + k0 / 2);
-    const __half sc = reinterpret_cast<const __half*>(scales)[row * (size_t)(s.d / kInt4Group) + k0 / kInt4Group];
-    const __half2 s2 = __halves2half2(sc, sc);
+    const __half2 s2 = __halves2half2(x.sc, x.sc);
 #pragma unroll
     for (int v = 0; v < 2; ++v) {
-      const uint4 w = __ldg(src + v);
-      const uint8_t* by = reinterpret_cast<const uint8_t*>(&w);
+      const uint8_t* by = reinterpret_cast<const uint8_t*>(&x.v[v]);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const int lo = (int)(by[i] & 0xF), hi = (int)(by[i] >> 4);
         const __half2 p = __halves2half2(__int2half_rn(lo >= 8 ? lo - 16 : lo), __int2half_rn(hi >= 8 ? hi - 16 : hi));
-        const __half2 x = __hmul2(p, s2);
-        h[16 * v + i] = *reinterpret_cast<const uint32_t*>(&x);
+        const __half2 y = __hmul2(p, s2);
+        h[16 * v + i] = *reinterpret_cast<const uint32_t*>(&y);
       }
     }
   }
@@ -215,6 +232,8 @@ __global__ void __launch_bounds__(kRThreads, 1)
   const size_t grow = ((size_t)(s.n_pre + p.iter) * s.max_lanes + b) * s.max_ctx + (size_t)row;
   const uint32_t idesc = idesc_f16_f32(128, 256, false, false);
   bool ok = true, issued = false;
+  RowSlice nxt;
+  load_row(s, p.codes, p.scales, grow, valid, 0, nxt);
   for (int ks = 0; ks < n_ks && ok; ++ks) {
     const int st = ks & 1, use = ks >> 1;
     if (ks >= 2 && !(ok = block_wait(&empty[st], (use - 1) & 1, abort_p))) break;
@@ -223,7 +242,8 @@ __global__ void __launch_bounds__(kRThreads, 1)
       for (int nb = 0; nb < NP / 128; ++nb)
         tma_load_2d(B[st] + nb * 16384, &tmWk, ks * 64, cb * NP + nb * 128, &full[st]);
     }
-    stage_row(s, p.codes, p.scales, grow, valid, ks * 64, A[st], r);
+    stage_row(s, nxt, valid, A[st], r);
+    if (ks + 1 < n_ks) load_row(s, p.codes, p.scales, grow, valid, (ks + 1) * 64, nxt);  // in flight during the MMAs
     fence_proxy_async_smem();
     __syncthreads();
     if (warp == 0) {
