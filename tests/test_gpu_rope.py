@@ -63,3 +63,27 @@ def test_rope_decode_matches_oracle(name, ctx, loops, base):
             assert err <= MAX_ABS and rel <= REL_L2, f"{name} lane {b} it {it}: max-abs {err:.3g} rel-L2 {rel:.3g}"
         f, fi, _ = oracle.cpp.residual_norm_check(w.residual(it, True), w.threshold, it, np.array(w.loops), f, fi)
     assert np.array_equal(dw.flags.cpu().numpy(), f) and np.array_equal(dw.first.cpu().numpy(), fi)
+
+
+def test_rope_decode_long_context():
+    """A 60,000-position lane: angles up to 6e4 rad, which the FP64 table must reduce exactly."""
+    import store_kv_attention_b200 as tl
+    from synth.device import DeviceWorkload
+    w = dataclasses.replace(small_variant(get_workload("tiny_fp16"), ctx=[60000, 17], loops=[1, 1]), L_max=1)
+    dw = DeviceWorkload(w)
+    ws = torch.zeros(tl.rope_workspace_bytes(dw.desc, w.B), dtype=torch.uint8, device="cuda")
+    dw.append_new(0)
+    tl.attn_decode_rope(dw.cache, 0, dw.loops, dw.ctx, dw.h_new[0], dw.W["q"], dw.W["k"], dw.W["v"], dw.out[0], ws)
+    torch.cuda.synchronize()
+    assert tl.poll_status(ws) == tl.TL_OK
+    got = dw.out[0].cpu().numpy()
+    W = [w.weight(k) for k in "qkv"]
+    for b in range(w.B):
+        rows = np.concatenate([w.h_rows(w.n_pre, b, 0, w.ctx[b]), w.h_new(0)[b:b + 1]])
+        c, s_ = oracle.cpp.quantize_rows(rows, w.fmt)
+        hh = oracle.cpp.dequantize_rows(c, s_, w.fmt, w.d)
+        want = rope_oracle.attend_rope(hh, w.h_new(0)[b], *W, w.H, w.hd)
+        g = got[b].astype(np.float64)
+        err = np.abs(g - want).max()
+        rel = np.linalg.norm(g - want) / np.linalg.norm(want)
+        assert err <= MAX_ABS and rel <= REL_L2, f"lane {b}: max-abs {err:.3g} rel-L2 {rel:.3g}"

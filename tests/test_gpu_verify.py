@@ -185,3 +185,33 @@ def test_tree_that_does_not_fit_is_skipped_and_reported():
     assert np.all(np.isfinite(got[0])) and np.all(np.isnan(got[1]))
     assert tl.poll_status(ws) == tl.TL_ERR_DEVICE_RANGE
     assert tl.poll_status(ws) == tl.TL_OK
+
+
+def test_prefill_long_chunk_spans_groups():
+    """A chunk of 70 tokens on 2 lanes (140 query tokens: three groups of the decode kernels),
+    sampled tokens against the oracle, the chunk rows bit-exact in the cache."""
+    import store_kv_attention_b200 as tl
+    from synth.device import DeviceWorkload
+    T = 70
+    w = _workload(2, [900, 3], [2, 2])
+    it = 0
+    dw = DeviceWorkload(w, max_ctx=max(w.ctx) + T + 1)
+    chunk = _tree_states(w, it, 1, T)[:, 0]
+    ws = torch.zeros(tl.verify_workspace_bytes(dw.desc, w.B, 1, T), dtype=torch.uint8, device="cuda")
+    out = torch.full((w.B, T, w.H, w.hd), float("nan"), dtype=torch.float32, device="cuda")
+    tl.prefill_attn(dw.cache, it, dw.loops, dw.ctx, _f16(chunk), dw.W["q"], dw.W["k"], dw.W["v"], out, ws)
+    torch.cuda.synchronize()
+    assert tl.poll_status(ws) == tl.TL_OK
+    got = out.cpu().numpy()
+    assert np.all(np.isfinite(got))
+    W = [w.weight(k) for k in "qkv"]
+    layer = w.n_pre + it
+    for b in range(w.B):
+        rows = np.concatenate([w.h_rows(layer, b, 0, w.ctx[b]), chunk[b]])
+        c, s = oracle.cpp.quantize_rows(rows, w.fmt)
+        cc, cs = _cache_rows(dw, layer, b, 0, w.ctx[b] + T)
+        assert np.array_equal(cc, c) and np.array_equal(cs.view(np.uint8), s.view(np.uint8))
+        hh = oracle.cpp.dequantize_rows(c, s, w.fmt, w.d)
+        for t in (0, 1, 63, 64, 69):
+            want = oracle.cpp.attend_absorbed(hh[: w.ctx[b] + t + 1], chunk[b, t], *W, w.H, w.hd)
+            _close(got[b, t], want, f"lane {b} token {t}")
