@@ -42,6 +42,9 @@ def parse_args():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--cpu-seconds", type=float, default=20.0, help="budget of the CPU-baseline sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-graph", action="store_true",
+                   help="decode: time the headline and per-step passes as eager calls instead of replays of "
+                        "a CUDA graph of one step")
     p.add_argument("--path", default="decode", choices=["decode", "verify", "prefill", "delta", "rope"],
                    help="decode (the headline); verify / prefill: tree verification / chunked prefill over the "
                         "cache; delta: the iteration-axis delta cache; rope: the rotary-embedding variant")
@@ -330,6 +333,25 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     if tl.poll_status(dw.cache) != tl.TL_OK:
         raise RuntimeError("device status after warm-up: " + tl.lib.tl_last_error_message().decode())
+    # One step (every loop iteration's tl_storeh_append_attn_decode call) captured as a CUDA graph:
+    # the same launches with the same arguments, replayed without the host's per-call overhead.
+    run_step = lambda: dw.step(fused_append=True)
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            dw.step(fused_append=True)
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(graph):
+            dw.step(fused_append=True)
+        run_step = graph.replay
+        for _ in range(max(3, args.warmup)):
+            run_step()
+        torch.cuda.synchronize()
+        if tl.poll_status(dw.cache) != tl.TL_OK:
+            raise RuntimeError("device status after graph warm-up: " + tl.lib.tl_last_error_message().decode())
 
     K = args.steps
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -341,7 +363,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     start.record(stream)
     for _ in range(K):
-        dw.step(fused_append=True)
+        run_step()
     end.record(stream)
     torch.cuda.synchronize()
     barrier()
@@ -349,7 +371,7 @@ def run_ours(args, rank, world, local_rank):
     step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     for a, b_ in step_ev:
         a.record(stream)
-        dw.step(fused_append=True)
+        run_step()
         b_.record(stream)
     torch.cuda.synchronize()
     step_ms_median = statistics.median(a.elapsed_time(b_) for a, b_ in step_ev)
@@ -461,6 +483,10 @@ def run_ours(args, rank, world, local_rank):
                                                  "timing": ("value and ms_per_step: K steps between one event "
                                                             "pair (no event between kernels); the median of K "
                                                             "per-step event pairs is reported beside it"),
+                                                 "launch": ("eager calls" if args.no_graph else
+                                                            "replays of a CUDA graph of one step (the step's "
+                                                            "calls captured once); the kernel pass and e2e "
+                                                            "run as eager calls"),
                                                  "step_frac_of_hbm_roofline": step_roofline_ms / (ms_max / K)}),
             "roofline": roofline,
             "cpu_baseline": cpu,

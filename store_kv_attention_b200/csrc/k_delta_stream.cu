@@ -410,8 +410,10 @@ __global__ void __launch_bounds__(kDSThreads, 1) delta_stream_kernel(const Delta
 cudaError_t launch_kernel(const DeltaStreamParams& p, int n_lanes, cudaStream_t st) {
   const size_t smem = 1024 + 32 * (size_t)p.s.d * 2 + 2 * (size_t)kStageBytes + 32 * 256;
   auto kern = delta_stream_kernel;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  int limit = 0;
+  cudaError_t e = dyn_smem_limit((const void*)kern, &limit);
   if (e != cudaSuccess) return e;
+  if (smem > (size_t)limit) return cudaErrorInvalidConfiguration;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(n_lanes, p.s_max, 1);
   cfg.blockDim = dim3(kDSThreads, 1, 1);

@@ -731,8 +731,10 @@ cudaError_t launch_qproj(const DecodeArgs& a, cudaStream_t st) {
   if (!make_tmap_f16(&tmWq, a.Wq, s.d, s.d, s.d, 64, 128) || !make_tmap_f16(&tmH, a.h_new, a.n_lanes, s.d, s.d, 64, w.nb) ||
       !make_tmap_f16(&tmWk, a.Wk, s.d, s.d, s.d, 64, 64))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(qproj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lay.total);
+  int limit = 0;
+  cudaError_t e = dyn_smem_limit((const void*)qproj_kernel, &limit);
   if (e != cudaSuccess) return e;
+  if (lay.total > (uint32_t)limit) return cudaErrorInvalidConfiguration;
   QProjParams p{s,
                 a.iter,
                 a.loops,
@@ -772,8 +774,10 @@ cudaError_t launch_oproj(const DecodeArgs& a, cudaStream_t st) {
   const OProjLayout lay(s, w.nb, CL, a.n_lanes, w.s_max);
   alignas(64) CUtensorMap tmWv;
   if (!make_tmap_f16(&tmWv, a.Wv, s.d, s.d, s.d, 64, 128)) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(oproj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lay.total);
+  int limit = 0;
+  cudaError_t e = dyn_smem_limit((const void*)oproj_kernel, &limit);
   if (e != cudaSuccess) return e;
+  if (lay.total > (uint32_t)limit) return cudaErrorInvalidConfiguration;
   OProjParams p{s,
                 a.iter,
                 a.loops,

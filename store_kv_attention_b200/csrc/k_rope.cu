@@ -349,8 +349,9 @@ cudaError_t launch_rope_scores(const DecodeArgs& a, float rope_base, float2* cs,
   alignas(64) CUtensorMap tmWk;
   if (!make_tmap_f16(&tmWk, a.Wk, s.d, s.d, s.d, 64, 128)) return cudaErrorInvalidValue;
   const size_t smem = 1024 + 2 * (size_t)kATile + 2 * (size_t)NP * 128 + (size_t)NP * 4;
-  e = cudaFuncSetAttribute(rope_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
+  int limit = 0;
+  if ((e = dyn_smem_limit((const void*)rope_score_kernel, &limit)) != cudaSuccess) return e;
+  if (smem > (size_t)limit) return cudaErrorInvalidConfiguration;
   RopeScoreParams p{s, a.iter, a.loops, a.ctx_len, (const uint8_t*)a.codes, (const uint8_t*)a.scales, qrot,
                     (const float2*)cs, scores, reinterpret_cast<uint32_t*>(a.ws + a.wl.status_off), NP};
   cfg.gridDim = dim3((unsigned)((s.max_ctx + 127) / 128), (unsigned)(s.d / NP), (unsigned)a.n_lanes);

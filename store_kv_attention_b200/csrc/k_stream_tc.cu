@@ -860,16 +860,13 @@ cudaError_t launch_fmt(const DecodeArgs& a, const CUtensorMap& tmap, cudaStream_
   const Shape& s = a.s;
   constexpr int NP = SPLIT ? 32 : 16;
   auto kern = stream_tc_kernel<FMT, SPLIT>;
-  cudaFuncAttributes fa;
-  cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+  int limit = 0;
+  cudaError_t e = dyn_smem_limit((const void*)kern, &limit);
   if (e != cudaSuccess) return e;
-  int dev = 0, optin = 0;
-  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-  if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
   // fixed regions (+ up to 1 KB of alignment), then as many 16 KB ring slots as fit, shared
   // between the score-side and the P.V-side rings
   const size_t fixed = 1024 + qimg_bytes(s.d) + 2 * (size_t)kPvStageBytes + 2 * (size_t)NP * 256;
-  const long long room = (long long)optin - (long long)fa.sharedSizeBytes - (long long)fixed;
+  const long long room = (long long)limit - (long long)fixed;
   const int slots = room > 0 ? (int)(room / kSlotBytes) : 0;
   using F = Fmt<FMT>;
   // ring sizes: about half the slots each, multiples of the sub-ring counts
@@ -877,7 +874,6 @@ cudaError_t launch_fmt(const DecodeArgs& a, const CUtensorMap& tmap, cudaStream_
   const int v_ring = std::min(kMaxRing, (slots - s_ring) / F::kOwnersV * F::kOwnersV);
   if (v_ring < F::kOwnersV || v_ring < 2 || s_ring < 2) return cudaErrorInvalidConfiguration;
   const size_t smem = fixed + (size_t)(s_ring + v_ring) * kSlotBytes;
-  if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
   StreamParams p{s,
                  a.iter,
                  a.loops,

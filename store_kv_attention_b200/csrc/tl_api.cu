@@ -4,6 +4,8 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "delta_internal.cuh"
 #include "tl_delta.h"
 #include "tl_internal.cuh"
@@ -117,6 +119,37 @@ void profile_stream_begin(cudaStream_t st) {
 void profile_stream_end(cudaStream_t st) {
   tl_profile* p = current_profile();
   if (p && p->recorded < p->capacity) cudaEventRecord((cudaEvent_t)p->end_events[p->recorded++], st);
+}
+
+cudaError_t dyn_smem_limit(const void* func, int* limit) {
+  struct Entry {
+    const void* func;
+    int dev, limit;
+  };
+  static std::mutex mu;
+  static Entry table[64];
+  static int n_entries = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < n_entries; ++i)
+      if (table[i].func == func && table[i].dev == dev) {
+        *limit = table[i].limit;
+        return cudaSuccess;
+      }
+  }
+  cudaFuncAttributes fa;
+  if ((e = cudaFuncGetAttributes(&fa, func)) != cudaSuccess) return e;
+  int optin = 0;
+  if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
+  const int lim = optin - (int)fa.sharedSizeBytes;
+  if ((e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, lim)) != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  if (n_entries < 64) table[n_entries++] = Entry{func, dev, lim};  // a full table only costs re-queries
+  *limit = lim;
+  return cudaSuccess;
 }
 
 }  // namespace tl

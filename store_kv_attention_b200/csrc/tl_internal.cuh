@@ -170,6 +170,13 @@ inline void count_launch(int n = 1) {
 void profile_stream_begin(cudaStream_t st);      // records begin_events[recorded] if installed
 void profile_stream_end(cudaStream_t st);        // records end_events[recorded++] if installed
 
+// ---------------------------------------------------------------- kernel launch limits
+// The largest dynamic shared memory a launch of `func` may request on the current device.  The
+// kernel is opted into it (cudaFuncAttributeMaxDynamicSharedMemorySize = the device's per-block
+// opt-in limit minus the kernel's static shared memory) the first time, and the limit is cached
+// per (kernel, device), so a decode call costs no attribute queries after the first (tl_api.cu).
+cudaError_t dyn_smem_limit(const void* func, int* limit);
+
 // ---------------------------------------------------------------- launchers (return cudaError_t)
 cudaError_t launch_append(const Shape& s, void* codes, void* scales, int layer, const __half* h_rows,
                           int n_lanes, int n_rows, const int32_t* start_pos, const int32_t* row_count,
