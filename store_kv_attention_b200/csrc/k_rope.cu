@@ -33,7 +33,7 @@ namespace {
 
 using namespace ptx;
 
-constexpr int kRThreads = 128;
+constexpr int kRThreads = 256;  // two threads per row of the tile, one per half of each 64-value K slice
 constexpr int kATile = 128 * 64 * 2;  // 128 rows x 64 fp16, K-major, 128-byte swizzle
 constexpr long long kRWait = 4000000000ll;
 
@@ -107,10 +107,10 @@ struct RopeScoreParams {
   int n_pass;          // K columns per CTA (a multiple of hd, at most 512)
 };
 
-// The raw codes of the 64 values [k0, k0 + 64) of one cached row (and, for INT4, their group
+// The raw codes of the 32 values [k0, k0 + 32) of one cached row (and, for INT4, their group
 // scale), loaded one K-step ahead of their use so that the loads are in flight during the MMAs.
 struct RowSlice {
-  uint4 v[8];
+  uint4 v[4];
   __half sc;
 };
 __device__ __forceinline__ void load_row(const Shape& s, const uint8_t* codes, const uint8_t* scales, size_t row,
@@ -119,62 +119,74 @@ __device__ __forceinline__ void load_row(const Shape& s, const uint8_t* codes, c
   if (s.fmt == TL_H_FP16) {
     const uint4* src = reinterpret_cast<const uint4*>(codes + row * (size_t)(2 * s.d) + 2 * k0);
 #pragma unroll
-    for (int v = 0; v < 8; ++v) x.v[v] = __ldg(src + v);
+    for (int v = 0; v < 4; ++v) x.v[v] = __ldg(src + v);
   } else if (s.fmt == TL_H_INT8_TOKEN) {
     const uint4* src = reinterpret_cast<const uint4*>(codes + row * (size_t)s.d + k0);
-#pragma unroll
-    for (int v = 0; v < 4; ++v) x.v[v] = __ldg(src + v);
-  } else {
-    const uint4* src = reinterpret_cast<const uint4*>(codes + row * (size_t)(s.d / 2) + k0 / 2);
     x.v[0] = __ldg(src);
     x.v[1] = __ldg(src + 1);
+  } else {
+    x.v[0] = __ldg(reinterpret_cast<const uint4*>(codes + row * (size_t)(s.d / 2) + k0 / 2));
     x.sc = reinterpret_cast<const __half*>(scales)[row * (size_t)(s.d / kInt4Group) + k0 / kInt4Group];
   }
 }
 
-// The loaded slice as fp16 pairs into a K-major swizzled A tile.  FP16 rows are copied, INT8
-// codes are converted exactly (the row scale is applied to the scores), INT4 codes are
-// multiplied by their group scale (rounded once to fp16).  Rows outside the lane give zeros.
-__device__ __forceinline__ void stage_row(const Shape& s, const RowSlice& x, bool valid, uint8_t* tile, int r) {
-  uint32_t h[32];
+// The loaded slice as fp16 pairs into half `hf` of row r of a K-major swizzled A tile, in the
+// natural K order.  FP16 rows are copied; INT8 codes and INT4 codes are converted exactly by the
+// exponent-bias ("magic number") identity of IEEE binary16 (a small integer n in the low
+// mantissa bits of 2^10 reads as 1024 + n; the method as used for INT4/INT8 dequantisation is
+// described by Kim et al., "Who Says Elephants Can't Run", arXiv:2211.10017), INT4 then
+// multiplied by its group scale (rounded once to fp16); the INT8 row scale is applied to the
+// scores.  Rows outside the lane give zeros.
+__device__ __forceinline__ void stage_row(const Shape& s, const RowSlice& x, bool valid, uint8_t* tile, int r, int hf) {
+  uint32_t h[16];
   if (!valid) {
 #pragma unroll
-    for (int i = 0; i < 32; ++i) h[i] = 0u;
+    for (int i = 0; i < 16; ++i) h[i] = 0u;
   } else if (s.fmt == TL_H_FP16) {
 #pragma unroll
-    for (int v = 0; v < 8; ++v) {
+    for (int v = 0; v < 4; ++v) {
       h[4 * v] = x.v[v].x;
       h[4 * v + 1] = x.v[v].y;
       h[4 * v + 2] = x.v[v].z;
       h[4 * v + 3] = x.v[v].w;
     }
   } else if (s.fmt == TL_H_INT8_TOKEN) {
+    const __half2 bias = __halves2half2(__float2half_rn(1152.0f), __float2half_rn(1152.0f));
 #pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      const int8_t* c = reinterpret_cast<const int8_t*>(&x.v[v]);
+    for (int v = 0; v < 2; ++v) {
+      const uint32_t w[4] = {x.v[v].x, x.v[v].y, x.v[v].z, x.v[v].w};
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const __half2 p = __halves2half2(__int2half_rn(c[2 * i]), __int2half_rn(c[2 * i + 1]));
-        h[8 * v + i] = *reinterpret_cast<const uint32_t*>(&p);
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t y = w[q] ^ 0x80808080u;            // offset binary: code + 128
+        const uint32_t a = prmt(y, 0x64646464u, 0x5140u);  // (1024 + b0, 1024 + b1)
+        const uint32_t c = prmt(y, 0x64646464u, 0x7362u);  // (b2, b3)
+        const __half2 ha = __hsub2(*reinterpret_cast<const __half2*>(&a), bias);
+        const __half2 hc = __hsub2(*reinterpret_cast<const __half2*>(&c), bias);
+        h[8 * v + 2 * q] = *reinterpret_cast<const uint32_t*>(&ha);
+        h[8 * v + 2 * q + 1] = *reinterpret_cast<const uint32_t*>(&hc);
       }
     }
   } else {
     const __half2 s2 = __halves2half2(x.sc, x.sc);
+    const __half2 bias = __halves2half2(__float2half_rn(1032.0f), __float2half_rn(1032.0f));
+    const uint32_t w[4] = {x.v[0].x, x.v[0].y, x.v[0].z, x.v[0].w};
 #pragma unroll
-    for (int v = 0; v < 2; ++v) {
-      const uint8_t* by = reinterpret_cast<const uint8_t*>(&x.v[v]);
+    for (int q = 0; q < 4; ++q) {  // word q: values 8 q .. 8 q + 7, low nibble first
+      const uint32_t t = w[q] & 0x0F0F0F0Fu, u = (w[q] >> 4) & 0x0F0F0F0Fu;  // even / odd values
+      const uint32_t sel[4] = {0x4400u, 0x5511u, 0x6622u, 0x7733u};           // pair (2k, 2k + 1)
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int lo = (int)(by[i] & 0xF), hi = (int)(by[i] >> 4);
-        const __half2 p = __halves2half2(__int2half_rn(lo >= 8 ? lo - 16 : lo), __int2half_rn(hi >= 8 ? hi - 16 : hi));
-        const __half2 y = __hmul2(p, s2);
-        h[16 * v + i] = *reinterpret_cast<const uint32_t*>(&y);
+      for (int k = 0; k < 4; ++k) {
+        // (nibble ^ 8) = code + 8 in the mantissa of 1024: 1032 + code, exact
+        const uint32_t pr = lop3_and_xor(prmt(t, u, sel[k]), 0x000F000Fu, 0x64086408u);
+        const __half2 y = __hmul2(__hsub2(*reinterpret_cast<const __half2*>(&pr), bias), s2);
+        h[4 * q + k] = *reinterpret_cast<const uint32_t*>(&y);
       }
     }
   }
 #pragma unroll
-  for (int v = 0; v < 8; ++v)
-    *reinterpret_cast<uint4*>(tile + r * 128 + ((v ^ (r & 7)) << 4)) = make_uint4(h[4 * v], h[4 * v + 1], h[4 * v + 2], h[4 * v + 3]);
+  for (int v = 0; v < 4; ++v)
+    *reinterpret_cast<uint4*>(tile + r * 128 + (((4 * hf + v) ^ (r & 7)) << 4)) =
+        make_uint4(h[4 * v], h[4 * v + 1], h[4 * v + 2], h[4 * v + 3]);
 }
 
 __device__ __forceinline__ bool block_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
@@ -182,7 +194,8 @@ __device__ __forceinline__ bool block_wait(uint64_t* bar, uint32_t parity, volat
   return __syncthreads_and(w) != 0;
 }
 
-// grid (tiles of 128 rows, column blocks of n_pass, lanes), block 128 (thread r = tile row r)
+// grid (tiles of 128 rows, column blocks of n_pass, lanes), block 256: thread t takes row
+// r = t & 127 of the tile and half t >> 7 of each 64-value K slice
 __global__ void __launch_bounds__(kRThreads, 1)
     rope_score_kernel(const __grid_constant__ CUtensorMap tmWk, const RopeScoreParams p) {
   const Shape& s = p.s;
@@ -203,8 +216,8 @@ __global__ void __launch_bounds__(kRThreads, 1)
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
 
-  const int warp = threadIdx.x >> 5, r = threadIdx.x;
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const int warp = threadIdx.x >> 5, r = threadIdx.x & 127, hf = threadIdx.x >> 7;
+  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;  // TMEM lane quarter of the warp = rows r
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&full[i], 1);
@@ -232,18 +245,26 @@ __global__ void __launch_bounds__(kRThreads, 1)
   const size_t grow = ((size_t)(s.n_pre + p.iter) * s.max_lanes + b) * s.max_ctx + (size_t)row;
   const uint32_t idesc = idesc_f16_f32(128, 256, false, false);
   bool ok = true, issued = false;
+  // W_k tiles of K-step k go into stage k & 1.  Step k stages its A slice while the MMAs of step
+  // k - 1 run, issues its own MMAs, then waits for those of step k - 1 and loads the W_k tiles of
+  // step k + 1 into the stage they freed, so each W_k load has a whole MMA period to land.
+  int b_issued = 0;  // W_k loads issued (K-steps 0 .. b_issued - 1)
+  auto load_b = [&](int ks) {
+    const int st = ks & 1;
+    mbar_expect_tx(&full[st], (uint32_t)NP * 128);
+    for (int nb = 0; nb < NP / 128; ++nb) tma_load_2d(B[st] + nb * 16384, &tmWk, ks * 64, cb * NP + nb * 128, &full[st]);
+  };
+  if (threadIdx.x == 0) {
+    load_b(0);
+    b_issued = 1;
+  }
   RowSlice nxt;
-  load_row(s, p.codes, p.scales, grow, valid, 0, nxt);
+  load_row(s, p.codes, p.scales, grow, valid, 32 * hf, nxt);
   for (int ks = 0; ks < n_ks && ok; ++ks) {
     const int st = ks & 1, use = ks >> 1;
-    if (ks >= 2 && !(ok = block_wait(&empty[st], (use - 1) & 1, abort_p))) break;
-    if (threadIdx.x == 0) {
-      mbar_expect_tx(&full[st], (uint32_t)NP * 128);
-      for (int nb = 0; nb < NP / 128; ++nb)
-        tma_load_2d(B[st] + nb * 16384, &tmWk, ks * 64, cb * NP + nb * 128, &full[st]);
-    }
-    stage_row(s, nxt, valid, A[st], r);
-    if (ks + 1 < n_ks) load_row(s, p.codes, p.scales, grow, valid, (ks + 1) * 64, nxt);  // in flight during the MMAs
+    // A[st] was last read by the MMAs of step ks - 2, waited for at step ks - 1
+    stage_row(s, nxt, valid, A[st], r, hf);
+    if (ks + 1 < n_ks) load_row(s, p.codes, p.scales, grow, valid, (ks + 1) * 64 + 32 * hf, nxt);  // in flight during the MMAs
     fence_proxy_async_smem();
     __syncthreads();
     if (warp == 0) {
@@ -265,7 +286,13 @@ __global__ void __launch_bounds__(kRThreads, 1)
       }
     }
     issued = true;
-    ok = __syncthreads_and(!*abort_p) != 0;
+    if (!(ok = __syncthreads_and(!*abort_p) != 0)) break;
+    // the MMAs of step ks - 1 are done: stage st ^ 1 is free for the W_k tiles of step ks + 1
+    if (ks >= 1 && !(ok = block_wait(&empty[st ^ 1], ((ks - 1) >> 1) & 1, abort_p))) break;
+    if (threadIdx.x == 0 && ks + 1 < n_ks) {
+      load_b(ks + 1);
+      b_issued = ks + 2;
+    }
   }
   // the last K-step's MMAs complete on empty[(n_ks - 1) & 1]
   if (ok) ok = block_wait(&empty[(n_ks - 1) & 1], ((n_ks - 1) >> 1) & 1, abort_p);
@@ -277,7 +304,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
     const int half = s.hd / 2;
     const float2* cs = p.cs + (size_t)(valid ? row : 0) * half;
     const float sr = (s.fmt == TL_H_INT8_TOKEN && valid) ? reinterpret_cast<const float*>(p.scales)[grow] : 1.0f;
-    for (int h = 0; h < NP / s.hd; ++h) {
+    for (int h = hf; h < NP / s.hd; h += 2) {  // the two warps of a lane quarter take alternate heads
       float acc = 0.0f;
       for (int i0 = 0; i0 < half; i0 += 16) {
         uint32_t k1[16], k2[16];
@@ -310,6 +337,14 @@ __global__ void __launch_bounds__(kRThreads, 1)
       while (!mbar_try_wait(&fin, 0) && clock64() - t0 < kRWait) {
       }
     }
+    if (!ok && threadIdx.x == 0)
+      // nor may a W_k load still be writing shared memory when the CTA exits: the latest load of
+      // each stage (bounded waits)
+      for (int k = b_issued - 1; k >= 0 && k >= b_issued - 2; --k) {
+        const long long t1 = clock64();
+        while (!mbar_try_wait(&full[k & 1], (k >> 1) & 1) && clock64() - t1 < kRWait) {
+        }
+      }
     tc_fence_after();
     tmem_dealloc(tbase, NP <= 256 ? 256 : 512);
   }
