@@ -89,17 +89,29 @@ __device__ __forceinline__ void rebuild32(const DeltaStreamParams& p, size_t row
   }
   const size_t level_rows = (size_t)s.max_lanes * s.max_ctx;
   const int head = k0 / s.hd;
-  for (int l = 1; l <= p.iter; ++l) {
-    const size_t lr = (size_t)(l - 1) * level_rows + row;
-    const float sc = __half2float(p.scales[lr * s.H + head]);
-    const uint4* c = reinterpret_cast<const uint4*>(p.deltas + lr * s.d + k0);
+  // levels four at a time: their loads are issued together, then added in level order
+  for (int l0 = 1; l0 <= p.iter; l0 += 4) {
+    uint4 cw[4][2];
+    float sc[4];
 #pragma unroll
-    for (int v = 0; v < 2; ++v) {
-      const uint4 w = __ldg(c + v);
-      const int8_t* b = reinterpret_cast<const int8_t*>(&w);
+    for (int j = 0; j < 4; ++j)
+      if (l0 + j <= p.iter) {
+        const size_t lr = (size_t)(l0 + j - 1) * level_rows + row;
+        sc[j] = __half2float(p.scales[lr * s.H + head]);
+        const uint4* c = reinterpret_cast<const uint4*>(p.deltas + lr * s.d + k0);
+        cw[j][0] = __ldg(c);
+        cw[j][1] = __ldg(c + 1);
+      }
 #pragma unroll
-      for (int i = 0; i < 16; ++i) acc[16 * v + i] = __fadd_rn(acc[16 * v + i], __fmul_rn((float)b[i], sc));
-    }
+    for (int j = 0; j < 4; ++j)
+      if (l0 + j <= p.iter) {
+#pragma unroll
+        for (int v = 0; v < 2; ++v) {
+          const int8_t* b = reinterpret_cast<const int8_t*>(&cw[j][v]);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) acc[16 * v + i] = __fadd_rn(acc[16 * v + i], __fmul_rn((float)b[i], sc[j]));
+        }
+      }
   }
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
