@@ -484,3 +484,21 @@ def test_split_rows_option_matches_oracle_and_solo(name, ctx, loops, split):
         solo.step(fused_append=True)
         torch.cuda.synchronize()
         assert np.array_equal(out[:, b].view(np.uint32), solo.out[:, 0].cpu().numpy().view(np.uint32)), f"lane {b}"
+
+
+def test_call_with_no_active_lane_writes_nothing():
+    """Every lane past its loop count at this iteration: the call launches, writes no output,
+    appends no row, leaves the flags alone and reports nothing."""
+    import store_kv_attention_b200 as tl
+    w = _small("int4_2b", [5, 300, 1500], [2, 1, 3])
+    w.L_max = 4
+    dw = _dw(w)
+    before = dw.cache.codes.clone()
+    it = 3                                  # every lane has loops <= 3
+    dw.out[it].fill_(float("nan"))
+    dw.decode(it, append=True)
+    torch.cuda.synchronize()
+    assert np.all(np.isnan(dw.out[it].cpu().numpy()))
+    assert torch.equal(before, dw.cache.codes)
+    assert np.all(dw.flags.cpu().numpy() == 0) and np.all(dw.first.cpu().numpy() == -1)
+    assert tl.poll_status(dw.cache) == tl.TL_OK
