@@ -18,8 +18,8 @@
 // oproj (one launch):  u_j = sum_s w_s U_sj (the exact merge of the splits), out_j = W_v[j] u_j
 //   Rank k of cluster mb merges the K-slice k of u for the block's heads and every lane into
 //   an fp16 hi/lo B operand, multiplies it by its W_v tiles, and the ranks' partial outputs
-//   are summed in rank order through distributed shared memory.  Each CTA also runs the
-//   FP64 safety check of one lane.
+//   are summed in rank order through distributed shared memory.  The CTAs also run the
+//   FP64 safety check, the lanes dealt out over them in turn.
 //
 // Every reduction runs in a fixed order, so a lane's result does not depend on the
 // other lanes of the batch or on scheduling.  All mbarrier waits are bounded; every
@@ -400,7 +400,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
 //   as a separate merge), writes it as the fp16 hi/lo B operand in shared memory, and
 //   multiplies it with its W_v tile (prefetched at kernel start).  The K slices are reduced
 //   through DSMEM in rank order, as in qproj.  CTA (k, mb) also runs the per-iteration
-//   safety check of lane mb * CL + k.
+//   safety check of lanes mb * CL + k, mb * CL + k + the CTA count, ...
 struct OProjParams {
   Shape s;
   int iter;
@@ -490,10 +490,12 @@ __global__ void __launch_bounds__(kOProjThreads, 1)
 
   __shared__ uint64_t act_slot;
   const uint64_t act = active_mask(s, p.iter, p.loops, p.ctx_len, p.n_lanes, &act_slot);
-  // the safety check of one lane per CTA (it depends only on the residual)
-  const int nl = mb * CL + k;
-  if (p.residual && nl < p.n_lanes && ((act >> nl) & 1))
-    norm_check_lane<kOProjThreads>(p.residual, nl, s.d, p.threshold, p.iter, p.flags, p.first, p.norms);
+  // the safety check of lanes mb * CL + k, + the CTA count, ... (it depends only on the residual;
+  // the trip count and the lane's activity are the same for every thread of the CTA)
+  if (p.residual)
+    for (int nl = mb * CL + k; nl < p.n_lanes; nl += CL * (int)gridDim.y)
+      if ((act >> nl) & 1)
+        norm_check_lane<kOProjThreads>(p.residual, nl, s.d, p.threshold, p.iter, p.flags, p.first, p.norms);
 
   pdl_wait();     // the split partials come from the streaming kernel just before
   pdl_trigger();  // TMEM is held
@@ -714,8 +716,14 @@ bool make_tmap_f16(void* tmap, const void* base, uint64_t rows, uint64_t cols, u
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Cluster size of the projection kernels: K splits of d, each a multiple of 64 wide.
-int proj_cluster(int d) { return d / 64 < 8 ? d / 64 : 8; }
+// Cluster size of the projection kernels: the largest power of two up to 8 that divides d / 64,
+// so that every K slice (d / CL) is a whole number of 64-value tiles and every rank's share of
+// the 128 rows of a block (128 / CL) is a whole number of 8-row groups.
+int proj_cluster(int d) {
+  int cl = 8;
+  while (cl > 1 && (d / 64) % cl != 0) cl >>= 1;
+  return cl;
+}
 
 // Dynamic shared memory oproj_kernel needs for a call (its merge weights grow with the splits).
 size_t oproj_smem_bytes(const Shape& s, int n_lanes, int s_max) {

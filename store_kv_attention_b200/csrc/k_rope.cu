@@ -355,7 +355,8 @@ __global__ void __launch_bounds__(kRThreads, 1)
 bool make_tmap_f16(void* tmap, const void* base, uint64_t rows, uint64_t cols, uint64_t pitch_elems,
                    uint32_t box_cols, uint32_t box_rows);
 
-int rope_pass_cols(const Shape& s) { return s.d < 512 ? s.d : 512; }
+// Output columns of K per CTA: 512 where they divide d_model, else 256 (d_model is a multiple of 256).
+int rope_pass_cols(const Shape& s) { return s.d % 512 == 0 ? 512 : 256; }
 
 cudaError_t launch_rope_scores(const DecodeArgs& a, float rope_base, float2* cs, float* qrot, float* scores,
                                cudaStream_t st) {

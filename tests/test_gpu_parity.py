@@ -306,8 +306,9 @@ def test_decode_full_size_sampled(name, samples):
 
 @pytest.mark.parametrize("fmt", [0, 1, 2])
 def test_fused_append_more_lanes_than_ctas(fmt):
-    """d = 256 runs the projection kernel on 8 CTAs, so with 40 lanes the fused append's lane
-    loop makes several trips per CTA."""
+    """d = 256 runs the projection kernels on 8 CTAs, so with 40 lanes the fused append's lane
+    loop and the safety check's lane loop make several trips per CTA (lanes 0-19 over the
+    threshold, 20-39 under it)."""
     import dataclasses
     base = get_workload("tiny_fp16")
     n = 40
@@ -315,7 +316,7 @@ def test_fused_append_more_lanes_than_ctas(fmt):
     ctx[3], ctx[5] = 0, 1
     loops = [1 + (b % 3) for b in range(n)]
     w = dataclasses.replace(base, fmt=fmt, ctx=ctx, loops=loops, L_max=3, name=f"d256_fmt{fmt}_40lanes",
-                            outlier_p=0.01 if fmt == 1 else 0.0, outlier_mul=8.0)
+                            outlier_p=0.01 if fmt == 1 else 0.0, outlier_mul=8.0, forced_lanes=20)
     sep, fus = _dw(w, flag_mix=True, fill=False), _dw(w, flag_mix=True, fill=False)
     for dw in (sep, fus):
         dw.cache.codes.fill_(0x5A)
@@ -331,6 +332,13 @@ def test_fused_append_more_lanes_than_ctas(fmt):
     a = fus.out.cpu().numpy()
     assert np.array_equal(a.view(np.uint32), sep.out.cpu().numpy().view(np.uint32))
     assert torch.equal(sep.flags, fus.flags) and torch.equal(sep.first, fus.first)
+    # the safety check of every lane (more lanes than CTAs: each CTA checks several)
+    f = np.zeros(w.B, np.uint8)
+    fi = np.full(w.B, -1, np.int32)
+    for it in range(w.L_max):
+        f, fi, _ = oracle.cpp.residual_norm_check(w.residual(it, True), w.threshold, it, np.array(w.loops), f, fi)
+    assert 0 < f.sum() < w.B
+    assert np.array_equal(fus.flags.cpu().numpy(), f) and np.array_equal(fus.first.cpu().numpy(), fi)
     for it in range(w.L_max):
         bs = [b for b in range(w.B) if it < w.loops[b]]
         want_c, want_s = oracle.cpp.quantize_rows(w.h_new(it)[bs], w.fmt)

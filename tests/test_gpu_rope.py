@@ -87,3 +87,30 @@ def test_rope_decode_long_context():
         err = np.abs(g - want).max()
         rel = np.linalg.norm(g - want) / np.linalg.norm(want)
         assert err <= MAX_ABS and rel <= REL_L2, f"lane {b}: max-abs {err:.3g} rel-L2 {rel:.3g}"
+
+
+@pytest.mark.parametrize("d,H,hd,fmt", [(768, 12, 64, 0), (1536, 12, 128, 2)], ids=["d768_fp16", "d1536_int4"])
+def test_rope_decode_d_model_not_a_multiple_of_512(d, H, hd, fmt):
+    """Every head's scores when 512 does not divide d_model (the K columns in blocks of 256)."""
+    import store_kv_attention_b200 as tl
+    from synth.device import DeviceWorkload
+    from synth.workloads import Workload
+    w = Workload(name=f"rope_d{d}", d=d, H=H, hd=hd, n_pre=1, L_max=1, fmt=fmt, seed=77, ctx=[300, 1025],
+                 loops=[1, 1], residual_scale=1.0, threshold=50.0)
+    dw = DeviceWorkload(w)
+    ws = torch.zeros(tl.rope_workspace_bytes(dw.desc, w.B), dtype=torch.uint8, device="cuda")
+    dw.append_new(0)
+    tl.attn_decode_rope(dw.cache, 0, dw.loops, dw.ctx, dw.h_new[0], dw.W["q"], dw.W["k"], dw.W["v"], dw.out[0], ws)
+    torch.cuda.synchronize()
+    assert tl.poll_status(ws) == tl.TL_OK
+    got = dw.out[0].cpu().numpy()
+    W = [w.weight(k) for k in "qkv"]
+    for b in range(w.B):
+        rows = np.concatenate([w.h_rows(w.n_pre, b, 0, w.ctx[b]), w.h_new(0)[b:b + 1]])
+        c, s_ = oracle.cpp.quantize_rows(rows, w.fmt)
+        hh = oracle.cpp.dequantize_rows(c, s_, w.fmt, w.d)
+        want = rope_oracle.attend_rope(hh, w.h_new(0)[b], *W, w.H, w.hd)
+        g = got[b].astype(np.float64)
+        err = np.abs(g - want).max()
+        rel = np.linalg.norm(g - want) / np.linalg.norm(want)
+        assert err <= MAX_ABS and rel <= REL_L2, f"lane {b}: max-abs {err:.3g} rel-L2 {rel:.3g}"
