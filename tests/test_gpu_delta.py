@@ -106,6 +106,8 @@ def _weights(seed, d):
     (1024, 16, 3, [500, 64], 600),
     (1024, 16, 8, [1030, 5], 1100),      # deep levels, a context over two splits
     (2048, 16, 4, [1100, 300], 1200),    # the 2B-like shape
+    (768, 12, 3, [300, 40], 400),        # projection clusters of 4 (d_model / 64 = 12)
+    (1280, 10, 3, [200, 700], 800),
 ])
 def test_decode_matches_oracle(d, H, L_max, ctx, max_ctx):
     import oracle

@@ -215,3 +215,35 @@ def test_prefill_long_chunk_spans_groups():
         for t in (0, 1, 63, 64, 69):
             want = oracle.cpp.attend_absorbed(hh[: w.ctx[b] + t + 1], chunk[b, t], *W, w.H, w.hd)
             _close(got[b, t], want, f"lane {b} token {t}")
+
+
+
+@pytest.mark.parametrize("d,H,hd,fmt", [(768, 12, 64, 0), (1280, 10, 128, 2)], ids=["d768_fp16", "d1280_int4"])
+def test_tree_verify_unusual_shapes(d, H, hd, fmt):
+    """Tree verification where the projection kernels run on clusters of 4 (d_model / 64 = 12, 20)."""
+    import store_kv_attention_b200 as tl
+    from synth.device import DeviceWorkload
+    from synth.workloads import Workload
+    K, D, it = 2, 3, 0
+    w = Workload(name=f"tree_d{d}", d=d, H=H, hd=hd, n_pre=1, L_max=1, fmt=fmt, seed=57, ctx=[0, 129, 1030],
+                 loops=[1, 1, 1], residual_scale=1.0, threshold=50.0)
+    dw = DeviceWorkload(w, max_ctx=max(w.ctx) + K * D + 1)
+    h_tree = _tree_states(w, it, K, D)
+    ws = torch.zeros(tl.verify_workspace_bytes(dw.desc, w.B, K, D), dtype=torch.uint8, device="cuda")
+    out = torch.full((w.B, K, D, w.H, w.hd), float("nan"), dtype=torch.float32, device="cuda")
+    tl.verify_attn(dw.cache, it, dw.loops, dw.ctx, _f16(h_tree), dw.W["q"], dw.W["k"], dw.W["v"], out, ws)
+    torch.cuda.synchronize()
+    assert tl.poll_status(ws) == tl.TL_OK
+    got = out.cpu().numpy()
+    W = [w.weight(k) for k in "qkv"]
+    layer = w.n_pre + it
+    for b in range(w.B):
+        cc, cs = oracle.cpp.quantize_rows(w.h_rows(layer, b, 0, w.ctx[b]), w.fmt)
+        h_ctx = oracle.cpp.dequantize_rows(cc, cs, w.fmt, w.d)
+        tc, ts = oracle.cpp.quantize_rows(h_tree[b].reshape(K * D, w.d), w.fmt)
+        h_rows = oracle.cpp.dequantize_rows(tc, ts, w.fmt, w.d).reshape(K, D, w.d)
+        for k in range(K):
+            for t in range(D):
+                rows = tree_oracle.tree_rows(h_ctx, h_rows, k, t)
+                want = oracle.cpp.attend_absorbed(rows, h_tree[b, k, t], *W, w.H, w.hd)
+                _close(got[b, k, t], want, f"d {d} lane {b} branch {k} depth {t}")
