@@ -247,3 +247,33 @@ def test_tree_verify_unusual_shapes(d, H, hd, fmt):
                 rows = tree_oracle.tree_rows(h_ctx, h_rows, k, t)
                 want = oracle.cpp.attend_absorbed(rows, h_tree[b, k, t], *W, w.H, w.hd)
                 _close(got[b, k, t], want, f"d {d} lane {b} branch {k} depth {t}")
+
+
+def test_large_tree_over_groups_and_tiles():
+    """8 branches x 20 tokens on 2 lanes: 320 query tokens in 5 groups of the decode kernels, each
+    token's own-branch rows crossing a 128-row tile edge for the second lane."""
+    import store_kv_attention_b200 as tl
+    from synth.device import DeviceWorkload
+    K, D, it = 8, 20, 0
+    w = _workload(2, [5, 100], [1, 1], L_max=1)
+    dw = DeviceWorkload(w, max_ctx=max(w.ctx) + K * D + 1)
+    h_tree = _tree_states(w, it, K, D)
+    ws = torch.zeros(tl.verify_workspace_bytes(dw.desc, w.B, K, D), dtype=torch.uint8, device="cuda")
+    out = torch.full((w.B, K, D, w.H, w.hd), float("nan"), dtype=torch.float32, device="cuda")
+    tl.verify_attn(dw.cache, it, dw.loops, dw.ctx, _f16(h_tree), dw.W["q"], dw.W["k"], dw.W["v"], out, ws)
+    torch.cuda.synchronize()
+    assert tl.poll_status(ws) == tl.TL_OK
+    got = out.cpu().numpy()
+    assert np.all(np.isfinite(got))
+    W = [w.weight(k) for k in "qkv"]
+    layer = w.n_pre + it
+    for b in range(w.B):
+        cc, cs = oracle.cpp.quantize_rows(w.h_rows(layer, b, 0, w.ctx[b]), w.fmt)
+        h_ctx = oracle.cpp.dequantize_rows(cc, cs, w.fmt, w.d)
+        tc, ts = oracle.cpp.quantize_rows(h_tree[b].reshape(K * D, w.d), w.fmt)
+        h_rows = oracle.cpp.dequantize_rows(tc, ts, w.fmt, w.d).reshape(K, D, w.d)
+        for k in (0, 3, 7):
+            for t in (0, 1, 19):
+                rows = tree_oracle.tree_rows(h_ctx, h_rows, k, t)
+                want = oracle.cpp.attend_absorbed(rows, h_tree[b, k, t], *W, w.H, w.hd)
+                _close(got[b, k, t], want, f"lane {b} branch {k} depth {t}")
