@@ -336,20 +336,27 @@ def run_ours(args, rank, world, local_rank):
     # One step (every loop iteration's tl_storeh_append_attn_decode call) captured as a CUDA graph:
     # the same launches with the same arguments, replayed without the host's per-call overhead.
     run_step = lambda: dw.step(fused_append=True)
+    launch_mode = "eager calls"
     if not args.no_graph:
-        graph = torch.cuda.CUDAGraph()
-        side = torch.cuda.Stream()
-        side.wait_stream(stream)
-        with torch.cuda.stream(side):
-            dw.step(fused_append=True)
-        stream.wait_stream(side)
-        torch.cuda.synchronize()
-        with torch.cuda.graph(graph):
-            dw.step(fused_append=True)
-        run_step = graph.replay
-        for _ in range(max(3, args.warmup)):
-            run_step()
-        torch.cuda.synchronize()
+        try:
+            graph = torch.cuda.CUDAGraph()
+            side = torch.cuda.Stream()
+            side.wait_stream(stream)
+            with torch.cuda.stream(side):
+                dw.step(fused_append=True)
+            stream.wait_stream(side)
+            torch.cuda.synchronize()
+            with torch.cuda.graph(graph):
+                dw.step(fused_append=True)
+            for _ in range(max(3, args.warmup)):
+                graph.replay()
+            torch.cuda.synchronize()
+            run_step = graph.replay
+            launch_mode = ("replays of a CUDA graph of one step (the step's calls captured once); the kernel pass "
+                           "and e2e run as eager calls")
+        except RuntimeError as e:  # capture unsupported here: time eager calls and say so
+            torch.cuda.synchronize()
+            launch_mode = "eager calls (CUDA-graph capture failed: %s)" % str(e).splitlines()[0][:120]
         if tl.poll_status(dw.cache) != tl.TL_OK:
             raise RuntimeError("device status after graph warm-up: " + tl.lib.tl_last_error_message().decode())
 
@@ -483,10 +490,7 @@ def run_ours(args, rank, world, local_rank):
                                                  "timing": ("value and ms_per_step: K steps between one event "
                                                             "pair (no event between kernels); the median of K "
                                                             "per-step event pairs is reported beside it"),
-                                                 "launch": ("eager calls" if args.no_graph else
-                                                            "replays of a CUDA graph of one step (the step's "
-                                                            "calls captured once); the kernel pass and e2e "
-                                                            "run as eager calls"),
+                                                 "launch": launch_mode,
                                                  "step_frac_of_hbm_roofline": step_roofline_ms / (ms_max / K)}),
             "roofline": roofline,
             "cpu_baseline": cpu,
