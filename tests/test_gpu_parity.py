@@ -510,3 +510,43 @@ def test_call_with_no_active_lane_writes_nothing():
     assert torch.equal(before, dw.cache.codes)
     assert np.all(dw.flags.cpu().numpy() == 0) and np.all(dw.first.cpu().numpy() == -1)
     assert tl.poll_status(dw.cache) == tl.TL_OK
+
+
+def test_call_with_fewer_lanes_than_the_cache_holds():
+    """A cache sized for 8 lanes, called with its first 3: the rows are addressed with the cache's
+    lane stride, and each lane gives the bits of the 8-lane call (the lanes are independent)."""
+    import store_kv_attention_b200 as tl
+    w = _small("int8_b16", [3, 700, 1500, 20, 1030, 5, 260, 999], [2] * 8)
+    w.L_max = 2
+    full = _dw(w)
+    full.step()
+    torch.cuda.synchronize()
+    part = _dw(w)
+    n = 3
+    out = torch.full((w.L_max, n, w.H, w.hd), float("nan"), dtype=torch.float32, device="cuda")
+    for it in range(w.L_max):
+        part.append_new(it)
+        tl.attn_decode(part.cache, it, part.loops[:n], part.ctx[:n], part.h_new[it][:n].contiguous(), part.W["q"],
+                       part.W["k"], part.W["v"], out[it], residual=part.residual[it][:n].contiguous(),
+                       threshold=w.threshold, abort_flags=part.flags[:n], first_abort_iter=part.first[:n])
+    torch.cuda.synchronize()
+    assert tl.poll_status(part.cache) == tl.TL_OK
+    a, b = full.out[:, :n].cpu().numpy(), out.cpu().numpy()
+    assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+    assert torch.equal(full.flags[:n], part.flags[:n]) and torch.equal(full.first[:n], part.first[:n])
+
+
+def test_cache_without_pre_layers():
+    """n_pre = 0: the loop block's layers start at layer 0 of the cache."""
+    w = _small("tiny_fp16", [0, 77, 300], [2, 1, 2])
+    w.n_pre = 0
+    dw = _dw(w)
+    dw.step()
+    torch.cuda.synchronize()
+    out = dw.out.cpu().numpy()
+    for it in range(w.L_max):
+        for b in range(w.B):
+            if it < w.loops[b]:
+                _assert_close(out[it, b], _oracle_lane(w, it, b), f"n_pre 0 lane {b} it {it}")
+            else:
+                assert np.all(np.isnan(out[it, b]))
