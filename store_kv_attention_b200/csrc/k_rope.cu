@@ -42,7 +42,8 @@ __global__ void rope_table_kernel(int rows, int half, int hd, double base, float
   ptx::pdl_trigger();
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= rows * half) return;
-  const int c = idx / half, i = idx % half;
+  // angle index major: [half][rows], so the rows of a tile read consecutive entries
+  const int i = idx / rows, c = idx % rows;
   const double theta = pow(base, -2.0 * (double)i / (double)hd);
   double sn, cn;
   sincos((double)c * theta, &sn, &cn);
@@ -86,7 +87,7 @@ __global__ void rope_query_kernel(Shape s, int iter, const int32_t* loops, const
   const float scale = 1.4426950408889634f / sqrtf((float)s.hd);
   const int pos = ctx_len[b];  // the query's position (its own row)
   for (int i = threadIdx.x; i < half; i += blockDim.x) {
-    const float2 c = cs[(size_t)pos * half + i];
+    const float2 c = cs[(size_t)i * s.max_ctx + pos];
     const float x1 = q[i], x2 = q[i + half];
     qrot[(size_t)b * s.d + j * s.hd + i] = (x1 * c.x - x2 * c.y) * scale;
     qrot[(size_t)b * s.d + j * s.hd + i + half] = (x2 * c.x + x1 * c.y) * scale;
@@ -302,10 +303,10 @@ __global__ void __launch_bounds__(kRThreads, 1)
     // lane's end read position 0's angles and store nothing
     tc_fence_after();
     const int half = s.hd / 2;
-    const float2* cs = p.cs + (size_t)(valid ? row : 0) * half;
+    const float2* cs = p.cs + (valid ? row : 0);  // entry i of this row at cs[i * max_ctx]
     const float sr = (s.fmt == TL_H_INT8_TOKEN && valid) ? reinterpret_cast<const float*>(p.scales)[grow] : 1.0f;
     for (int h = hf; h < NP / s.hd; h += 2) {  // the two warps of a lane quarter take alternate heads
-      float acc = 0.0f;
+      float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // four chains, summed in a fixed order
       for (int i0 = 0; i0 < half; i0 += 16) {
         uint32_t k1[16], k2[16];
         tmem_ld16(tbase + lane_off + h * s.hd + i0, k1);
@@ -313,15 +314,15 @@ __global__ void __launch_bounds__(kRThreads, 1)
         tmem_ld_wait();
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float2 c = cs[i0 + i];
+          const float2 c = cs[(size_t)(i0 + i) * s.max_ctx];
           const float a1 = __uint_as_float(k1[i]), a2 = __uint_as_float(k2[i]);
           const float r1 = a1 * c.x - a2 * c.y, r2 = a2 * c.x + a1 * c.y;
-          acc = fmaf(qs[h * s.hd + i0 + i], r1, acc);
-          acc = fmaf(qs[h * s.hd + half + i0 + i], r2, acc);
+          acc[i & 3] = fmaf(qs[h * s.hd + i0 + i], r1, acc[i & 3]);
+          acc[i & 3] = fmaf(qs[h * s.hd + half + i0 + i], r2, acc[i & 3]);
         }
       }
       const int j = (cb * NP) / s.hd + h;
-      if (valid) p.scores[((size_t)b * s.max_ctx + row) * kMaxHeads + j] = acc * sr;
+      if (valid) p.scores[((size_t)b * s.max_ctx + row) * kMaxHeads + j] = ((acc[0] + acc[1]) + (acc[2] + acc[3])) * sr;
     }
   }
 

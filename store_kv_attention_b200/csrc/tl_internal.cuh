@@ -227,7 +227,7 @@ size_t oproj_smem_bytes(const Shape& s, int n_lanes, int s_max);
 bool make_tmap_f16(void* tmap, const void* base, uint64_t rows, uint64_t cols, uint64_t pitch_elems,
                    uint32_t box_cols, uint32_t box_rows);
 cudaError_t launch_stream(const DecodeArgs& a, cudaStream_t st);
-// RoPE variant (k_rope.cu): cos / sin table [max_ctx][hd/2], rotated queries [n_lanes][d] and the
+// RoPE variant (k_rope.cu): cos / sin table [hd/2][max_ctx] (angle index major), rotated queries [n_lanes][d] and the
 // scores [n_lanes][max_ctx][16] the streaming kernel then takes (DecodeArgs::scores).
 cudaError_t launch_rope_scores(const DecodeArgs& a, float rope_base, float2* cs, float* qrot, float* scores,
                                cudaStream_t st);
