@@ -23,9 +23,9 @@
 //   softmax:    S -> P (fp16 hi / lo), lazy rescale of U^T
 //   P.V pass:   for each unit, rebuild again -> hi / lo into shared memory (MN-major) ->
 //               4 x 8 SS MMAs (h hi / lo times P hi / lo) into U^T
-// The passes run one after the other in all eight warps (no warp specialisation): warps w and
-// w + 4 own the same 32 rows (TMEM lane quarter w) and rebuild alternate 32-value chunks of each
-// unit; the softmax and the epilogue run in warps 0-3.  The delta cache reads (1 + iter) rows
+// The passes run one after the other in all sixteen warps (no warp specialisation): warps w,
+// w + 4, w + 8 and w + 12 own the same 32 rows (TMEM lane quarter w) and rebuild one 32-value
+// chunk of each unit each; the softmax and the epilogue run in warps 0-3.  The delta cache reads (1 + iter) rows
 // per position, and this kernel is written for clarity of the rebuild first.  Every wait is bounded; on expiry the kernel records a timeout in the status
 // word, waits (bounded) for its MMAs in flight, frees its TMEM and returns.
 #include <math_constants.h>
@@ -39,7 +39,7 @@ namespace {
 
 using namespace ptx;
 
-constexpr int kDSThreads = 256;                 // eight warps: two per TMEM lane quarter (32 rows)
+constexpr int kDSThreads = 512;                 // sixteen warps: four per TMEM lane quarter (32 rows)
 constexpr int kStageBytes = 128 * 256;          // one unit of one part, 128 rows x 128 fp16, MN-major
 constexpr long long kDWait = 4000000000ll;      // ~2 s of SM clocks
 
@@ -89,29 +89,19 @@ __device__ __forceinline__ void rebuild32(const DeltaStreamParams& p, size_t row
   }
   const size_t level_rows = (size_t)s.max_lanes * s.max_ctx;
   const int head = k0 / s.hd;
-  // levels four at a time: their loads are issued together, then added in level order
-  for (int l0 = 1; l0 <= p.iter; l0 += 4) {
-    uint4 cw[4][2];
-    float sc[4];
+  // one level per trip, added in level order: with sixteen warps a thread has 128 registers, and
+  // batching the loads of two or four levels spilled and measured slower
+  for (int l = 1; l <= p.iter; ++l) {
+    const size_t lr = (size_t)(l - 1) * level_rows + row;
+    const float sc = __half2float(p.scales[lr * s.H + head]);
+    const uint4* c = reinterpret_cast<const uint4*>(p.deltas + lr * s.d + k0);
+    const uint4 cw[2] = {__ldg(c), __ldg(c + 1)};
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
-      if (l0 + j <= p.iter) {
-        const size_t lr = (size_t)(l0 + j - 1) * level_rows + row;
-        sc[j] = __half2float(p.scales[lr * s.H + head]);
-        const uint4* c = reinterpret_cast<const uint4*>(p.deltas + lr * s.d + k0);
-        cw[j][0] = __ldg(c);
-        cw[j][1] = __ldg(c + 1);
-      }
+    for (int v = 0; v < 2; ++v) {
+      const int8_t* bv = reinterpret_cast<const int8_t*>(&cw[v]);
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
-      if (l0 + j <= p.iter) {
-#pragma unroll
-        for (int v = 0; v < 2; ++v) {
-          const int8_t* b = reinterpret_cast<const int8_t*>(&cw[j][v]);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) acc[16 * v + i] = __fadd_rn(acc[16 * v + i], __fmul_rn((float)b[i], sc[j]));
-        }
-      }
+      for (int i = 0; i < 16; ++i) acc[16 * v + i] = __fadd_rn(acc[16 * v + i], __fmul_rn((float)bv[i], sc));
+    }
   }
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
@@ -160,12 +150,16 @@ __global__ void __launch_bounds__(kDSThreads, 1) delta_stream_kernel(const Delta
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
   __shared__ float red[4][16];
+  __shared__ float m_sh[16];       // running maximum per head (the same for every row)
+  __shared__ float l_sh[16][128];  // running sum per head and tile row
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int quarter = warp & 3, grp = warp >> 2;  // grp 0 also runs the softmax and the epilogue
   const int r = quarter * 32 + lane;              // this thread's row of a tile = its TMEM lane
   const int xr = r & 7;
   const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+  for (int i = threadIdx.x; i < 16 * 128; i += kDSThreads) l_sh[i >> 7][i & 127] = 0.0f;
+  if (threadIdx.x < 16) m_sh[threadIdx.x] = -CUDART_INF_F;
   if (threadIdx.x == 0) {
     mbar_init(&bar_q, 1);
     mbar_init(&bar_mma, 1);
@@ -211,13 +205,6 @@ __global__ void __launch_bounds__(kDSThreads, 1) delta_stream_kernel(const Delta
   const uint64_t p_desc = sdesc_sw128(smem_addr(ps), 16, 1024);
   const size_t row_base = (size_t)b * s.max_ctx;
 
-  float m_used[16], l_part[16];
-#pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    m_used[j] = -CUDART_INF_F;
-    l_part[j] = 0.0f;
-  }
-
   for (int t = 0; t < n_tiles && ok; ++t) {
     const int row0 = r_begin + t * 128;
     const bool valid = row0 + r < r_end;
@@ -225,10 +212,9 @@ __global__ void __launch_bounds__(kDSThreads, 1) delta_stream_kernel(const Delta
 
     // ---------------------------------------------------------------- score pass
     for (int u = 0; u < n_units && ok; ++u) {
-      uint32_t hi[16], lo[16];
-#pragma unroll
-      for (int qq = 0; qq < 2; ++qq) {
-        const int q = grp + 2 * qq;  // this warp's 32-value chunks of the unit
+      {
+        const int q = grp;  // this warp's 32-value chunk of the unit
+        uint32_t hi[16], lo[16];
         rebuild32(p, row, valid, u * 128 + q * 32, hi, lo);
         tmem_st16(tbase + lane_off + kColHi + q * 16, hi);
         tmem_st16(tbase + lane_off + kColLo + q * 16, lo);
@@ -259,8 +245,8 @@ __global__ void __launch_bounds__(kDSThreads, 1) delta_stream_kernel(const Delta
     if (!ok) break;
 
     // ---------------------------------------------------------------- online softmax of the tile
-    // warps 0-3 (one thread per row); warps 4-7 only pass the block barriers
-    float sc[16], alpha[16];
+    // warps 0-3 (one thread per row); warps 4-15 only pass the block barriers
+    float sc[16], alpha[16], m_new[16];
     bool rescale = false;
     if (grp == 0) {
       uint32_t v[16];
@@ -286,24 +272,29 @@ __global__ void __launch_bounds__(kDSThreads, 1) delta_stream_kernel(const Delta
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         const float tm = fmaxf(fmaxf(red[0][j], red[1][j]), fmaxf(red[2][j], red[3][j]));
+        const float mu = m_sh[j];
         alpha[j] = 1.0f;
-        if (tm > m_used[j] + 8.0f) {  // lazy rescale: P stays below 2^8 otherwise
-          if (m_used[j] != -CUDART_INF_F) {
-            alpha[j] = exp2f(m_used[j] - tm);
+        m_new[j] = mu;
+        if (tm > mu + 8.0f) {  // lazy rescale: P stays below 2^8 otherwise
+          if (mu != -CUDART_INF_F) {
+            alpha[j] = exp2f(mu - tm);
             rescale = true;
           }
-          m_used[j] = tm;
+          m_new[j] = tm;
         }
       }
     }
-    __syncthreads();  // red is reused below
+    __syncthreads();  // red is reused and m_sh rewritten below
     if (grp == 0) {
       float pr[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        pr[j] = (valid && j < s.H) ? exp2f(sc[j] - m_used[j]) : 0.0f;
-        l_part[j] = l_part[j] * alpha[j] + pr[j];
+        pr[j] = (valid && j < s.H) ? exp2f(sc[j] - m_new[j]) : 0.0f;
+        l_sh[j][r] = l_sh[j][r] * alpha[j] + pr[j];
       }
+      if (threadIdx.x == 0)
+#pragma unroll
+        for (int j = 0; j < 16; ++j) m_sh[j] = m_new[j];
       if (__any_sync(0xffffffffu, rescale) && t > 0) {
         // the P.V MMAs of the earlier tiles are complete (each was waited for)
         for (int u = 0; u < n_units; ++u) {
@@ -326,9 +317,8 @@ __global__ void __launch_bounds__(kDSThreads, 1) delta_stream_kernel(const Delta
 
     // ---------------------------------------------------------------- P.V pass
     for (int u = 0; u < n_units && ok; ++u) {
-#pragma unroll
-      for (int qq = 0; qq < 2; ++qq) {
-        const int q = grp + 2 * qq;  // this warp's 32-value chunks of the unit
+      {
+        const int q = grp;  // this warp's 32-value chunk of the unit
         uint32_t hi[16], lo[16];
         rebuild32(p, row, valid, u * 128 + q * 32, hi, lo);
         // values q*32 .. q*32+31 of the unit: atom-column q / 2, 16-byte vectors 4 (q & 1) .. + 3
@@ -384,7 +374,7 @@ __global__ void __launch_bounds__(kDSThreads, 1) delta_stream_kernel(const Delta
     }
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
-      float v = l_part[j];
+      float v = l_sh[j][r];
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
       if (lane == 0) red[warp][j] = v;
@@ -394,11 +384,7 @@ __global__ void __launch_bounds__(kDSThreads, 1) delta_stream_kernel(const Delta
   if (ok && threadIdx.x < 16) {
     const size_t part = (size_t)b * p.s_max + split;
     const int j = threadIdx.x;
-    float m = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i)
-      if (i == j) m = m_used[i];
-    p.ml[(part * kMaxHeads + j) * 2 + 0] = m;
+    p.ml[(part * kMaxHeads + j) * 2 + 0] = m_sh[j];
     p.ml[(part * kMaxHeads + j) * 2 + 1] = red[0][j] + red[1][j] + red[2][j] + red[3][j];
   }
 
