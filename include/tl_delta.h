@@ -8,8 +8,8 @@
  * an INT8 delta with one fp16 scale per head.  The state of iteration i is rebuilt as
  *     h^i = anchor + sum_{j=1..i} scale_j[head] * code_j        (FP32 prefix sum)
  * This header covers the cache layout, the writer, and a decode over the cache: the new
- * token's state is written, the attended rows are rebuilt, and the store-h FP16 decode
- * kernels run over the rebuilt rows (tl_delta_attn_decode).
+ * token's state is written, then the store-h decode runs with the FP32 prefix sum as its
+ * dequantisation stage, inside the kernel that attends the rows (tl_delta_attn_decode).
  *
  * Conventions are those of tl_storeh.h: caller-owned device memory, asynchronous on a
  * stream, host-side validation before any launch (a non-TL_OK return enqueues nothing,
@@ -73,7 +73,9 @@ TL_API tl_status tl_delta_append(const tl_delta_desc* desc, tl_delta_cache cache
                                  tl_stream_t stream);
 
 /* Workspace bytes of tl_delta_attn_decode for n_lanes lanes: the store-h decode workspace
- * (status word first) plus n_lanes x max_ctx x d_model fp16 rows for the rebuilt states.
+ * (status word first) in the layout of 256-row splits with hi and lo absorbed-query images,
+ * plus two int32 [n_lanes] arrays of per-lane loop flags.  The rebuilt states are never
+ * stored.
  * Errors: the desc errors, TL_ERR_INVALID_ARG (n_lanes <= 0, NULL), TL_ERR_CAPACITY
  * (n_lanes > max_lanes), TL_ERR_UNSUPPORTED (n_lanes > 64, n_heads > 16, max_ctx > 65536). */
 TL_API tl_status tl_delta_workspace_bytes(const tl_delta_desc* desc, int32_t n_lanes, size_t* bytes);
@@ -88,15 +90,17 @@ TL_API tl_status tl_delta_workspace_bytes(const tl_delta_desc* desc, int32_t n_l
  * skipped and recorded; tl_storeh_poll_status on this workspace reports it):
  *   1. h_new is written as the state of iteration iter at position ctx_len[b], exactly as
  *      tl_delta_append does;
- *   2. h^iter of positions 0..ctx_len[b] is rebuilt (FP32 prefix sum, rounded to fp16);
- *   3. q = W_q h_new attends those rows with K = W_k h, V = W_v h (the store-h decode);
- *   4. with a residual, the safety check of iteration iter runs as in tl_residual_norm_check.
+ *   2. q = W_q h_new attends positions 0..ctx_len[b] with K = W_k h, V = W_v h (the
+ *      store-h decode), where each attended row h^iter is rebuilt inside the streaming
+ *      kernel by the FP32 prefix sum above and enters the tensor cores as an fp16 hi + lo
+ *      pair per value (about 22 significant bits), the absorbed query and the softmax
+ *      weights likewise;
+ *   3. with a residual, the safety check of iteration iter runs as in tl_residual_norm_check.
  * Other lanes' out rows are left unwritten.  Errors: as tl_storeh_attn_decode, plus the
- * desc errors above.
- * Known accuracy gap of this composition: step 2 rounds the FP32 rebuild to fp16 before
- * attention, an error the exact rebuild does not have.  At d_model 256 the outputs meet
- * the store-h bar (max-abs 2e-3, relative L2 1e-3); at d_model 1024 one output element was
- * measured at max-abs 2.22e-3, above that bar, and d_model 2048 has not been run. */
+ * desc errors above, and TL_ERR_UNSUPPORTED for n_heads > 16.
+ * Accuracy: against the FP64 rebuild and attention, outputs meet the store-h bar (max-abs
+ * 2e-3, relative L2 1e-3) in the seeded GPU tests at d_model 256, 768, 1024 (3 and 8 loop
+ * iterations), 1280 and 2048. */
 TL_API tl_status tl_delta_attn_decode(const tl_delta_desc* desc, tl_delta_cache cache, int32_t iter,
                                       const int32_t* loops, const int32_t* ctx_len, const void* h_new,
                                       const void* W_q, const void* W_k, const void* W_v, float* out,
