@@ -76,10 +76,14 @@ __device__ __forceinline__ void rebuild32(const DeltaStreamParams& p, size_t row
     return;
   }
   const uint4* a = reinterpret_cast<const uint4*>(p.anchor + row * s.d + k0);
+  uint4 aw[4];
+#pragma unroll
+  for (int v = 0; v < 4; ++v) aw[v] = __ldg(a + v);
+  const size_t level_rows = (size_t)s.max_lanes * s.max_ctx;
+  const int head = k0 / s.hd;
 #pragma unroll
   for (int v = 0; v < 4; ++v) {
-    const uint4 w = __ldg(a + v);
-    const __half2* h2 = reinterpret_cast<const __half2*>(&w);
+    const __half2* h2 = reinterpret_cast<const __half2*>(&aw[v]);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const float2 f = __half22float2(h2[i]);
@@ -87,15 +91,25 @@ __device__ __forceinline__ void rebuild32(const DeltaStreamParams& p, size_t row
       acc[8 * v + 2 * i + 1] = f.y;
     }
   }
-  const size_t level_rows = (size_t)s.max_lanes * s.max_ctx;
-  const int head = k0 / s.hd;
-  // one level per trip, added in level order: with sixteen warps a thread has 128 registers, and
-  // batching the loads of two or four levels spilled and measured slower
+  uint4 n0 = make_uint4(0, 0, 0, 0), n1 = n0;
+  float nsc = 0.0f;
+  if (p.iter >= 1) {
+    nsc = __half2float(p.scales[row * s.H + head]);
+    const uint4* c = reinterpret_cast<const uint4*>(p.deltas + row * s.d + k0);
+    n0 = __ldg(c);
+    n1 = __ldg(c + 1);
+  }
+  // level l + 1's loads are issued before level l is added, in level order
   for (int l = 1; l <= p.iter; ++l) {
-    const size_t lr = (size_t)(l - 1) * level_rows + row;
-    const float sc = __half2float(p.scales[lr * s.H + head]);
-    const uint4* c = reinterpret_cast<const uint4*>(p.deltas + lr * s.d + k0);
-    const uint4 cw[2] = {__ldg(c), __ldg(c + 1)};
+    const uint4 cw[2] = {n0, n1};
+    const float sc = nsc;
+    if (l < p.iter) {
+      const size_t lr = (size_t)l * level_rows + row;
+      nsc = __half2float(p.scales[lr * s.H + head]);
+      const uint4* c = reinterpret_cast<const uint4*>(p.deltas + lr * s.d + k0);
+      n0 = __ldg(c);
+      n1 = __ldg(c + 1);
+    }
 #pragma unroll
     for (int v = 0; v < 2; ++v) {
       const int8_t* bv = reinterpret_cast<const int8_t*>(&cw[v]);
