@@ -25,9 +25,10 @@
 //               4 x 8 SS MMAs (h hi / lo times P hi / lo) into U^T
 // The passes run one after the other in all sixteen warps (no warp specialisation): warps w,
 // w + 4, w + 8 and w + 12 own the same 32 rows (TMEM lane quarter w) and rebuild one 32-value
-// chunk of each unit each; the softmax and the epilogue run in warps 0-3.  The delta cache reads (1 + iter) rows
-// per position, and this kernel is written for clarity of the rebuild first.  Every wait is bounded; on expiry the kernel records a timeout in the status
-// word, waits (bounded) for its MMAs in flight, frees its TMEM and returns.
+// chunk of each unit each; the softmax and the epilogue run in warps 0-3.  The delta cache
+// reads (1 + iter) rows per position, and this kernel is written for clarity of the rebuild
+// first.  Every wait is bounded; on expiry the kernel records a timeout in the status word,
+// waits (bounded) for its MMAs in flight, frees its TMEM and returns.
 #include <math_constants.h>
 
 #include "delta_internal.cuh"
